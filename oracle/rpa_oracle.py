@@ -1,0 +1,300 @@
+"""fp64 CPU oracle for ragged paged attention.  TEST INFRASTRUCTURE ONLY.
+
+Only the tests, ``__graft_entry__.smoke()`` and the benchmark's CPU-baseline leg may import
+this module.  It shares no code with the CUDA library and never imports it.
+
+What it computes (plain definitions, written out; no tiling, no fusion, no reordering):
+
+* ``write_kv``      -- the KV-cache scatter.  For token ``i`` of sequence ``b`` the absolute
+  position is ``past_b + i`` with ``past_b = seq_lens_k[b] - q_len_b``; the page is
+  ``block_table[b, pos // page_size]`` and the slot ``pos % page_size``.
+  ([WebGPU] Optimized PagedAttention implementation (2/n), squashed commit "Phase 1b.1":
+  ScatterKVToPagedCacheProgram index math.)
+* ``attention``     -- exact softmax attention of every query row against the keys it may
+  see, gathered through the block table.  Query ``i`` of sequence ``b`` sits at absolute
+  position ``past_b + i`` and, when causal, sees keys ``0 .. past_b + i`` (bottom-right
+  alignment: same page, commit "FlashAttention: optional seqlens_q input", which sets the
+  per-batch past length to ``total_kv_b - seqlens_q[b]``).  Query head ``hq`` reads KV head
+  ``hq // (Hq / Hkv)``.  With per-group block tables (CompactAttention: Accelerating
+  Chunked Prefill with Block-Union KV Selection, Core claim and Fig. 3) only keys whose
+  block is listed in the table of the row's KV group are visible.
+  Output ``o = sum_j softmax_j(scale * q.k_j) v_j`` and ``lse = log sum_j exp(scale*q.k_j)``
+  (natural log); a row that sees no key gets ``o = 0`` and ``lse = -inf``.
+* ``merge_partials`` -- the log-sum-exp merge of attention over disjoint key sets (the
+  split-reduce pair FlashAttentionPagedDecodeQKV / FlashAttentionPagedDecodeVxReduce of the
+  WebGPU page, "What's shipped").
+* ``build_group_tables`` -- Q-block union, then intra-group union, then the ascending list
+  of selected KV blocks per (sequence, KV group) (CompactAttention, Core claim; Fig. 3).
+
+Inputs are bf16 bit patterns (numpy ``uint16``) or torch bf16 tensors; every bf16 value is
+widened exactly to fp64 before any arithmetic.  Cache writes move the bf16 bit patterns
+unchanged.
+"""
+from __future__ import annotations
+
+import math
+from typing import Iterable, List, Optional, Sequence, Tuple
+
+import numpy as np
+
+SEQ_MAJOR = 0
+HEAD_MAJOR = 1
+
+
+# --------------------------------------------------------------------------------------
+# bf16 handling
+# --------------------------------------------------------------------------------------
+
+def bits16(x) -> np.ndarray:
+    """bf16 values as their uint16 bit patterns (a copy-free view where possible)."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            assert x.dtype == torch.bfloat16, x.dtype
+            return x.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+    except ImportError:  # pragma: no cover
+        pass
+    x = np.asarray(x)
+    assert x.dtype == np.uint16, x.dtype
+    return x
+
+
+def widen(bits: np.ndarray) -> np.ndarray:
+    """Exact bf16 -> fp64: a bf16 is the top half of an IEEE fp32."""
+    b = np.ascontiguousarray(bits, dtype=np.uint16)
+    return (b.astype(np.uint32) << np.uint32(16)).view(np.float32).astype(np.float64)
+
+
+def ints(x) -> np.ndarray:
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return x.detach().cpu().numpy().astype(np.int64)
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(x).astype(np.int64)
+
+
+# --------------------------------------------------------------------------------------
+# Batch bookkeeping
+# --------------------------------------------------------------------------------------
+
+def seq_ranges(cu_seqlens_q, seq_lens_k) -> List[Tuple[int, int, int, int]]:
+    """Per sequence: (first token, q_len, kv_len, past) with past = kv_len - q_len."""
+    cu = ints(cu_seqlens_q)
+    kv = ints(seq_lens_k)
+    out = []
+    for b in range(len(kv)):
+        t0 = int(cu[b])
+        q_len = int(cu[b + 1] - cu[b])
+        kv_len = int(kv[b])
+        out.append((t0, q_len, kv_len, kv_len - q_len))
+    return out
+
+
+def page_of(block_table: np.ndarray, layout: int, b: int, h: int, pos: np.ndarray,
+            page_size: int) -> np.ndarray:
+    """Physical page that holds absolute position ``pos`` of sequence ``b`` (KV head ``h``
+    in the head-major layout)."""
+    if layout == SEQ_MAJOR:
+        return block_table[b, pos // page_size]
+    return block_table[b, h, pos // page_size]
+
+
+# --------------------------------------------------------------------------------------
+# a2: KV write (scatter)
+# --------------------------------------------------------------------------------------
+
+def write_kv(k_pool, v_pool, k_new, v_new, block_table, cu_seqlens_q, seq_lens_k,
+             page_size: int, layout: int = SEQ_MAJOR):
+    """Return copies of the pools with every new token's K/V written into its slot."""
+    kp = bits16(k_pool).copy()
+    vp = bits16(v_pool).copy()
+    kn = bits16(k_new)
+    vn = bits16(v_new)
+    bt = ints(block_table)
+    num_kv_heads = kn.shape[1]
+    for b, (t0, q_len, kv_len, past) in enumerate(seq_ranges(cu_seqlens_q, seq_lens_k)):
+        for i in range(q_len):
+            t = t0 + i
+            pos = past + i
+            slot = pos % page_size
+            if layout == SEQ_MAJOR:
+                page = bt[b, pos // page_size]
+                kp[page, slot] = kn[t]
+                vp[page, slot] = vn[t]
+            else:
+                for h in range(num_kv_heads):
+                    page = bt[b, h, pos // page_size]
+                    kp[page, slot] = kn[t, h]
+                    vp[page, slot] = vn[t, h]
+    return kp, vp
+
+
+def logical_rows(pool, block_table, layout: int, b: int, h: int, n: int,
+                 page_size: int) -> np.ndarray:
+    """Keys (or values) ``0 .. n-1`` of sequence ``b``, KV head ``h``, gathered through the
+    block table: uint16 ``[n, D]``."""
+    p = bits16(pool)
+    bt = ints(block_table)
+    pos = np.arange(n, dtype=np.int64)
+    pages = page_of(bt, layout, b, h, pos, page_size)
+    slots = pos % page_size
+    if layout == SEQ_MAJOR:
+        return p[pages, slots, h]
+    return p[pages, slots]
+
+
+# --------------------------------------------------------------------------------------
+# a3-a5, a8: attention
+# --------------------------------------------------------------------------------------
+
+def visible_keys(pos: int, kv_len: int, causal: bool, page_size: int,
+                 selected_blocks: Optional[set]) -> np.ndarray:
+    """Indices of the keys a query at absolute position ``pos`` may attend to."""
+    hi = min(kv_len, pos + 1) if causal else kv_len
+    j = np.arange(hi, dtype=np.int64)
+    if selected_blocks is not None:
+        blocks = np.fromiter(selected_blocks, dtype=np.int64, count=len(selected_blocks))
+        j = j[np.isin(j // page_size, blocks)]
+    return j
+
+
+def attend_row(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float):
+    """Softmax attention of one fp64 query row over fp64 keys/values (rows of K, V).
+
+    Returns (o [D], lse).  With no keys: (0, -inf)."""
+    if K.shape[0] == 0:
+        return np.zeros(q.shape[0], dtype=np.float64), -math.inf
+    s = scale * (K @ q)
+    m = np.max(s)
+    w = np.exp(s - m)
+    z = np.sum(w)
+    o = (w @ V) / z
+    return o, float(m + math.log(z))
+
+
+def attention(q, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k, *, scale: float,
+              causal: bool, page_size: int, layout: int = SEQ_MAJOR, num_kv_heads: int,
+              group_table=None, group_count=None,
+              rows: Optional[Iterable[Tuple[int, int]]] = None):
+    """Attention of every (token, query head) row -- or of ``rows`` only -- against the pools
+    *as given* (call ``write_kv`` first for the fused semantics).
+
+    Returns ``(out [T, Hq, D] fp64, lse [T, Hq] fp64)``; rows not computed are NaN.
+    """
+    qb = bits16(q)
+    T, Hq, D = qb.shape
+    Hkv = int(num_kv_heads)
+    G = Hq // Hkv
+    seqs = seq_ranges(cu_seqlens_q, seq_lens_k)
+    gt = ints(group_table) if group_table is not None else None
+    gc = ints(group_count) if group_count is not None else None
+
+    out = np.full((T, Hq, D), np.nan, dtype=np.float64)
+    lse = np.full((T, Hq), np.nan, dtype=np.float64)
+
+    if rows is None:
+        wanted = None
+    else:
+        wanted = {}
+        for t, hq in rows:
+            wanted.setdefault(int(t), set()).add(int(hq))
+
+    for b, (t0, q_len, kv_len, past) in enumerate(seqs):
+        if q_len == 0:
+            continue
+        toks = range(t0, t0 + q_len)
+        if wanted is not None:
+            toks = [t for t in toks if t in wanted]
+            if not toks:
+                continue
+        for hk in range(Hkv):
+            heads = [hk * G + g for g in range(G)]
+            if wanted is not None and not any(h in wanted[t] for t in toks for h in heads):
+                continue
+            K = widen(logical_rows(k_pool, block_table, layout, b, hk, kv_len, page_size))
+            V = widen(logical_rows(v_pool, block_table, layout, b, hk, kv_len, page_size))
+            selected = None
+            if gt is not None:
+                selected = set(int(x) for x in gt[b, hk, :int(gc[b, hk])])
+            for t in toks:
+                pos = past + (t - t0)
+                idx = visible_keys(pos, kv_len, causal, page_size, selected)
+                for hq in heads:
+                    if wanted is not None and hq not in wanted[t]:
+                        continue
+                    o, l = attend_row(widen(qb[t, hq]), K[idx], V[idx], scale)
+                    out[t, hq] = o
+                    lse[t, hq] = l
+    return out, lse
+
+
+def forward(q, k_new, v_new, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k, *,
+            scale: float, causal: bool, page_size: int, layout: int = SEQ_MAJOR,
+            group_table=None, group_count=None, rows=None):
+    """The fused step: write the new tokens' K/V into the pools, then attend.
+
+    Returns ``(out, lse, k_pool_after, v_pool_after)``."""
+    kp, vp = write_kv(k_pool, v_pool, k_new, v_new, block_table, cu_seqlens_q, seq_lens_k,
+                      page_size, layout)
+    num_kv_heads = bits16(k_new).shape[1]
+    out, lse = attention(q, kp, vp, block_table, cu_seqlens_q, seq_lens_k, scale=scale,
+                         causal=causal, page_size=page_size, layout=layout,
+                         num_kv_heads=num_kv_heads, group_table=group_table,
+                         group_count=group_count, rows=rows)
+    return out, lse, kp, vp
+
+
+# --------------------------------------------------------------------------------------
+# a4: log-sum-exp merge of partial results
+# --------------------------------------------------------------------------------------
+
+def merge_partials(parts: Sequence[Tuple[np.ndarray, float]]):
+    """Combine attention results over disjoint key sets: ``M = max lse_i``,
+    ``w_i = exp(lse_i - M)``, ``o = sum w_i o_i / sum w_i``, ``lse = M + log sum w_i``."""
+    lses = np.array([p[1] for p in parts], dtype=np.float64)
+    if np.all(np.isneginf(lses)):
+        return np.zeros_like(parts[0][0]), -math.inf
+    M = np.max(lses)
+    w = np.exp(lses - M)
+    o = sum(wi * p[0] for wi, p in zip(w, parts)) / np.sum(w)
+    return o, float(M + math.log(np.sum(w)))
+
+
+# --------------------------------------------------------------------------------------
+# a7: block-union tables
+# --------------------------------------------------------------------------------------
+
+def build_group_tables(mask, num_kv_heads: int):
+    """Per-(sequence, KV group) tables of selected KV blocks.
+
+    Step 1 (Q-block union): a query head needs KV block ``kb`` if any of its query blocks
+    selects it.  Step 2 (intra-group union): a KV group needs ``kb`` if any query head of the
+    group needs it; query head ``hq`` belongs to group ``hq // (Hq / Hkv)``.  Step 3: list the
+    needed blocks in ascending order.
+
+    ``mask`` is uint8 ``[B, Hq, nqb, nkb]``.  Returns ``(table int32 [B, Hkv, nkb],
+    count int32 [B, Hkv])``; table entries past ``count`` are -1.
+    """
+    m = np.asarray(mask.numpy() if hasattr(mask, "numpy") else mask).astype(np.uint8)
+    B, Hq, nqb, nkb = m.shape
+    Hkv = int(num_kv_heads)
+    G = Hq // Hkv
+    head_union = np.zeros((B, Hq, nkb), dtype=bool)
+    for b in range(B):
+        for hq in range(Hq):
+            for qb in range(nqb):
+                head_union[b, hq] |= m[b, hq, qb] != 0
+    group_union = np.zeros((B, Hkv, nkb), dtype=bool)
+    for b in range(B):
+        for hq in range(Hq):
+            group_union[b, hq // G] |= head_union[b, hq]
+    table = np.full((B, Hkv, nkb), -1, dtype=np.int32)
+    count = np.zeros((B, Hkv), dtype=np.int32)
+    for b in range(B):
+        for g in range(Hkv):
+            sel = [kb for kb in range(nkb) if group_union[b, g, kb]]
+            table[b, g, :len(sel)] = sel
+            count[b, g] = len(sel)
+    return table, count

@@ -1,0 +1,381 @@
+"""Pins for the fp64 oracle: each test checks it against something other than itself --
+hand-derived fixtures, a library routine (torch SDPA / logsumexp), closed forms, invariants
+and brute force -- chosen so that a dropped term, a wrong sign or index, or a transposed
+operand in the oracle fails at least one of them.  CPU only."""
+import itertools
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from oracle import rpa_oracle as orc
+from ragged_paged_attention_forward_b200 import workloads as wl
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _oracle_forward(batch, **kw):
+    return orc.forward(batch.q, batch.k_new, batch.v_new, batch.k_pool, batch.v_pool,
+                       batch.block_table, batch.cu_seqlens_q, batch.seq_lens_k,
+                       scale=kw.pop("scale", batch.scale), causal=kw.pop("causal", batch.causal),
+                       page_size=batch.page_size, layout=batch.layout, **kw)
+
+
+def _f64(t):
+    return t.to(torch.float64)
+
+
+def _sdpa_row(q_row, K, V, scale):
+    """Library attention (torch SDPA, fp64, no mask) of one query row over rows K, V."""
+    o = F.scaled_dot_product_attention(q_row.view(1, 1, -1), K.unsqueeze(0), V.unsqueeze(0),
+                                       scale=scale)
+    return o.view(-1).numpy()
+
+
+# ------------------------------------------------------------------------------------
+# KV write
+# ------------------------------------------------------------------------------------
+
+def _read_golden(name):
+    rows = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                rows.append(line.split())
+    return rows
+
+
+def test_scatter_matches_hand_derived_slots():
+    P, Hkv, D = 16, 2, 8
+    kv_lens, q_lens = [19, 33], [2, 3]
+    bt = np.array([[5, 2, 9], [7, 0, 4]], dtype=np.int32)
+    cu = np.array([0, 2, 5], dtype=np.int32)
+    sentinel = np.uint16(0x7FC1)
+    kp = np.full((10, P, Hkv, D), sentinel, dtype=np.uint16)
+    vp = np.full((10, P, Hkv, D), sentinel, dtype=np.uint16)
+    T = 5
+    kn = (np.arange(T * Hkv * D, dtype=np.uint16).reshape(T, Hkv, D) + 0x3F00)
+    vn = (np.arange(T * Hkv * D, dtype=np.uint16).reshape(T, Hkv, D) + 0x4000)
+    kp2, vp2 = orc.write_kv(kp, vp, kn, vn, bt, cu, np.array(kv_lens, dtype=np.int32), P)
+    expected = {}
+    for tok, page, slot in _read_golden("scatter_tiny.txt"):
+        expected[(int(page), int(slot))] = int(tok)
+    for page in range(10):
+        for slot in range(P):
+            if (page, slot) in expected:
+                t = expected[(page, slot)]
+                assert np.array_equal(kp2[page, slot], kn[t])
+                assert np.array_equal(vp2[page, slot], vn[t])
+            else:
+                assert np.all(kp2[page, slot] == sentinel)
+                assert np.all(vp2[page, slot] == sentinel)
+
+
+@pytest.mark.parametrize("layout", [wl.SEQ_MAJOR, wl.HEAD_MAJOR])
+def test_write_then_gather_returns_logical_sequence(layout):
+    b = wl.ragged_batch([1, 17, 40, 64, 65], [1, 5, 40, 3, 2], 4, 2, 16, 16, seed=11,
+                        layout=layout)
+    kp, vp = orc.write_kv(b.k_pool, b.v_pool, b.k_new, b.v_new, b.block_table,
+                          b.cu_seqlens_q, b.seq_lens_k, b.page_size, b.layout)
+    for s, kv in enumerate(b.kv_lens()):
+        for h in range(b.num_kv_heads):
+            got_k = orc.logical_rows(kp, b.block_table, layout, s, h, kv, b.page_size)
+            got_v = orc.logical_rows(vp, b.block_table, layout, s, h, kv, b.page_size)
+            assert np.array_equal(got_k, orc.bits16(b.k_logical[s][:, h]))
+            assert np.array_equal(got_v, orc.bits16(b.v_logical[s][:, h]))
+    # bytes the write must not touch keep their poison pattern
+    before = orc.bits16(b.k_pool)
+    changed = np.any(kp != before, axis=tuple(range(1, kp.ndim)))
+    assert int(changed.sum()) <= sum(math.ceil(q / b.page_size) + 1 for q in b.q_lens()) * (
+        b.num_kv_heads if layout == wl.HEAD_MAJOR else 1)
+
+
+# ------------------------------------------------------------------------------------
+# Attention against a library routine and against closed forms
+# ------------------------------------------------------------------------------------
+
+def _sdpa_reference(batch, scale=None):
+    """Attention of each row as torch SDPA over the *logical* (unpaged) prefix of keys the
+    row may see; uses the generator's logical rows, never the pool."""
+    scale = batch.scale if scale is None else scale
+    G = batch.num_q_heads // batch.num_kv_heads
+    T, Hq, D = batch.q.shape
+    out = np.zeros((T, Hq, D))
+    cu = batch.cu_seqlens_q.tolist()
+    for s, kv in enumerate(batch.kv_lens()):
+        q_len = cu[s + 1] - cu[s]
+        past = kv - q_len
+        for i in range(q_len):
+            t = cu[s] + i
+            n = min(kv, past + i + 1) if batch.causal else kv
+            for hq in range(Hq):
+                K = _f64(batch.k_logical[s][:n, hq // G])
+                V = _f64(batch.v_logical[s][:n, hq // G])
+                out[t, hq] = _sdpa_row(_f64(batch.q[t, hq]), K, V, scale)
+    return out
+
+
+@pytest.mark.parametrize("case", ["tiny", "ragged", "mha", "noncausal"])
+def test_oracle_equals_library_attention_over_logical_prefix(case):
+    if case == "tiny":
+        b = wl.tiny()
+    elif case == "ragged":
+        b = wl.ragged_batch([5, 70, 33, 129], [5, 1, 17, 40], 8, 2, 32, 16, seed=3)
+    elif case == "mha":
+        b = wl.ragged_batch([9, 48], [3, 48], 3, 3, 16, 32, seed=4, scale=0.37)
+    else:
+        b = wl.ragged_batch([20, 35], [4, 6], 4, 1, 16, 16, seed=5, causal=False)
+    out, lse, _, _ = _oracle_forward(b)
+    ref = _sdpa_reference(b)
+    assert np.max(np.abs(out - ref)) < 1e-12
+
+
+def test_causal_prefill_without_past_equals_library_causal_mask():
+    b = wl.ragged_batch([37], [37], 2, 2, 16, 16, seed=6)
+    out, _, _, _ = _oracle_forward(b)
+    q = _f64(b.q).permute(1, 0, 2)                     # [H, T, D]
+    k = _f64(b.k_logical[0]).permute(1, 0, 2)
+    v = _f64(b.v_logical[0]).permute(1, 0, 2)
+    ref = F.scaled_dot_product_attention(q, k, v, is_causal=True, scale=b.scale)
+    assert np.max(np.abs(out - ref.permute(1, 0, 2).numpy())) < 1e-12
+
+
+def test_causal_boundary_by_perturbation():
+    """Row at absolute position p must change when key/value p changes and must not change
+    when any key/value after p changes (mixed q_len with past > 0)."""
+    b = wl.ragged_batch([30, 12], [6, 12], 2, 1, 16, 16, seed=8)
+    out, _, kp, vp = _oracle_forward(b)
+    seqs = orc.seq_ranges(b.cu_seqlens_q, b.seq_lens_k)
+    for s, (t0, q_len, kv_len, past) in enumerate(seqs):
+        for i in range(q_len):
+            p = past + i
+            for j, expect_change in ((p, True), (p + 1, False), (kv_len - 1, p == kv_len - 1)):
+                if j >= kv_len:
+                    continue
+                kp2, vp2 = kp.copy(), vp.copy()
+                page = int(b.block_table[s, j // b.page_size])
+                vp2[page, j % b.page_size] = orc.bits16(
+                    torch.full((b.num_kv_heads, b.head_dim), 3.0, dtype=torch.bfloat16))
+                o2, _ = orc.attention(b.q, kp2, vp2, b.block_table, b.cu_seqlens_q,
+                                      b.seq_lens_k, scale=b.scale, causal=True,
+                                      page_size=b.page_size, num_kv_heads=b.num_kv_heads,
+                                      rows=[(t0 + i, 0)])
+                changed = not np.array_equal(o2[t0 + i, 0], out[t0 + i, 0])
+                assert changed == expect_change, (s, i, j)
+
+
+def test_constant_values_return_that_value():
+    b = wl.ragged_batch([3, 50, 130], [3, 1, 9], 4, 2, 16, 16, seed=9)
+    c = torch.randn(2, 16, generator=torch.Generator().manual_seed(1)).to(torch.bfloat16)
+    b.v_new[:] = c
+    vp = b.v_pool.clone()
+    used = ~torch.isnan(vp.float())
+    vp[used] = c.unsqueeze(0).unsqueeze(0).expand_as(vp)[used]
+    b.v_pool = vp
+    out, _, _, _ = _oracle_forward(b)
+    G = 2
+    expect = _f64(c)[torch.arange(4) // G].numpy()
+    for t in range(b.num_tokens):
+        assert np.max(np.abs(out[t] - expect)) <= 4e-16 * np.max(np.abs(expect)) * 10
+
+
+def test_single_visible_key_gets_weight_one():
+    # kv_len 1 decode, and row 0 of a prefill without past
+    b = wl.ragged_batch([1, 7], [1, 7], 2, 2, 16, 16, seed=10)
+    out, lse, _, _ = _oracle_forward(b)
+    for t, s in ((0, 0), (1, 1)):
+        for hq in range(2):
+            v0 = orc.widen(orc.bits16(b.v_logical[s][0, hq]))
+            k0 = orc.widen(orc.bits16(b.k_logical[s][0, hq]))
+            assert np.array_equal(out[t, hq], v0)
+            q = orc.widen(orc.bits16(b.q[t, hq]))
+            assert lse[t, hq] == pytest.approx(b.scale * float(q @ k0), abs=1e-14)
+
+
+def test_zero_scale_gives_mean_and_log_count():
+    b = wl.ragged_batch([10, 64], [4, 2], 2, 1, 16, 16, seed=12)
+    out, lse, _, _ = _oracle_forward(b, scale=0.0)
+    seqs = orc.seq_ranges(b.cu_seqlens_q, b.seq_lens_k)
+    for s, (t0, q_len, kv_len, past) in enumerate(seqs):
+        for i in range(q_len):
+            n = past + i + 1
+            mean = _f64(b.v_logical[s][:n, 0]).mean(0).numpy()
+            for hq in range(2):
+                assert np.max(np.abs(out[t0 + i, hq] - mean)) < 1e-14
+                assert lse[t0 + i, hq] == pytest.approx(math.log(n), abs=1e-14)
+
+
+def test_one_dominant_key_closed_form():
+    """All keys zero except key m = a*e_0: o = (e^s v_m + sum_{j!=m} v_j) / (e^s + n - 1)
+    with s = scale * a * q_0."""
+    b = wl.ragged_batch([40], [1], 1, 1, 16, 16, seed=13, causal=False)
+    m, a = 17, 4.0
+    kp = torch.zeros_like(b.k_pool)
+    page = int(b.block_table[0, m // 16])
+    kp[page, m % 16, 0, 0] = a
+    b.k_pool = kp
+    b.k_new = torch.zeros_like(b.k_new)
+    out, lse, _, vp = _oracle_forward(b)
+    q0 = float(_f64(b.q[0, 0, 0]))
+    s = b.scale * a * q0
+    V = orc.widen(orc.logical_rows(vp, b.block_table, 0, 0, 0, 40, 16))
+    expect = (math.exp(s) * V[m] + V.sum(0) - V[m]) / (math.exp(s) + 39)
+    assert np.max(np.abs(out[0, 0] - expect)) < 1e-13
+    assert lse[0, 0] == pytest.approx(math.log(math.exp(s) + 39), abs=1e-13)
+
+
+def test_lse_matches_library_logsumexp():
+    b = wl.ragged_batch([33, 8], [5, 8], 4, 2, 16, 16, seed=14)
+    _, lse, kp, _ = _oracle_forward(b)
+    seqs = orc.seq_ranges(b.cu_seqlens_q, b.seq_lens_k)
+    for s, (t0, q_len, kv_len, past) in enumerate(seqs):
+        for i in range(q_len):
+            for hq in range(4):
+                K = _f64(b.k_logical[s][:past + i + 1, hq // 2])
+                ref = torch.logsumexp(b.scale * (K @ _f64(b.q[t0 + i, hq])), 0).item()
+                assert lse[t0 + i, hq] == pytest.approx(ref, abs=1e-12)
+
+
+def test_gqa_equals_mha_with_replicated_kv_heads():
+    b = wl.ragged_batch([21, 50], [3, 50], 8, 2, 16, 16, seed=15)
+    G = 4
+    mha = wl.ragged_batch([21, 50], [3, 50], 8, 8, 16, 16, seed=15)
+    mha.q = b.q
+    mha.k_new = b.k_new.repeat_interleave(G, dim=1)
+    mha.v_new = b.v_new.repeat_interleave(G, dim=1)
+    mha.block_table = b.block_table
+    mha.k_pool = b.k_pool.repeat_interleave(G, dim=2)
+    mha.v_pool = b.v_pool.repeat_interleave(G, dim=2)
+    o1, l1, _, _ = _oracle_forward(b)
+    o2, l2, _, _ = _oracle_forward(mha)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_page_permutation_invariance_is_bit_exact():
+    b = wl.ragged_batch([17, 64, 130, 5], [1, 1, 5, 5], 4, 2, 32, 16, seed=16)
+    b2 = wl.permute_pages(b, seed=99)
+    assert not torch.equal(b.block_table, b2.block_table)
+    o1, l1, _, _ = _oracle_forward(b)
+    o2, l2, _, _ = _oracle_forward(b2)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_head_major_equals_seq_major_bit_exact():
+    b = wl.ragged_batch([17, 64, 130], [1, 30, 5], 4, 2, 32, 16, seed=17)
+    hm = wl.to_head_major(b)
+    o1, l1, kp, _ = _oracle_forward(b)
+    o2, l2, kph, _ = _oracle_forward(hm)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_split_merge_equals_unsplit():
+    g = np.random.default_rng(0)
+    b = wl.ragged_batch([300], [1], 1, 1, 64, 16, seed=18)
+    _, _, kp, vp = _oracle_forward(b)
+    K = orc.widen(orc.logical_rows(kp, b.block_table, 0, 0, 0, 300, 16))
+    V = orc.widen(orc.logical_rows(vp, b.block_table, 0, 0, 0, 300, 16))
+    q = orc.widen(orc.bits16(b.q[0, 0]))
+    whole = orc.attend_row(q, K, V, b.scale)
+    for cuts in ([150], [16, 64, 200], sorted(g.choice(np.arange(1, 300), 9, replace=False))):
+        edges = [0] + list(cuts) + [300]
+        parts = [orc.attend_row(q, K[a:c], V[a:c], b.scale) for a, c in zip(edges, edges[1:])]
+        parts.append(orc.attend_row(q, K[:0], V[:0], b.scale))   # an empty split
+        o, l = orc.merge_partials(parts)
+        assert np.max(np.abs(o - whole[0])) < 1e-12
+        assert l == pytest.approx(whole[1], abs=1e-12)
+
+
+# ------------------------------------------------------------------------------------
+# Block-union tables
+# ------------------------------------------------------------------------------------
+
+def test_group_tables_hand_derived_fixture():
+    rows = _read_golden("group_tables_tiny.txt")
+    mask = np.zeros((1, 4, 2, 5), dtype=np.uint8)
+    expect = {}
+    for r in rows:
+        if r[0] == "mask":
+            mask[0, int(r[1]), int(r[2])] = [int(x) for x in r[3:]]
+        else:
+            expect[int(r[1])] = (int(r[2]), [int(x) for x in r[3:]])
+    table, count = orc.build_group_tables(mask, 2)
+    for g, (n, entries) in expect.items():
+        assert count[0, g] == n
+        assert table[0, g].tolist() == entries
+
+
+@pytest.mark.parametrize("Hq,Hkv,nqb,nkb", [(4, 2, 2, 2), (2, 1, 2, 3), (4, 1, 1, 4)])
+def test_group_tables_exhaustive(Hq, Hkv, nqb, nkb):
+    """Every mask of the shape: a block is listed for a group iff some query head of the
+    group selects it in some query block (complete and minimal); ascending, no duplicates."""
+    G = Hq // Hkv
+    nbits = Hq * nqb * nkb
+    bits = ((np.arange(2 ** nbits)[:, None] >> np.arange(nbits)) & 1).astype(np.uint8)
+    for code in range(2 ** nbits):
+        mask = bits[code].reshape(1, Hq, nqb, nkb)
+        table, count = orc.build_group_tables(mask, Hkv)
+        for g in range(Hkv):
+            need = [kb for kb in range(nkb)
+                    if any(mask[0, hq, qb, kb] for hq in range(g * G, (g + 1) * G)
+                           for qb in range(nqb))]
+            n = int(count[0, g])
+            assert table[0, g, :n].tolist() == need
+            assert all(x == -1 for x in table[0, g, n:])
+
+
+def test_sparse_all_ones_equals_dense_and_truncation():
+    P = 16
+    b = wl.ragged_batch([200], [40], 4, 2, 16, P, seed=19, layout=wl.HEAD_MAJOR)
+    nkb = math.ceil(200 / P)
+    dense, dlse, _, _ = _oracle_forward(b)
+    ones = np.ones((1, 4, 3, nkb), dtype=np.uint8)
+    table, count = orc.build_group_tables(ones, 2)
+    o1, l1, _, _ = _oracle_forward(b, group_table=table, group_count=count)
+    assert np.array_equal(o1, dense) and np.array_equal(l1, dlse)
+    # keep blocks 0..c only: equals attention over the prefix min(p+1, (c+1)*P)
+    c = 7
+    trunc = np.zeros_like(ones)
+    trunc[..., :c + 1] = 1
+    table, count = orc.build_group_tables(trunc, 2)
+    o2, _, _, _ = _oracle_forward(b, group_table=table, group_count=count)
+    past = 160
+    for i in range(40):
+        n = min(past + i + 1, (c + 1) * P)
+        for hq in range(4):
+            K = _f64(b.k_logical[0][:n, hq // 2])
+            V = _f64(b.v_logical[0][:n, hq // 2])
+            ref = _sdpa_row(_f64(b.q[i, hq]), K, V, b.scale)
+            assert np.max(np.abs(o2[i, hq] - ref)) < 1e-12
+
+
+def test_sparse_row_with_no_visible_block_is_zero():
+    P = 16
+    b = wl.ragged_batch([64], [64], 2, 1, 16, P, seed=20, layout=wl.HEAD_MAJOR)
+    mask = np.zeros((1, 2, 1, 4), dtype=np.uint8)
+    mask[..., 3] = 1            # only the last block: rows before position 48 see nothing
+    table, count = orc.build_group_tables(mask, 1)
+    out, lse, _, _ = _oracle_forward(b, group_table=table, group_count=count)
+    assert np.all(out[:48] == 0) and np.all(np.isneginf(lse[:48]))
+    assert np.all(np.isfinite(lse[48:]))
+
+
+def test_tolerance_is_reachable_with_bf16_inputs_and_fp32_accumulation():
+    """An fp32-accumulating computation that rounds P to bf16 stays well inside
+    max-abs 2e-2 / mean-abs 2e-3 of the fp64 oracle on a decode-shaped batch."""
+    b = wl.ragged_batch([700, 1500, 2300], [1, 1, 1], 32, 8, 128, 16, seed=21)
+    out, _, _, _ = _oracle_forward(b)
+    err = []
+    for s, kv in enumerate(b.kv_lens()):
+        for hq in range(32):
+            K = b.k_logical[s][:, hq // 4].float()
+            V = b.v_logical[s][:, hq // 4].float()
+            sc = (K @ b.q[s, hq].float()) * b.scale
+            p = torch.exp(sc - sc.max())
+            o = (p.to(torch.bfloat16).float() @ V) / p.sum()
+            err.append(np.abs(o.to(torch.bfloat16).double().numpy() - out[s, hq]))
+    err = np.concatenate(err)
+    assert err.max() < 2e-2 / 4 and err.mean() < 2e-3 / 4
