@@ -1,0 +1,221 @@
+/*
+ * rpa.h -- ragged paged attention for NVIDIA B200 (sm_100a): the C ABI of librpa.so.
+ *
+ * One call attends a packed, variable-length batch of query tokens from many sequences
+ * (pure decode, pure prefill, or a mix) against a KV cache held in fixed-size pages that
+ * each sequence reaches through a block table, and writes the new tokens' K/V into their
+ * cache slots first.  The method is the one of "Ragged Paged Attention: A High-Performance
+ * and Flexible LLM Inference Kernel for TPU" (Key ideas: ragged tiling over paged KV, the
+ * cache write fused with attention, specialised decode / prefill / mixed kernels); the
+ * operator's inputs and conventions follow "[WebGPU] Optimized PagedAttention
+ * implementation (2/n)" (packed varlen Q with cumulative_seqlens_q, seqlens_k, block_table,
+ * a paged cache of shape (num_blocks, block_size, kv_num_heads, head_size), in-place cache,
+ * token_count == 0 is a no-op); the per-group block tables and the KV-head-major layout
+ * follow "CompactAttention: Accelerating Chunked Prefill with Block-Union KV Selection"
+ * (Core claim; Fig. 3; Fig. 4).
+ *
+ * Notation: B sequences, T = cu_seqlens_q[B] query tokens, Hq query heads, Hkv KV heads
+ * (Hq % Hkv == 0, G = Hq / Hkv, query head hq reads KV head hq / G), head dim D, page size P.
+ * q_len_b = cu_seqlens_q[b+1] - cu_seqlens_q[b]; kv_len_b = seq_lens_k[b] is the context
+ * length INCLUDING the q_len_b new tokens, which occupy positions past_b .. kv_len_b - 1
+ * with past_b = kv_len_b - q_len_b.  Query i of sequence b sits at position past_b + i and,
+ * when causal, sees keys 0 .. past_b + i.
+ *
+ * Memory: every device buffer, the workspace and the stream belong to the caller.  All
+ * bf16 tensors are dense row-major with the shapes given; every device pointer must be
+ * 16-byte aligned.  Calls are asynchronous on the given stream (a cudaStream_t passed as
+ * void*; NULL = the legacy default stream); argument errors are detected on the host,
+ * returned at once, and nothing is launched.  Functions are thread-safe except that a
+ * plan must not be used by two threads at once.
+ */
+#ifndef RPA_H
+#define RPA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define RPA_API __attribute__((visibility("default")))
+#else
+#define RPA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum rpa_status {
+  RPA_OK = 0,
+  RPA_ERR_INVALID_ARG = -1,          /* null/misaligned pointer, inconsistent arguments   */
+  RPA_ERR_UNSUPPORTED = -2,          /* a shape or mode this build does not implement     */
+  RPA_ERR_SHAPE = -3,                /* lengths that contradict each other                */
+  RPA_ERR_WORKSPACE_TOO_SMALL = -4,  /* workspace smaller than rpa_plan reported          */
+  RPA_ERR_CUDA = -5,                 /* a CUDA runtime call failed (see rpa_last_error)   */
+  RPA_ERR_DEVICE_CHECK = -6          /* a kernel gave up a bounded wait (rpa_device_error)*/
+} rpa_status;
+
+typedef enum rpa_layout {
+  /* pool [num_pages, P, Hkv, D]; block_table [B, max_blocks_per_seq]                     */
+  RPA_LAYOUT_SEQ_MAJOR = 0,
+  /* pool [num_pages, P, D], one page per (sequence, KV head, block);
+     block_table [B, Hkv, max_blocks_per_seq] (CompactAttention, Fig. 4)                   */
+  RPA_LAYOUT_HEAD_MAJOR = 1
+} rpa_layout;
+
+typedef enum rpa_batch_class {
+  RPA_CLASS_AUTO = 0,
+  RPA_CLASS_DECODE = 1,   /* every sequence has q_len <= 1                                 */
+  RPA_CLASS_PREFILL = 2,  /* every non-empty sequence has q_len >= 32                      */
+  RPA_CLASS_MIXED = 3     /* anything else                                                 */
+} rpa_batch_class;
+
+typedef struct rpa_shape {
+  int32_t num_seqs;            /* B  >= 0                                                  */
+  int32_t num_tokens;          /* T  == cu_seqlens_q[B]                                    */
+  int32_t num_q_heads;         /* Hq                                                       */
+  int32_t num_kv_heads;        /* Hkv, Hq % Hkv == 0                                       */
+  int32_t head_dim;            /* D in {64, 128}                                           */
+  int32_t page_size;           /* P, power of two, 16 <= P <= 256                          */
+  int32_t num_pages;           /* pages in each of the K and V pools                       */
+  int32_t max_blocks_per_seq;  /* last dimension of block_table (and of group_table)       */
+  int32_t layout;              /* rpa_layout                                               */
+  int32_t causal;              /* 1 = causal (bottom-right aligned), 0 = all kv_len keys   */
+} rpa_shape;
+
+typedef struct rpa_plan_options {
+  int32_t force_class;         /* rpa_batch_class; AUTO lets the planner choose            */
+  int32_t decode_split_keys;   /* keys per decode split, multiple of 64; 0 = automatic     */
+  int32_t sparse;              /* 1: rpa_forward will be given group tables                */
+  int32_t reserved[5];         /* must be zero                                             */
+} rpa_plan_options;
+
+typedef struct rpa_plan_info {
+  int32_t batch_class;         /* rpa_batch_class chosen                                   */
+  int32_t num_decode_items;    /* (sequence, key split) items of the decode kernel         */
+  int32_t num_prefill_tiles;   /* (sequence, 128-query tile) items of the prefill kernel   */
+  int32_t num_merge_rows;      /* query tokens whose decode splits need the LSE merge      */
+  int32_t launches_forward;    /* kernels rpa_forward launches (KV write included)         */
+  int32_t launches_write;      /* kernels rpa_write_kv launches                            */
+  int32_t decode_split_keys;   /* split size used                                          */
+  int32_t reserved;
+  size_t workspace_bytes;      /* device workspace rpa_forward needs                       */
+} rpa_plan_info;
+
+typedef struct rpa_plan_s* rpa_plan_t;
+
+/*
+ * rpa_plan -- validate a batch and build its work lists on the host (the planner that
+ * picks decode, prefill or mixed kernels: "Ragged Paged Attention ..." Key ideas,
+ * distribution-aware compilation; the decode/prefill threshold q_len < 32 of the WebGPU
+ * page, "Correctness invariants").
+ *
+ *   shape            host struct, read during the call only.
+ *   cu_seqlens_q     HOST int32 [B+1], non-decreasing, cu[0] == 0, cu[B] == T.
+ *   seq_lens_k       HOST int32 [B], q_len_b <= kv_len_b,
+ *                    ceil(kv_len_b / P) <= max_blocks_per_seq.
+ *   opts             optional (NULL = defaults).
+ *   out_plan         receives a plan that owns host memory only; free with
+ *                    rpa_plan_destroy.  The plan is valid for device copies of
+ *                    cu_seqlens_q / seq_lens_k holding the same values.
+ *   workspace_bytes  optional; receives the device workspace size rpa_forward needs
+ *                    (256-byte aligned buffer supplied by the caller).
+ * Returns RPA_OK, RPA_ERR_INVALID_ARG, RPA_ERR_SHAPE or RPA_ERR_UNSUPPORTED (head_dim not
+ * 64/128, page size not a power of two in [16, 256], HEAD_MAJOR required for sparse).
+ */
+RPA_API rpa_status rpa_plan(const rpa_shape* shape, const int32_t* cu_seqlens_q,
+                    const int32_t* seq_lens_k, const rpa_plan_options* opts,
+                    rpa_plan_t* out_plan, size_t* workspace_bytes);
+
+/* rpa_plan_get_info -- what the planner chose (host only, no device work). */
+RPA_API rpa_status rpa_plan_get_info(rpa_plan_t plan, rpa_plan_info* info);
+
+/* rpa_plan_destroy -- frees the plan's host memory; NULL is ignored. */
+RPA_API void rpa_plan_destroy(rpa_plan_t plan);
+
+/*
+ * rpa_write_kv -- scatter the new tokens' K/V into their cache slots, in place
+ * (ScatterKVToPagedCacheProgram of the WebGPU page, commit "Phase 1b.1": for token i of
+ * sequence b, pos = past_b + i, page = block_table[b, pos / P], slot = pos % P; the
+ * head-major layout uses block_table[b, h, pos / P] per KV head h).  Bytes are copied
+ * unchanged; slots not addressed are not touched.
+ *
+ *   k_new, v_new       device bf16 [T, Hkv, D].
+ *   k_pool, v_pool     device bf16 pools in shape.layout, updated in place.
+ *   block_table        device int32, see rpa_layout.
+ *   cu_seqlens_q       device int32 [B+1] (same values as given to rpa_plan).
+ *   seq_lens_k         device int32 [B].
+ *   workspace          unused by this call; may be NULL.
+ * T == 0 returns RPA_OK and launches nothing.
+ */
+RPA_API rpa_status rpa_write_kv(rpa_plan_t plan, const void* k_new, const void* v_new,
+                        void* k_pool, void* v_pool, const int32_t* block_table,
+                        const int32_t* cu_seqlens_q, const int32_t* seq_lens_k,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * rpa_forward -- the fused step: write the new tokens' K/V (when k_new/v_new are given)
+ * and compute, for every query token t and query head hq,
+ *     out[t, hq] = sum_j softmax_j(scale * q[t,hq] . K_j) V_j
+ * over the keys j the token may see (causal mask; with group tables only keys whose
+ * block -- of P tokens -- is listed for the row's KV group).  Exact attention: a
+ * split-KV decode kernel with an LSE merge for short query rows, a tensor-core
+ * (tcgen05/TMEM) kernel fed by TMA through the block table for the rest.
+ *
+ *   q                 device bf16 [T, Hq, D].
+ *   k_new, v_new      device bf16 [T, Hkv, D], or both NULL when the cache already holds
+ *                     the new tokens (e.g. after rpa_write_kv).
+ *   k_pool, v_pool    device bf16 pools (written in place, then read: the alias rule
+ *                     of the WebGPU page -- input and output cache are one buffer).
+ *   block_table, cu_seqlens_q, seq_lens_k   as for rpa_write_kv.
+ *   group_table       device int32 [B, Hkv, max_blocks_per_seq] of ascending logical
+ *                     block indices (rpa_build_group_tables output), or NULL; requires
+ *                     RPA_LAYOUT_HEAD_MAJOR and a plan made with opts.sparse = 1.
+ *   group_count       device int32 [B, Hkv] valid entries per table row, or NULL.
+ *   scale             softmax scale (typically 1/sqrt(D)); any finite value.
+ *   out               device bf16 [T, Hq, D] (round-to-nearest-even).
+ *   lse               device fp32 [T, Hq] natural-log log-sum-exp of the scaled scores,
+ *                     or NULL.  A row with no visible key gets out = 0, lse = -inf.
+ *   workspace         device buffer of at least rpa_plan's workspace_bytes.
+ * T == 0 returns RPA_OK and launches nothing.  Sequences with q_len == 0 are skipped.
+ */
+RPA_API rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const void* v_new,
+                       void* k_pool, void* v_pool, const int32_t* block_table,
+                       const int32_t* cu_seqlens_q, const int32_t* seq_lens_k,
+                       const int32_t* group_table, const int32_t* group_count, float scale,
+                       void* out, float* lse, void* workspace, size_t workspace_bytes,
+                       void* stream);
+
+/*
+ * rpa_build_group_tables -- block-union KV selection (CompactAttention, Core claim and
+ * Fig. 3): for every sequence b and KV group g, the ascending list of KV blocks kb such
+ * that some query head hq of the group (hq / (Hq/Hkv) == g) selects kb in some query
+ * block: table[b, g, 0 .. count[b,g]-1]; remaining entries are set to -1.
+ *
+ *   mask    device uint8 [B, Hq, nqb, nkb], nonzero = selected.
+ *   table   device int32 [B, Hkv, nkb].
+ *   count   device int32 [B, Hkv].
+ * Bit-exact and deterministic.  nkb <= 65536.
+ */
+RPA_API rpa_status rpa_build_group_tables(const uint8_t* mask, int32_t num_seqs, int32_t num_q_heads,
+                                  int32_t num_kv_heads, int32_t num_q_blocks,
+                                  int32_t num_kv_blocks, int32_t* table, int32_t* count,
+                                  void* stream);
+
+/*
+ * rpa_device_error -- read (and optionally clear) the library's device error word on the
+ * current device.  Kernels never spin without bound: a wait that runs out records a code
+ * here and the kernel returns early.  Synchronizes the device.  *code = 0 means no error.
+ */
+RPA_API rpa_status rpa_device_error(int32_t* code, int32_t clear);
+
+/* rpa_status_string -- static description of a status code. */
+RPA_API const char* rpa_status_string(rpa_status status);
+
+/* rpa_last_error -- thread-local detail of the last failure on this thread ("" if none). */
+RPA_API const char* rpa_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RPA_H */

@@ -1,0 +1,431 @@
+// Split-KV decode over the paged cache, and the log-sum-exp merge of the splits.
+//
+// What it computes: for every (sequence, KV head, key split) the partial softmax attention of
+// the sequence's short query (q_len * G <= 32 rows: every query head of the KV group for
+// every query token) over keys [k_begin, k_end), read in place through the block table.  This
+// is the split-reduce decode of "[WebGPU] Optimized PagedAttention implementation (2/n)"
+// ("What's shipped": FlashAttentionPagedDecodeQKV + FlashAttentionPagedDecodeVxReduce,
+// selected for max_seqlen_q < 32) and the decode specialisation of "Ragged Paged Attention:
+// A High-Performance and Flexible LLM Inference Kernel for TPU" (Key ideas).
+//
+// B200 design:
+//  * one producer warp streams the split's pages with TMA (one block-table lookup per page,
+//    not per slot): boxes of [min(P, 64) slots x 64 dims] per page and half-row, 128-byte
+//    swizzled, into a 3-4 stage ring of 64-key stages completed on mbarriers;
+//  * four consumer warps each own 16 keys of a stage.  S^T = K Q^T runs on the tensor cores
+//    (mma.sync m16n8k16, keys in M, the G heads x q tokens of the group in N), the online
+//    softmax works per query column with three shuffles, P^T is turned into the B operand by
+//    movmatrix, and O^T += V^T P^T runs on the tensor cores again; K and V are read from HBM
+//    exactly once per KV group;
+//  * the four warps' states are combined in shared memory; a sequence with one split writes
+//    the final bf16 output, otherwise the split's normalised output and log2-domain LSE go to
+//    the workspace for the merge kernel.
+//  Key slots past k_end (the tail of the last page, possibly NaN) are masked in S and their V
+//  rows are zeroed in shared memory before the P.V product.
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "ptx.cuh"
+#include "rpa_internal.h"
+
+namespace rpa {
+namespace {
+
+constexpr int kConsumerWarps = 4;
+constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
+constexpr int kMaxItemPages = kMaxSplitKeys / 16 + 1;
+
+template <int D>
+struct DecodeGeom {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kStageKeys = kDecodeStageKeys;                 // 64
+  static constexpr int kHalfBytes = kStageKeys * 128;                 // 8 KB per half-row tile
+  static constexpr int kTensorStageBytes = kHalves * kHalfBytes;      // K (or V) per stage
+  static constexpr int kStages = D == 128 ? 3 : 4;
+  static constexpr int kKOff = 0;
+  static constexpr int kVOff = kStages * kTensorStageBytes;
+  static constexpr int kPagesOff = 2 * kStages * kTensorStageBytes;
+  static constexpr int kBarOff = kPagesOff + kMaxItemPages * 4 + 64;
+  static constexpr int kBytes = kBarOff + 2 * kStages * 8 + 16;
+  static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
+};
+
+struct alignas(16) U4 {
+  uint32_t x, y, z, w;
+};
+
+template <int D, int NT>
+__global__ void __launch_bounds__(kDecodeThreads, 1)
+    decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
+                        const __grid_constant__ CUtensorMap vmap, DecodeLaunch p) {
+  using Geo = DecodeGeom<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* Ks = smem + Geo::kKOff;
+  uint8_t* Vs = smem + Geo::kVOff;
+  int32_t* pages = reinterpret_cast<int32_t*>(smem + Geo::kPagesOff);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + Geo::kBarOff);
+  uint64_t* empty = full + Geo::kStages;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + Geo::kStages);
+
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const DecodeItem it = p.items[blockIdx.x];
+  const int h = blockIdx.y;
+  const int Hq = p.num_q_heads;
+  const int G = Hq / p.num_kv_heads;
+  const int rows = it.q_len * G;
+  const int past = it.kv_len - it.q_len;
+  const int nstages = (it.k_end - it.k_begin + Geo::kStageKeys - 1) / Geo::kStageKeys;
+  const int P = p.kv.page_size;
+  const int log2P = p.kv.log2_page;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Geo::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kConsumerWarps) {
+    // ---------------------------------------------------------------- producer warp
+    const int first_blk = it.k_begin >> log2P;
+    const int last_blk = (it.k_end - 1) >> log2P;
+    const int npg = last_blk - first_blk + 1;
+    const int32_t* bt_row =
+        p.kv.layout == 0
+            ? p.kv.block_table + (size_t)it.seq * p.kv.max_blocks
+            : p.kv.block_table + ((size_t)it.seq * p.kv.num_kv_heads + h) * p.kv.max_blocks;
+    for (int j = lane; j < npg; j += 32) pages[j] = __ldg(bt_row + first_blk + j);
+    __syncwarp();
+    if (lane == 0) {
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+      const int hcoord = p.kv.layout == 0 ? h : 0;
+      const int box_rows = P < Geo::kStageKeys ? P : Geo::kStageKeys;
+      const uint32_t box_bytes = (uint32_t)box_rows * 128u;
+      int issued = 0;
+      for (int s = 0; s < nstages; ++s) {
+        const int slot = s % Geo::kStages;
+        if (s >= Geo::kStages &&
+            !wait_bounded(&empty[slot], ((s / Geo::kStages) - 1) & 1, abort_flag, p.err,
+                          kErrDecodeWait))
+          break;
+        const int kst = it.k_begin + s * Geo::kStageKeys;
+        const int kend = min(kst + Geo::kStageKeys, it.k_end);
+        const int b0 = kst >> log2P;
+        const int b1 = (kend - 1) >> log2P;
+        const int nbox = b1 - b0 + 1;
+        mbar_arrive_expect_tx(&full[slot], 2u * Geo::kHalves * box_bytes * (uint32_t)nbox);
+        for (int bi = 0; bi < nbox; ++bi) {
+          const int blk = b0 + bi;
+          const int page = pages[blk - first_blk];
+          const int srow = P >= Geo::kStageKeys ? (kst & (P - 1)) : 0;
+          const int drow = P >= Geo::kStageKeys ? 0 : blk * P - kst;
+#pragma unroll
+          for (int half = 0; half < Geo::kHalves; ++half) {
+            const int off = slot * Geo::kTensorStageBytes + half * Geo::kHalfBytes + drow * 128;
+            tma_load_4d(Ks + off, &kmap, half * 64, hcoord, srow, page, &full[slot]);
+            tma_load_4d(Vs + off, &vmap, half * 64, hcoord, srow, page, &full[slot]);
+          }
+        }
+        ++issued;
+      }
+      if (*abort_flag) {
+        // let copies already in flight land before the CTA's shared memory goes away
+        for (int s = max(0, issued - Geo::kStages); s < issued; ++s)
+          wait_bounded(&full[s % Geo::kStages], (s / Geo::kStages) & 1, abort_flag, nullptr, 0,
+                       kWaitTimeoutNs / 8);
+      }
+    }
+    __syncwarp();
+    return;  // the consumers keep the CTA (and its shared memory) alive until they finish
+  } else {
+    // ---------------------------------------------------------------- consumer warps
+    constexpr int KT = D / 16;
+    uint32_t bq[NT][KT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      const int col = nt * 8 + (lane >> 2);
+      const bool ok = col < rows;
+      const int tok = it.t0 + (ok ? col / G : 0);
+      const int hq = h * G + (ok ? col % G : 0);
+      const uint32_t* qrow =
+          reinterpret_cast<const uint32_t*>(p.q + ((size_t)tok * Hq + hq) * D);
+#pragma unroll
+      for (int kk = 0; kk < KT; ++kk) {
+        bq[nt][kk][0] = ok ? __ldg(qrow + kk * 8 + (lane & 3)) : 0u;
+        bq[nt][kk][1] = ok ? __ldg(qrow + kk * 8 + 4 + (lane & 3)) : 0u;
+      }
+    }
+    float m[NT][2], ls[NT][2];
+    float acc[KT][NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+      m[nt][0] = m[nt][1] = -CUDART_INF_F;
+      ls[nt][0] = ls[nt][1] = 0.f;
+#pragma unroll
+      for (int mt = 0; mt < KT; ++mt) acc[mt][nt][0] = acc[mt][nt][1] = acc[mt][nt][2] =
+          acc[mt][nt][3] = 0.f;
+    }
+    // column -> visible-key limit (exclusive) for the causal mask
+    int lim[NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int col = nt * 8 + 2 * (lane & 3) + j;
+        const int tok_i = col < rows ? col / G : 0;
+        lim[nt][j] = p.causal ? min(it.k_end, past + tok_i + 1) : it.k_end;
+      }
+
+    const int ar = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;  // K ldmatrix row
+    const int vr = warp * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;  // V ldmatrix.trans row
+    for (int s = 0; s < nstages; ++s) {
+      const int slot = s % Geo::kStages;
+      if (!wait_bounded(&full[slot], (s / Geo::kStages) & 1, abort_flag, p.err, kErrDecodeWait))
+        break;
+      const int key0 = it.k_begin + s * Geo::kStageKeys + warp * 16;
+      if (key0 < it.k_end) {
+        const uint32_t kbase = smem_u32(Ks + slot * Geo::kTensorStageBytes);
+        float c[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0.f;
+#pragma unroll
+        for (int kk = 0; kk < KT; ++kk) {
+          const int chunk = 2 * kk + (lane >> 4);
+          const uint32_t addr = kbase + (chunk >> 3) * Geo::kHalfBytes + ar * 128 +
+                                (((chunk & 7) ^ (ar & 7)) << 4);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4(addr, a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            mma_bf16_16816(c[nt], a0, a1, a2, a3, bq[nt][kk][0], bq[nt][kk][1]);
+        }
+        const int k_lo = key0 + (lane >> 2);
+        const int k_hi = k_lo + 8;
+        uint32_t bp[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+          float pl[2], ph[2];
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            const float s_lo = k_lo < lim[nt][j] ? c[nt][j] * p.scale_log2 : -CUDART_INF_F;
+            const float s_hi = k_hi < lim[nt][j] ? c[nt][2 + j] * p.scale_log2 : -CUDART_INF_F;
+            float tmax = fmaxf(s_lo, s_hi);
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
+            tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 16));
+            const float m_new = fmaxf(m[nt][j], tmax);
+            const float m_use = m_new == -CUDART_INF_F ? 0.f : m_new;
+            const float alpha = fast_exp2(m[nt][j] - m_use);
+            pl[j] = fast_exp2(s_lo - m_use);
+            ph[j] = fast_exp2(s_hi - m_use);
+            ls[nt][j] = ls[nt][j] * alpha + pl[j] + ph[j];
+            m[nt][j] = m_new;
+#pragma unroll
+            for (int mt = 0; mt < KT; ++mt) {
+              acc[mt][nt][j] *= alpha;
+              acc[mt][nt][2 + j] *= alpha;
+            }
+          }
+          bp[nt][0] = movmatrix_trans(pack_bf16(pl[0], pl[1]));
+          bp[nt][1] = movmatrix_trans(pack_bf16(ph[0], ph[1]));
+        }
+        uint8_t* vtile = Vs + slot * Geo::kTensorStageBytes;
+        const int nvalid = it.k_end - key0;
+        if (nvalid < 16) {
+          // rows past the last key may hold anything (NaN poison): P is 0 there, V must be 0
+          const int nz = (16 - nvalid) * Geo::kHalves * 8;
+          for (int i = lane; i < nz; i += 32) {
+            const int row = nvalid + i / (Geo::kHalves * 8);
+            const int rem = i % (Geo::kHalves * 8);
+            *reinterpret_cast<U4*>(vtile + (rem >> 3) * Geo::kHalfBytes +
+                                   (warp * 16 + row) * 128 + (rem & 7) * 16) = U4{0, 0, 0, 0};
+          }
+          __syncwarp();
+        }
+        const uint32_t vbase = smem_u32(vtile);
+#pragma unroll
+        for (int mt = 0; mt < KT; ++mt) {
+          const int chunk = 2 * mt + ((lane >> 3) & 1);
+          const uint32_t addr = vbase + (chunk >> 3) * Geo::kHalfBytes + vr * 128 +
+                                (((chunk & 7) ^ (vr & 7)) << 4);
+          uint32_t a0, a1, a2, a3;
+          ldsm_x4_trans(addr, a0, a1, a2, a3);
+#pragma unroll
+          for (int nt = 0; nt < NT; ++nt)
+            mma_bf16_16816(acc[mt][nt], a0, a1, a2, a3, bp[nt][0], bp[nt][1]);
+        }
+        if (nvalid < 16) fence_proxy_async_smem();  // generic writes before the next TMA
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[slot]);
+    }
+    // row sums: reduce the per-lane partials over the 8 lanes of each column
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        float v = ls[nt][j];
+        v += __shfl_xor_sync(0xffffffffu, v, 4);
+        v += __shfl_xor_sync(0xffffffffu, v, 8);
+        v += __shfl_xor_sync(0xffffffffu, v, 16);
+        ls[nt][j] = v;
+      }
+    // every consumer warp has waited on every stage, so all copies have landed; once all
+    // four are done reading, the stage ring is free for the combine
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    // --------------------------------------------- combine the four warps (reuse K ring)
+    constexpr int COLS = 8 * NT;
+    constexpr int OPAD = D + 4;
+    float* red_m = reinterpret_cast<float*>(smem);
+    float* red_l = red_m + kConsumerWarps * COLS;
+    float* red_o = red_l + kConsumerWarps * COLS;
+    if (!*abort_flag) {
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const int col = nt * 8 + 2 * (lane & 3) + j;
+          if ((lane >> 2) == 0) {
+            red_m[warp * COLS + col] = m[nt][j];
+            red_l[warp * COLS + col] = ls[nt][j];
+          }
+          float* o = red_o + (warp * COLS + col) * OPAD;
+#pragma unroll
+          for (int mt = 0; mt < KT; ++mt) {
+            o[mt * 16 + (lane >> 2)] = acc[mt][nt][j];
+            o[mt * 16 + (lane >> 2) + 8] = acc[mt][nt][2 + j];
+          }
+        }
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (!*abort_flag) {
+      const int Hkv = p.num_kv_heads;
+      for (int idx = threadIdx.x; idx < rows * D; idx += kConsumerWarps * 32) {
+        const int col = idx / D;
+        const int d = idx - col * D;
+        float M = -CUDART_INF_F;
+#pragma unroll
+        for (int w = 0; w < kConsumerWarps; ++w) M = fmaxf(M, red_m[w * COLS + col]);
+        float L = 0.f, O = 0.f;
+        if (M != -CUDART_INF_F) {
+#pragma unroll
+          for (int w = 0; w < kConsumerWarps; ++w) {
+            const float f = fast_exp2(red_m[w * COLS + col] - M);
+            L += red_l[w * COLS + col] * f;
+            O += red_o[(w * COLS + col) * OPAD + d] * f;
+          }
+        }
+        const float o = L > 0.f ? O / L : 0.f;
+        const float lse2 = L > 0.f ? M + fast_log2(L) : -CUDART_INF_F;
+        const int tok = it.t0 + col / G;
+        const int hq = h * G + col % G;
+        if (it.part_slot < 0) {
+          const __nv_bfloat16 ob = __float2bfloat16_rn(o);
+          p.out[((size_t)tok * Hq + hq) * D + d] = *reinterpret_cast<const uint16_t*>(&ob);
+          if (d == 0 && p.lse) p.lse[(size_t)tok * Hq + hq] = lse2 * 0.69314718055994531f;
+        } else {
+          const size_t prow = ((size_t)it.part_slot * Hkv + h) * p.rows_per_item + col;
+          p.part_o[prow * D + d] = o;
+          if (d == 0) p.part_lse[prow] = lse2;
+        }
+      }
+    }
+  }
+}
+
+template <int D>
+__global__ void __launch_bounds__(128) merge_kernel(MergeLaunch p) {
+  const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  const int Hq = p.num_q_heads;
+  if (gw >= p.num_rows * Hq) return;
+  const int r = gw / Hq;
+  const int hq = gw - r * Hq;
+  const int G = Hq / p.num_kv_heads;
+  const MergeRow mr = p.rows[r];
+  const int h = hq / G;
+  const int col = mr.local * G + (hq - h * G);
+  constexpr int E = D / 32;
+  float M = -CUDART_INF_F;
+  for (int s = 0; s < mr.nsplit; ++s) {
+    const size_t prow = ((size_t)(mr.first_slot + s) * p.num_kv_heads + h) * p.rows_per_item + col;
+    M = fmaxf(M, p.part_lse[prow]);
+  }
+  float acc[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc[e] = 0.f;
+  float W = 0.f;
+  if (M != -CUDART_INF_F) {
+    for (int s = 0; s < mr.nsplit; ++s) {
+      const size_t prow =
+          ((size_t)(mr.first_slot + s) * p.num_kv_heads + h) * p.rows_per_item + col;
+      const float l = p.part_lse[prow];
+      const float w = l == -CUDART_INF_F ? 0.f : fast_exp2(l - M);
+      W += w;
+      const float* po = p.part_o + prow * D;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] += w * po[e * 32 + lane];
+    }
+  }
+  const float inv = W > 0.f ? 1.f / W : 0.f;
+  uint16_t* o = p.out + ((size_t)mr.token * Hq + hq) * D;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const __nv_bfloat16 ob = __float2bfloat16_rn(acc[e] * inv);
+    o[e * 32 + lane] = *reinterpret_cast<const uint16_t*>(&ob);
+  }
+  if (lane == 0 && p.lse)
+    p.lse[(size_t)mr.token * Hq + hq] =
+        W > 0.f ? (M + fast_log2(W)) * 0.69314718055994531f : -CUDART_INF_F;
+}
+
+template <int D, int NT>
+cudaError_t launch_decode_t(const DecodeLaunch& p, cudaStream_t stream) {
+  using Geo = DecodeGeom<D>;
+  // 4-D box over the pool: (dims, kv head, slot, page); head-major pools use one "head".
+  CUtensorMap kmap, vmap;
+  cudaError_t e = encode_kv_map(&kmap, p.kv.k_pool, p.kv, D, kDecodeStageKeys);
+  if (e != cudaSuccess) return e;
+  e = encode_kv_map(&vmap, p.kv.v_pool, p.kv, D, kDecodeStageKeys);
+  if (e != cudaSuccess) return e;
+  auto kern = decode_split_kernel<D, NT>;
+  e = ensure_smem_attr(reinterpret_cast<const void*>(kern), Geo::kAlloc);
+  if (e != cudaSuccess) return e;
+  dim3 grid(p.num_items, p.num_kv_heads);
+  kern<<<grid, kDecodeThreads, Geo::kAlloc, stream>>>(kmap, vmap, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeLaunch& p, int nt, cudaStream_t stream) {
+  if (p.num_items <= 0) return cudaSuccess;
+  if (p.head_dim == 128) {
+    if (nt == 1) return launch_decode_t<128, 1>(p, stream);
+    if (nt == 2) return launch_decode_t<128, 2>(p, stream);
+    return launch_decode_t<128, 4>(p, stream);
+  }
+  if (nt == 1) return launch_decode_t<64, 1>(p, stream);
+  if (nt == 2) return launch_decode_t<64, 2>(p, stream);
+  return launch_decode_t<64, 4>(p, stream);
+}
+
+cudaError_t launch_merge(const MergeLaunch& p, cudaStream_t stream) {
+  if (p.num_rows <= 0) return cudaSuccess;
+  const long warps = (long)p.num_rows * p.num_q_heads;
+  const int blocks = (int)((warps + 3) / 4);
+  if (p.head_dim == 128)
+    merge_kernel<128><<<blocks, 128, 0, stream>>>(p);
+  else
+    merge_kernel<64><<<blocks, 128, 0, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace rpa

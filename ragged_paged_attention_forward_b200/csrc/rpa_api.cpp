@@ -1,0 +1,552 @@
+// C ABI of librpa.so (include/rpa.h): argument validation, the host planner and the launch
+// sequence of one step.
+//
+// The planner is the distribution-aware part of "Ragged Paged Attention: A High-Performance
+// and Flexible LLM Inference Kernel for TPU" (Key ideas): it classifies the batch (decode /
+// prefill / mixed, with the q_len < 32 decode threshold of "[WebGPU] Optimized PagedAttention
+// implementation (2/n)", "Correctness invariants") and slices the ragged batch into work
+// items without padding: (sequence, key split) items for the split-KV decode kernel and
+// (sequence, 128-query tile) items for the tensor-core kernel, heaviest first.  The work lists
+// are built once on the host and copied into the caller's workspace by rpa_forward.
+#include <cuda_runtime.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+#include <cmath>
+#include <new>
+#include <string>
+#include <vector>
+
+#include "rpa.h"
+#include "rpa_internal.h"
+
+namespace rpa {
+
+namespace {
+thread_local std::string g_last_error;
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int ilog2(int x) {
+  int r = 0;
+  while ((1 << r) < x) ++r;
+  return r;
+}
+}  // namespace
+
+void set_last_error(const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+}
+
+}  // namespace rpa
+
+using namespace rpa;
+
+struct rpa_plan_s {
+  rpa_shape shape;
+  rpa_plan_options opts;
+  int batch_class = RPA_CLASS_AUTO;
+  int split_keys = 0;
+  int decode_nt = 1;
+  std::vector<DecodeItem> dec_items;
+  std::vector<MergeRow> merge_rows;
+  std::vector<PrefillTile> pf_tiles;
+  int num_part_slots = 0;
+  // workspace layout: [decode items][merge rows][prefill tiles] | [partial O][partial LSE]
+  size_t off_dec = 0, off_merge = 0, off_pf = 0, meta_bytes = 0;
+  size_t off_part_o = 0, off_part_lse = 0, ws_bytes = 0;
+  std::vector<uint8_t> meta;  // host image of the metadata region
+  int launches_forward = 0;
+  int launches_write = 0;
+};
+
+#define RPA_FAIL(code, ...)            \
+  do {                                 \
+    rpa::set_last_error(__VA_ARGS__);  \
+    return (code);                     \
+  } while (0)
+
+namespace {
+
+rpa_status check_cuda(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return RPA_OK;
+  rpa::set_last_error("%s: %s", what, cudaGetErrorString(e));
+  return RPA_ERR_CUDA;
+}
+
+rpa_status validate_shape(const rpa_shape& s) {
+  if (s.num_seqs < 0 || s.num_tokens < 0)
+    RPA_FAIL(RPA_ERR_SHAPE, "num_seqs (%d) and num_tokens (%d) must be >= 0", s.num_seqs,
+             s.num_tokens);
+  if (s.num_q_heads <= 0 || s.num_kv_heads <= 0)
+    RPA_FAIL(RPA_ERR_SHAPE, "head counts must be positive (Hq=%d, Hkv=%d)", s.num_q_heads,
+             s.num_kv_heads);
+  if (s.num_q_heads % s.num_kv_heads != 0)
+    RPA_FAIL(RPA_ERR_SHAPE, "num_q_heads (%d) must be a multiple of num_kv_heads (%d)",
+             s.num_q_heads, s.num_kv_heads);
+  if (s.head_dim != 64 && s.head_dim != 128)
+    RPA_FAIL(RPA_ERR_UNSUPPORTED, "head_dim %d is not supported (64 or 128)", s.head_dim);
+  if (s.page_size < 16 || s.page_size > 256 || (s.page_size & (s.page_size - 1)) != 0)
+    RPA_FAIL(RPA_ERR_UNSUPPORTED, "page_size %d must be a power of two in [16, 256]",
+             s.page_size);
+  if (s.num_pages <= 0) RPA_FAIL(RPA_ERR_SHAPE, "num_pages (%d) must be > 0", s.num_pages);
+  if (s.max_blocks_per_seq <= 0)
+    RPA_FAIL(RPA_ERR_SHAPE, "max_blocks_per_seq (%d) must be > 0", s.max_blocks_per_seq);
+  if (s.layout != RPA_LAYOUT_SEQ_MAJOR && s.layout != RPA_LAYOUT_HEAD_MAJOR)
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "unknown layout %d", s.layout);
+  if (s.causal != 0 && s.causal != 1) RPA_FAIL(RPA_ERR_INVALID_ARG, "causal must be 0 or 1");
+  return RPA_OK;
+}
+
+// Decode items hold every query row of their sequence in the N dimension of the warp MMAs:
+// q_len * G <= 32.
+constexpr int kMaxDecodeRows = 32;
+
+int auto_split_keys(long total_key_heads, int sms) {
+  // aim for >= ~8 CTAs per SM (two resident, four waves) without splits under 256 keys
+  const long target_ctas = (long)sms * 8;
+  long s = total_key_heads / std::max(1L, target_ctas);
+  s = (s + kDecodeStageKeys - 1) / kDecodeStageKeys * kDecodeStageKeys;
+  s = std::max<long>(s, kMinSplitKeys);
+  s = std::min<long>(s, kMaxSplitKeys);
+  return (int)s;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* rpa_status_string(rpa_status s) {
+  switch (s) {
+    case RPA_OK: return "RPA_OK";
+    case RPA_ERR_INVALID_ARG: return "RPA_ERR_INVALID_ARG";
+    case RPA_ERR_UNSUPPORTED: return "RPA_ERR_UNSUPPORTED";
+    case RPA_ERR_SHAPE: return "RPA_ERR_SHAPE";
+    case RPA_ERR_WORKSPACE_TOO_SMALL: return "RPA_ERR_WORKSPACE_TOO_SMALL";
+    case RPA_ERR_CUDA: return "RPA_ERR_CUDA";
+    case RPA_ERR_DEVICE_CHECK: return "RPA_ERR_DEVICE_CHECK";
+  }
+  return "RPA_ERR_UNKNOWN";
+}
+
+const char* rpa_last_error(void) { return g_last_error.c_str(); }
+
+rpa_status rpa_plan(const rpa_shape* shape, const int32_t* cu_seqlens_q,
+                    const int32_t* seq_lens_k, const rpa_plan_options* opts,
+                    rpa_plan_t* out_plan, size_t* workspace_bytes) {
+  g_last_error.clear();
+  if (!shape || !out_plan) RPA_FAIL(RPA_ERR_INVALID_ARG, "shape and out_plan must not be NULL");
+  *out_plan = nullptr;
+  rpa_status st = validate_shape(*shape);
+  if (st != RPA_OK) return st;
+  const rpa_shape& s = *shape;
+  const int B = s.num_seqs;
+  if (B > 0 && (!cu_seqlens_q || !seq_lens_k))
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "cu_seqlens_q and seq_lens_k (host arrays) are required");
+  rpa_plan_options o;
+  memset(&o, 0, sizeof(o));
+  if (opts) o = *opts;
+  for (int i = 0; i < 5; ++i)
+    if (o.reserved[i] != 0) RPA_FAIL(RPA_ERR_INVALID_ARG, "plan option reserved[%d] != 0", i);
+  if (o.force_class < RPA_CLASS_AUTO || o.force_class > RPA_CLASS_MIXED)
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "unknown force_class %d", o.force_class);
+  if (o.decode_split_keys != 0 &&
+      (o.decode_split_keys % kDecodeStageKeys != 0 || o.decode_split_keys < kDecodeStageKeys ||
+       o.decode_split_keys > kMaxSplitKeys))
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "decode_split_keys %d must be a multiple of %d in [%d, %d]",
+             o.decode_split_keys, kDecodeStageKeys, kDecodeStageKeys, kMaxSplitKeys);
+  if (o.sparse && s.layout != RPA_LAYOUT_HEAD_MAJOR)
+    RPA_FAIL(RPA_ERR_UNSUPPORTED, "block-union tables need the KV-head-major layout");
+
+  // ---- lengths
+  if (B > 0) {
+    if (cu_seqlens_q[0] != 0) RPA_FAIL(RPA_ERR_SHAPE, "cu_seqlens_q[0] must be 0");
+    for (int b = 0; b < B; ++b) {
+      const int q_len = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
+      if (q_len < 0) RPA_FAIL(RPA_ERR_SHAPE, "cu_seqlens_q is decreasing at %d", b);
+      const int kv = seq_lens_k[b];
+      if (kv < 0) RPA_FAIL(RPA_ERR_SHAPE, "seq_lens_k[%d] = %d < 0", b, kv);
+      if (q_len > kv)
+        RPA_FAIL(RPA_ERR_SHAPE, "sequence %d: q_len %d exceeds kv_len %d", b, q_len, kv);
+      const long blocks = ((long)kv + s.page_size - 1) / s.page_size;
+      if (blocks > s.max_blocks_per_seq)
+        RPA_FAIL(RPA_ERR_SHAPE, "sequence %d: kv_len %d needs %ld pages > max_blocks_per_seq %d",
+                 b, kv, blocks, s.max_blocks_per_seq);
+    }
+  }
+  const int T = B > 0 ? cu_seqlens_q[B] : 0;
+  if (T != s.num_tokens)
+    RPA_FAIL(RPA_ERR_SHAPE, "cu_seqlens_q[B] = %d but num_tokens = %d", T, s.num_tokens);
+
+  rpa_plan_s* plan = new (std::nothrow) rpa_plan_s();
+  if (!plan) RPA_FAIL(RPA_ERR_INVALID_ARG, "out of host memory");
+  plan->shape = s;
+  plan->opts = o;
+
+  // ---- classification (affects speed only, never results)
+  const int G = s.num_q_heads / s.num_kv_heads;
+  bool all_decode = true, all_prefill = true;
+  for (int b = 0; b < B; ++b) {
+    const int q_len = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
+    if (q_len == 0) continue;
+    if (q_len > 1) all_decode = false;
+    if (q_len < 32) all_prefill = false;
+  }
+  int cls = all_decode ? RPA_CLASS_DECODE : (all_prefill ? RPA_CLASS_PREFILL : RPA_CLASS_MIXED);
+  if (o.force_class != RPA_CLASS_AUTO) cls = o.force_class;
+  plan->batch_class = cls;
+
+  // row routing: the split-KV decode kernel takes short rows whose query heads x tokens fit
+  // the warp MMA's N (<= 16 for mixed batches, <= 32 when forced / pure decode)
+  const int decode_rows_cap = (cls == RPA_CLASS_MIXED) ? 16 : kMaxDecodeRows;
+  std::vector<int> to_decode(B, 0);
+  long total_key_heads = 0;
+  int max_rows = 0;
+  for (int b = 0; b < B; ++b) {
+    const int q_len = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
+    if (q_len == 0) continue;
+    const bool dec = !o.sparse && cls != RPA_CLASS_PREFILL && q_len * G <= decode_rows_cap;
+    to_decode[b] = dec ? 1 : 0;
+    if (dec) {
+      total_key_heads += (long)seq_lens_k[b] * s.num_kv_heads;
+      max_rows = std::max(max_rows, q_len * G);
+    }
+  }
+  plan->decode_nt = max_rows <= 8 ? 1 : (max_rows <= 16 ? 2 : 4);
+  plan->split_keys = o.decode_split_keys ? o.decode_split_keys
+                                         : auto_split_keys(total_key_heads, device_sm_count());
+
+  // ---- decode items and merge rows
+  int slots = 0;
+  for (int b = 0; b < B; ++b) {
+    if (!to_decode[b]) continue;
+    const int t0 = cu_seqlens_q[b];
+    const int q_len = cu_seqlens_q[b + 1] - t0;
+    const int kv = seq_lens_k[b];
+    const int nsplit = (kv + plan->split_keys - 1) / plan->split_keys;
+    for (int sp = 0; sp < nsplit; ++sp) {
+      DecodeItem it;
+      it.seq = b;
+      it.t0 = t0;
+      it.q_len = q_len;
+      it.kv_len = kv;
+      it.k_begin = sp * plan->split_keys;
+      it.k_end = std::min(kv, (sp + 1) * plan->split_keys);
+      it.part_slot = nsplit > 1 ? slots + sp : -1;
+      it.pad = 0;
+      plan->dec_items.push_back(it);
+    }
+    if (nsplit > 1) {
+      for (int i = 0; i < q_len; ++i) plan->merge_rows.push_back(MergeRow{t0 + i, i, slots, nsplit});
+      slots += nsplit;
+    }
+  }
+  plan->num_part_slots = slots;
+  // longest items first so the tail of the grid is short
+  std::stable_sort(plan->dec_items.begin(), plan->dec_items.end(),
+                   [](const DecodeItem& a, const DecodeItem& b) {
+                     return (a.k_end - a.k_begin) > (b.k_end - b.k_begin);
+                   });
+
+  // ---- prefill tiles (heaviest first: most visible keys)
+  for (int b = 0; b < B; ++b) {
+    const int t0 = cu_seqlens_q[b];
+    const int q_len = cu_seqlens_q[b + 1] - t0;
+    if (q_len == 0 || to_decode[b]) continue;
+    for (int qs = 0; qs < q_len; qs += kPrefillTileRows) {
+      PrefillTile t;
+      t.seq = b;
+      t.t0 = t0;
+      t.q_len = q_len;
+      t.kv_len = seq_lens_k[b];
+      t.q_start = qs;
+      t.pad[0] = t.pad[1] = t.pad[2] = 0;
+      plan->pf_tiles.push_back(t);
+    }
+  }
+  auto work = [&](const PrefillTile& t) {
+    const long past = t.kv_len - t.q_len;
+    const long q_end = std::min(t.q_len, t.q_start + kPrefillTileRows);
+    return s.causal ? std::min<long>(t.kv_len, past + q_end) : (long)t.kv_len;
+  };
+  std::stable_sort(plan->pf_tiles.begin(), plan->pf_tiles.end(),
+                   [&](const PrefillTile& a, const PrefillTile& b) { return work(a) > work(b); });
+
+  // ---- workspace layout
+  size_t off = 0;
+  plan->off_dec = off;
+  off = align_up(off + plan->dec_items.size() * sizeof(DecodeItem), 256);
+  plan->off_merge = off;
+  off = align_up(off + plan->merge_rows.size() * sizeof(MergeRow), 256);
+  plan->off_pf = off;
+  off = align_up(off + plan->pf_tiles.size() * sizeof(PrefillTile), 256);
+  plan->meta_bytes = off;
+  const size_t rows_per_item = 8 * plan->decode_nt;
+  plan->off_part_o = off;
+  off = align_up(off + (size_t)slots * s.num_kv_heads * rows_per_item * s.head_dim * 4, 256);
+  plan->off_part_lse = off;
+  off = align_up(off + (size_t)slots * s.num_kv_heads * rows_per_item * 4, 256);
+  plan->ws_bytes = std::max<size_t>(off, 256);
+  plan->meta.assign(plan->meta_bytes, 0);
+  if (!plan->dec_items.empty())
+    memcpy(plan->meta.data() + plan->off_dec, plan->dec_items.data(),
+           plan->dec_items.size() * sizeof(DecodeItem));
+  if (!plan->merge_rows.empty())
+    memcpy(plan->meta.data() + plan->off_merge, plan->merge_rows.data(),
+           plan->merge_rows.size() * sizeof(MergeRow));
+  if (!plan->pf_tiles.empty())
+    memcpy(plan->meta.data() + plan->off_pf, plan->pf_tiles.data(),
+           plan->pf_tiles.size() * sizeof(PrefillTile));
+
+  plan->launches_write = T > 0 ? 1 : 0;
+  plan->launches_forward = (plan->dec_items.empty() ? 0 : 1) +
+                           (plan->merge_rows.empty() ? 0 : 1) +
+                           (plan->pf_tiles.empty() ? 0 : 1);
+  *out_plan = plan;
+  if (workspace_bytes) *workspace_bytes = plan->ws_bytes;
+  return RPA_OK;
+}
+
+rpa_status rpa_plan_get_info(rpa_plan_t plan, rpa_plan_info* info) {
+  if (!plan || !info) RPA_FAIL(RPA_ERR_INVALID_ARG, "plan and info must not be NULL");
+  memset(info, 0, sizeof(*info));
+  info->batch_class = plan->batch_class;
+  info->num_decode_items = (int32_t)plan->dec_items.size();
+  info->num_prefill_tiles = (int32_t)plan->pf_tiles.size();
+  info->num_merge_rows = (int32_t)plan->merge_rows.size();
+  info->launches_forward = plan->launches_forward;
+  info->launches_write = plan->launches_write;
+  info->decode_split_keys = plan->split_keys;
+  info->workspace_bytes = plan->ws_bytes;
+  return RPA_OK;
+}
+
+void rpa_plan_destroy(rpa_plan_t plan) { delete plan; }
+
+static rpa_status write_kv_impl(rpa_plan_t plan, const void* k_new, const void* v_new,
+                                void* k_pool, void* v_pool, const int32_t* block_table,
+                                const int32_t* cu_seqlens_q, const int32_t* seq_lens_k,
+                                cudaStream_t stream) {
+  const rpa_shape& s = plan->shape;
+  int* err = nullptr;
+  rpa_status st = check_cuda(device_error_word(&err), "device error word");
+  if (st != RPA_OK) return st;
+  WriteLaunch w;
+  w.k_new = static_cast<const uint16_t*>(k_new);
+  w.v_new = static_cast<const uint16_t*>(v_new);
+  w.k_pool = static_cast<uint16_t*>(k_pool);
+  w.v_pool = static_cast<uint16_t*>(v_pool);
+  w.block_table = block_table;
+  w.cu_seqlens_q = cu_seqlens_q;
+  w.seq_lens_k = seq_lens_k;
+  w.num_seqs = s.num_seqs;
+  w.num_tokens = s.num_tokens;
+  w.num_kv_heads = s.num_kv_heads;
+  w.head_dim = s.head_dim;
+  w.page_size = s.page_size;
+  w.max_blocks = s.max_blocks_per_seq;
+  w.layout = s.layout;
+  w.num_pages = s.num_pages;
+  w.err = err;
+  return check_cuda(launch_write_kv(w, stream), "write_kv launch");
+}
+
+static rpa_status check_common(rpa_plan_t plan, const void* k_pool, const void* v_pool,
+                               const int32_t* block_table, const int32_t* cu_seqlens_q,
+                               const int32_t* seq_lens_k) {
+  if (!plan) RPA_FAIL(RPA_ERR_INVALID_ARG, "plan must not be NULL");
+  if (!k_pool || !v_pool || !block_table || !cu_seqlens_q || !seq_lens_k)
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "pools, block_table, cu_seqlens_q and seq_lens_k are required");
+  if (!aligned16(k_pool) || !aligned16(v_pool))
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "k_pool / v_pool must be 16-byte aligned");
+  return RPA_OK;
+}
+
+rpa_status rpa_write_kv(rpa_plan_t plan, const void* k_new, const void* v_new, void* k_pool,
+                        void* v_pool, const int32_t* block_table, const int32_t* cu_seqlens_q,
+                        const int32_t* seq_lens_k, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  g_last_error.clear();
+  rpa_status st = check_common(plan, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k);
+  if (st != RPA_OK) return st;
+  if (plan->shape.num_tokens == 0) return RPA_OK;
+  if (!k_new || !v_new) RPA_FAIL(RPA_ERR_INVALID_ARG, "k_new and v_new are required");
+  if (!aligned16(k_new) || !aligned16(v_new))
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "k_new / v_new must be 16-byte aligned");
+  return write_kv_impl(plan, k_new, v_new, k_pool, v_pool, block_table, cu_seqlens_q,
+                       seq_lens_k, static_cast<cudaStream_t>(stream));
+}
+
+rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const void* v_new,
+                       void* k_pool, void* v_pool, const int32_t* block_table,
+                       const int32_t* cu_seqlens_q, const int32_t* seq_lens_k,
+                       const int32_t* group_table, const int32_t* group_count, float scale,
+                       void* out, float* lse, void* workspace, size_t workspace_bytes,
+                       void* stream_) {
+  g_last_error.clear();
+  rpa_status st = check_common(plan, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k);
+  if (st != RPA_OK) return st;
+  const rpa_shape& s = plan->shape;
+  cudaStream_t stream = static_cast<cudaStream_t>(stream_);
+  if (s.num_tokens == 0) return RPA_OK;
+  if (!q || !out) RPA_FAIL(RPA_ERR_INVALID_ARG, "q and out are required");
+  if (!aligned16(q) || !aligned16(out))
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "q / out must be 16-byte aligned");
+  if ((k_new == nullptr) != (v_new == nullptr))
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "k_new and v_new must both be given or both be NULL");
+  if (k_new && (!aligned16(k_new) || !aligned16(v_new)))
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "k_new / v_new must be 16-byte aligned");
+  if ((group_table == nullptr) != (group_count == nullptr))
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "group_table and group_count go together");
+  if (group_table && s.layout != RPA_LAYOUT_HEAD_MAJOR)
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "group tables need the KV-head-major layout");
+  if ((group_table != nullptr) != (plan->opts.sparse != 0))
+    RPA_FAIL(RPA_ERR_INVALID_ARG,
+             "group tables must be given exactly when the plan was made with opts.sparse = 1");
+  if (!std::isfinite(scale)) RPA_FAIL(RPA_ERR_INVALID_ARG, "scale must be finite");
+  if (!workspace || workspace_bytes < plan->ws_bytes)
+    RPA_FAIL(RPA_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes needed, %zu given",
+             plan->ws_bytes, workspace ? workspace_bytes : (size_t)0);
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
+
+  if (k_new) {
+    st = write_kv_impl(plan, k_new, v_new, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k,
+                       stream);
+    if (st != RPA_OK) return st;
+  }
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  if (plan->meta_bytes > 0) {
+    st = check_cuda(cudaMemcpyAsync(ws, plan->meta.data(), plan->meta_bytes,
+                                    cudaMemcpyHostToDevice, stream),
+                    "work-list copy");
+    if (st != RPA_OK) return st;
+  }
+  int* err = nullptr;
+  st = check_cuda(device_error_word(&err), "device error word");
+  if (st != RPA_OK) return st;
+
+  PagedKV kv;
+  kv.k_pool = k_pool;
+  kv.v_pool = v_pool;
+  kv.block_table = block_table;
+  kv.layout = s.layout;
+  kv.page_size = s.page_size;
+  kv.log2_page = ilog2(s.page_size);
+  kv.max_blocks = s.max_blocks_per_seq;
+  kv.num_kv_heads = s.num_kv_heads;
+  kv.num_pages = s.num_pages;
+  const float scale_log2 = scale * 1.4426950408889634f;
+
+  if (!plan->pf_tiles.empty()) {
+    PrefillLaunch p;
+    p.tiles = reinterpret_cast<const PrefillTile*>(ws + plan->off_pf);
+    p.num_tiles = (int32_t)plan->pf_tiles.size();
+    p.q = static_cast<const uint16_t*>(q);
+    p.num_tokens = s.num_tokens;
+    p.num_q_heads = s.num_q_heads;
+    p.num_kv_heads = s.num_kv_heads;
+    p.head_dim = s.head_dim;
+    p.causal = s.causal;
+    p.scale_log2 = scale_log2;
+    p.out = static_cast<uint16_t*>(out);
+    p.lse = lse;
+    p.group_table = group_table;
+    p.group_count = group_count;
+    p.err = err;
+    p.kv = kv;
+    st = check_cuda(launch_prefill(p, stream), "prefill launch");
+    if (st != RPA_OK) return st;
+  }
+  if (!plan->dec_items.empty()) {
+    DecodeLaunch d;
+    d.items = reinterpret_cast<const DecodeItem*>(ws + plan->off_dec);
+    d.num_items = (int32_t)plan->dec_items.size();
+    d.rows_per_item = 8 * plan->decode_nt;
+    d.q = static_cast<const uint16_t*>(q);
+    d.num_q_heads = s.num_q_heads;
+    d.num_kv_heads = s.num_kv_heads;
+    d.head_dim = s.head_dim;
+    d.causal = s.causal;
+    d.scale_log2 = scale_log2;
+    d.out = static_cast<uint16_t*>(out);
+    d.lse = lse;
+    d.part_o = reinterpret_cast<float*>(ws + plan->off_part_o);
+    d.part_lse = reinterpret_cast<float*>(ws + plan->off_part_lse);
+    d.err = err;
+    d.kv = kv;
+    st = check_cuda(launch_decode(d, plan->decode_nt, stream), "decode launch");
+    if (st != RPA_OK) return st;
+    if (!plan->merge_rows.empty()) {
+      MergeLaunch m;
+      m.rows = reinterpret_cast<const MergeRow*>(ws + plan->off_merge);
+      m.num_rows = (int32_t)plan->merge_rows.size();
+      m.rows_per_item = d.rows_per_item;
+      m.num_q_heads = s.num_q_heads;
+      m.num_kv_heads = s.num_kv_heads;
+      m.head_dim = s.head_dim;
+      m.part_o = d.part_o;
+      m.part_lse = d.part_lse;
+      m.out = d.out;
+      m.lse = lse;
+      st = check_cuda(launch_merge(m, stream), "merge launch");
+      if (st != RPA_OK) return st;
+    }
+  }
+  return RPA_OK;
+}
+
+rpa_status rpa_build_group_tables(const uint8_t* mask, int32_t num_seqs, int32_t num_q_heads,
+                                  int32_t num_kv_heads, int32_t num_q_blocks,
+                                  int32_t num_kv_blocks, int32_t* table, int32_t* count,
+                                  void* stream) {
+  g_last_error.clear();
+  if (num_seqs < 0 || num_q_heads <= 0 || num_kv_heads <= 0 || num_q_blocks < 0 ||
+      num_kv_blocks < 0)
+    RPA_FAIL(RPA_ERR_SHAPE, "invalid table-builder sizes");
+  if (num_q_heads % num_kv_heads != 0)
+    RPA_FAIL(RPA_ERR_SHAPE, "num_q_heads (%d) must be a multiple of num_kv_heads (%d)",
+             num_q_heads, num_kv_heads);
+  if (num_kv_blocks > 65536) RPA_FAIL(RPA_ERR_UNSUPPORTED, "num_kv_blocks > 65536");
+  if (num_seqs == 0) return RPA_OK;
+  if (!table || !count || (!mask && num_q_blocks > 0 && num_kv_blocks > 0))
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "mask, table and count are required");
+  return check_cuda(launch_group_tables(mask, num_seqs, num_q_heads, num_kv_heads, num_q_blocks,
+                                        num_kv_blocks, table, count,
+                                        static_cast<cudaStream_t>(stream)),
+                    "group-table launch");
+}
+
+rpa_status rpa_device_error(int32_t* code, int32_t clear) {
+  g_last_error.clear();
+  if (!code) RPA_FAIL(RPA_ERR_INVALID_ARG, "code must not be NULL");
+  int* err = nullptr;
+  rpa_status st = check_cuda(device_error_word(&err), "device error word");
+  if (st != RPA_OK) return st;
+  st = check_cuda(cudaDeviceSynchronize(), "synchronize");
+  if (st != RPA_OK) return st;
+  int v = 0;
+  st = check_cuda(cudaMemcpy(&v, err, sizeof(int), cudaMemcpyDeviceToHost), "read error word");
+  if (st != RPA_OK) return st;
+  *code = v;
+  if (clear && v != 0) {
+    const int zero = 0;
+    st = check_cuda(cudaMemcpy(err, &zero, sizeof(int), cudaMemcpyHostToDevice),
+                    "clear error word");
+    if (st != RPA_OK) return st;
+  }
+  return v == 0 ? RPA_OK : RPA_ERR_DEVICE_CHECK;
+}
+
+}  // extern "C"

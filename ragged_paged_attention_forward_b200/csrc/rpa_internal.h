@@ -1,0 +1,167 @@
+// Internal declarations shared by the host planner (rpa_api.cpp) and the kernels (*.cu).
+// Nothing here is part of the public ABI (include/rpa.h).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace rpa {
+
+// Keys handled by one pipeline stage of the decode kernel and by one tensor-core tile of the
+// prefill kernel.
+constexpr int kDecodeStageKeys = 64;
+constexpr int kPrefillTileKeys = 128;
+constexpr int kPrefillTileRows = 128;
+constexpr int kMaxSplitKeys = 4096;
+constexpr int kMinSplitKeys = 256;
+
+// Device error word codes (OR-ed together).
+enum DeviceErrorCode : int {
+  kErrDecodeWait = 1 << 0,
+  kErrPrefillWait = 1 << 1,
+  kErrBadIndex = 1 << 2,
+};
+
+// One (sequence, key range) item of the split-KV decode kernel; one CTA per (item, KV head).
+struct DecodeItem {
+  int32_t seq;
+  int32_t t0;         // first query token of the sequence
+  int32_t q_len;      // query tokens (all of them: a decode item covers the whole query)
+  int32_t kv_len;
+  int32_t k_begin;    // key range [k_begin, k_end), k_begin a multiple of kDecodeStageKeys
+  int32_t k_end;
+  int32_t part_slot;  // -1: single split, write the final output; else partial-result slot
+  int32_t pad;
+};
+static_assert(sizeof(DecodeItem) == 32, "DecodeItem layout");
+
+// One query token whose decode splits are merged (log-sum-exp reduce).
+struct MergeRow {
+  int32_t token;
+  int32_t local;       // query index inside its sequence
+  int32_t first_slot;  // partial slots first_slot .. first_slot + nsplit - 1
+  int32_t nsplit;
+};
+static_assert(sizeof(MergeRow) == 16, "MergeRow layout");
+
+// One 128-query-token tile of the prefill kernel; one CTA per (tile, query head).
+struct PrefillTile {
+  int32_t seq;
+  int32_t t0;       // first query token of the sequence
+  int32_t q_len;
+  int32_t kv_len;
+  int32_t q_start;  // local index of the tile's first query
+  int32_t pad[3];
+};
+static_assert(sizeof(PrefillTile) == 32, "PrefillTile layout");
+
+struct PagedKV {
+  const void* k_pool;
+  const void* v_pool;
+  const int32_t* block_table;
+  int32_t layout;          // 0 seq-major, 1 head-major
+  int32_t page_size;
+  int32_t log2_page;
+  int32_t max_blocks;
+  int32_t num_kv_heads;
+  int32_t num_pages;
+};
+
+struct DecodeLaunch {
+  const DecodeItem* items;
+  int32_t num_items;
+  int32_t rows_per_item;     // 8 * NT: stride of the partial-result rows
+  const uint16_t* q;         // bf16 [T, Hq, D]
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t causal;
+  float scale_log2;          // softmax scale * log2(e)
+  uint16_t* out;             // bf16 [T, Hq, D]
+  float* lse;                // [T, Hq] or null
+  float* part_o;             // [slots, Hkv, rows_per_item, D]
+  float* part_lse;           // [slots, Hkv, rows_per_item] (log2 domain)
+  int* err;
+  PagedKV kv;
+};
+
+struct MergeLaunch {
+  const MergeRow* rows;
+  int32_t num_rows;
+  int32_t rows_per_item;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  const float* part_o;
+  const float* part_lse;
+  uint16_t* out;
+  float* lse;
+};
+
+struct PrefillLaunch {
+  const PrefillTile* tiles;
+  int32_t num_tiles;
+  const uint16_t* q;
+  int32_t num_tokens;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t causal;
+  float scale_log2;
+  uint16_t* out;
+  float* lse;
+  const int32_t* group_table;  // [B, Hkv, max_blocks] or null
+  const int32_t* group_count;  // [B, Hkv] or null
+  int* err;
+  PagedKV kv;
+};
+
+struct WriteLaunch {
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  uint16_t* k_pool;
+  uint16_t* v_pool;
+  const int32_t* block_table;
+  const int32_t* cu_seqlens_q;
+  const int32_t* seq_lens_k;
+  int32_t num_seqs;
+  int32_t num_tokens;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t page_size;
+  int32_t max_blocks;
+  int32_t layout;
+  int32_t num_pages;
+  int* err;
+};
+
+// Launchers (return the cudaError_t of the launch).
+cudaError_t launch_write_kv(const WriteLaunch& p, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeLaunch& p, int nt, cudaStream_t stream);
+cudaError_t launch_merge(const MergeLaunch& p, cudaStream_t stream);
+cudaError_t launch_prefill(const PrefillLaunch& p, cudaStream_t stream);
+cudaError_t launch_group_tables(const uint8_t* mask, int B, int Hq, int Hkv, int nqb, int nkb,
+                                int32_t* table, int32_t* count, cudaStream_t stream);
+
+// Device error word of the current device (allocated by the library, lives until exit).
+cudaError_t device_error_word(int** ptr);
+
+// Host helpers (launch_util.cpp).
+// TMA map over a K or V pool seen as 4-D (dims, kv heads, slots, pages), innermost first; the
+// head-major pool is the same with a single "head".  Box: 64 dims x 1 head x
+// min(page_size, box_keys) slots x 1 page, 128-byte swizzle.
+cudaError_t encode_kv_map(CUtensorMap* map, const void* pool, const PagedKV& kv, int head_dim,
+                          int box_keys);
+// TMA map over Q [T, Hq, D] seen as 3-D (dims, heads, tokens); box 64 x 1 x box_rows.
+cudaError_t encode_q_map(CUtensorMap* map, const void* q, int num_tokens, int num_q_heads,
+                         int head_dim, int box_rows);
+// Raise a kernel's dynamic shared-memory limit once per device.
+cudaError_t ensure_smem_attr(const void* kernel, int bytes);
+int device_sm_count();
+
+// Sets the thread-local error text returned by rpa_last_error().
+void set_last_error(const char* fmt, ...);
+
+}  // namespace rpa

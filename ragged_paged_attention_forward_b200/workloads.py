@@ -313,11 +313,15 @@ def sparse(seed: int = 1005, poison: bool = True, kv_len: int = 131072, chunk: i
     batch = ragged_batch([kv_len], [chunk], 32, 8, 128, SPARSE_BLOCK, seed=seed,
                          layout=HEAD_MAJOR, poison=poison, keep_logical=keep_logical,
                          name="sparse")
+    return batch, sparse_mask(seed=seed, kv_len=kv_len, chunk=chunk)
+
+
+def sparse_mask(seed: int = 1005, kv_len: int = 131072, chunk: int = 2048) -> torch.Tensor:
+    """The block mask of the sparse chunked-prefill workload alone."""
     nqb = chunk // SPARSE_BLOCK
     nkb = math.ceil(kv_len / SPARSE_BLOCK)
-    mask = structured_block_mask(1, 32, 8, nqb, nkb, seed=seed + 1,
+    return structured_block_mask(1, 32, 8, nqb, nkb, seed=seed + 1,
                                  past_blocks=(kv_len - chunk) // SPARSE_BLOCK)
-    return batch, mask
 
 
 WORKLOADS = {

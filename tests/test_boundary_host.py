@@ -1,0 +1,153 @@
+"""The C ABI on the host: the library loads, exports every entry point that include/rpa.h
+declares, and rejects bad arguments before touching the device.  CPU only (no kernel runs:
+every call here returns before its first CUDA call)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from ragged_paged_attention_forward_b200 import api
+from ragged_paged_attention_forward_b200 import workloads as wl
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_functions():
+    src = open(os.path.join(ROOT, "include", "rpa.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(rpa_[a-z_]+)\s*\(", src)))
+
+
+def test_library_exports_every_declared_entry_point():
+    names = _declared_functions()
+    assert {"rpa_plan", "rpa_write_kv", "rpa_forward", "rpa_build_group_tables"} <= set(names)
+    L = ctypes.CDLL(api.LIB_PATH)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def _shape(**kw):
+    s = dict(num_seqs=2, num_tokens=2, num_q_heads=32, num_kv_heads=8, head_dim=128,
+             page_size=16, num_pages=100, max_blocks_per_seq=16, layout=0, causal=True,
+             cu_seqlens_q=[0, 1, 2], seq_lens_k=[40, 200])
+    s.update(kw)
+    return s
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(num_q_heads=30), api.RPA_ERR_SHAPE),
+    (dict(head_dim=96), api.RPA_ERR_UNSUPPORTED),
+    (dict(page_size=24), api.RPA_ERR_UNSUPPORTED),
+    (dict(page_size=8), api.RPA_ERR_UNSUPPORTED),
+    (dict(page_size=512), api.RPA_ERR_UNSUPPORTED),
+    (dict(seq_lens_k=[0, 200]), api.RPA_ERR_SHAPE),                    # q_len > kv_len
+    (dict(seq_lens_k=[40, 16 * 16 + 1]), api.RPA_ERR_SHAPE),           # too many pages
+    (dict(cu_seqlens_q=[0, 2, 1]), api.RPA_ERR_SHAPE),                 # decreasing
+    (dict(cu_seqlens_q=[1, 1, 2]), api.RPA_ERR_SHAPE),                 # cu[0] != 0
+    (dict(num_tokens=3), api.RPA_ERR_SHAPE),                           # cu[B] != T
+    (dict(layout=2), api.RPA_ERR_INVALID_ARG),
+    (dict(num_pages=0), api.RPA_ERR_SHAPE),
+    (dict(sparse=True), api.RPA_ERR_UNSUPPORTED),                      # sparse needs head-major
+    (dict(decode_split_keys=100), api.RPA_ERR_INVALID_ARG),
+    (dict(force_class=7), api.RPA_ERR_INVALID_ARG),
+])
+def test_plan_rejects(kw, status):
+    with pytest.raises(api.RPAError) as ei:
+        api.rpa_plan(**_shape(**kw))
+    assert ei.value.status == status
+    assert api.last_error() != ""
+
+
+def test_plan_classifies_and_sizes():
+    dec = wl.decode(num_seqs=8, keep_logical=False)
+    from tests.rpa_testing import plan_for
+    p = plan_for(dec)
+    info = p.info()
+    assert info.batch_class == api.CLASS_DECODE
+    assert info.num_prefill_tiles == 0 and info.num_decode_items >= 8
+    assert info.workspace_bytes == p.workspace_bytes > 0
+    split = info.decode_split_keys
+    assert split % 64 == 0
+    expect_items = sum(-(-kv // split) for kv in dec.kv_lens())
+    assert info.num_decode_items == expect_items
+    multi = sum(1 for kv in dec.kv_lens() if kv > split)
+    assert info.num_merge_rows == multi
+    assert info.launches_forward == 1 + (1 if multi else 0)
+
+    pf = wl.ragged_batch([300, 64], [300, 40], 8, 2, 64, 16, seed=1)
+    info = plan_for(pf).info()
+    assert info.batch_class == api.CLASS_PREFILL
+    assert info.num_prefill_tiles == 3 + 1 and info.num_decode_items == 0
+
+    mx = wl.ragged_batch([300, 64, 90], [300, 1, 3], 8, 2, 64, 16, seed=1)
+    info = plan_for(mx).info()
+    assert info.batch_class == api.CLASS_MIXED
+    assert info.num_prefill_tiles == 3
+    assert info.num_decode_items == 2    # q_len*G = 4 and 12 <= 16: decode kernel
+
+    forced = plan_for(mx, force_class=api.CLASS_PREFILL).info()
+    assert forced.num_decode_items == 0 and forced.num_prefill_tiles == 5
+
+
+def test_zero_tokens_is_a_no_op():
+    p = api.rpa_plan(**_shape(num_seqs=2, num_tokens=0, cu_seqlens_q=[0, 0, 0]))
+    fake = ctypes.c_void_p(1 << 20)
+    L = api.lib()
+    st = L.rpa_forward(p.handle, fake, None, None, fake, fake, fake, fake, fake, None, None,
+                       ctypes.c_float(0.1), fake, None, None, 0, None)
+    assert st == api.RPA_OK
+    st = L.rpa_write_kv(p.handle, None, None, fake, fake, fake, fake, fake, None, 0, None)
+    assert st == api.RPA_OK
+
+
+def _forward_status(plan, **over):
+    fake = 1 << 20
+    args = dict(q=fake, k_new=fake, v_new=fake, k_pool=fake, v_pool=fake, bt=fake, cu=fake,
+                kv=fake, gt=None, gc=None, scale=0.1, out=fake, lse=None, ws=fake,
+                ws_bytes=plan.workspace_bytes)
+    args.update(over)
+    P = lambda v: None if v is None else ctypes.c_void_p(v)
+    return api.lib().rpa_forward(plan.handle, P(args["q"]), P(args["k_new"]), P(args["v_new"]),
+                                 P(args["k_pool"]), P(args["v_pool"]), P(args["bt"]),
+                                 P(args["cu"]), P(args["kv"]), P(args["gt"]), P(args["gc"]),
+                                 ctypes.c_float(args["scale"]), P(args["out"]), P(args["lse"]),
+                                 P(args["ws"]), args["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(q=None), api.RPA_ERR_INVALID_ARG),
+    (dict(out=None), api.RPA_ERR_INVALID_ARG),
+    (dict(k_pool=None), api.RPA_ERR_INVALID_ARG),
+    (dict(q=(1 << 20) + 8), api.RPA_ERR_INVALID_ARG),          # misaligned
+    (dict(v_new=None), api.RPA_ERR_INVALID_ARG),               # k_new without v_new
+    (dict(gt=1 << 20, gc=1 << 20), api.RPA_ERR_INVALID_ARG),   # tables need head-major
+    (dict(gt=1 << 20), api.RPA_ERR_INVALID_ARG),               # table without count
+    (dict(ws_bytes=0), api.RPA_ERR_WORKSPACE_TOO_SMALL),
+    (dict(ws=None), api.RPA_ERR_WORKSPACE_TOO_SMALL),
+    (dict(ws=(1 << 20) + 16), api.RPA_ERR_INVALID_ARG),        # workspace not 256-aligned
+    (dict(scale=float("inf")), api.RPA_ERR_INVALID_ARG),
+])
+def test_forward_rejects_on_host(over, status):
+    p = api.rpa_plan(**_shape())
+    assert _forward_status(p, **over) == status
+
+
+def test_sparse_plan_requires_tables():
+    p = api.rpa_plan(**_shape(layout=1, sparse=True))
+    assert _forward_status(p) == api.RPA_ERR_INVALID_ARG          # tables missing
+    p2 = api.rpa_plan(**_shape(layout=1))
+    assert _forward_status(p2, gt=1 << 20, gc=1 << 20) == api.RPA_ERR_INVALID_ARG
+
+
+def test_group_table_builder_rejects():
+    L = api.lib()
+    assert L.rpa_build_group_tables(None, 1, 6, 4, 1, 1, None, None, None) == api.RPA_ERR_SHAPE
+    assert L.rpa_build_group_tables(None, 1, 4, 2, 1, 70000, None, None,
+                                    None) == api.RPA_ERR_UNSUPPORTED
+    assert L.rpa_build_group_tables(None, 0, 4, 2, 1, 4, None, None, None) == api.RPA_OK
+
+
+def test_status_strings():
+    for code in range(-6, 1):
+        assert api.status_string(code).startswith("RPA_")
