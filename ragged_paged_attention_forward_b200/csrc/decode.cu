@@ -45,9 +45,14 @@ struct DecodeGeom {
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kStages * kTensorStageBytes;
   static constexpr int kPagesOff = 2 * kStages * kTensorStageBytes;
-  static constexpr int kBarOff = kPagesOff + kMaxItemPages * 4 + 64;
+  static constexpr int kBarOff = (kPagesOff + kMaxItemPages * 4 + 127) / 128 * 128;
   static constexpr int kBytes = kBarOff + 2 * kStages * 8 + 16;
   static constexpr int kAlloc = kBytes + 1024;  // room to align the base to 1024
+  // TMA destinations with 128-byte swizzle start on 1024-byte boundaries; mbarriers need 8.
+  static_assert(kKOff % 1024 == 0 && kVOff % 1024 == 0 && kTensorStageBytes % 1024 == 0,
+                "stage alignment");
+  static_assert(kHalfBytes % 1024 == 0, "half-tile alignment");
+  static_assert(kBarOff % 8 == 0, "mbarrier alignment");
 };
 
 struct alignas(16) U4 {
@@ -187,7 +192,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     const int vr = warp * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;  // V ldmatrix.trans row
     for (int s = 0; s < nstages; ++s) {
       const int slot = s % Geo::kStages;
-      if (!wait_bounded(&full[slot], (s / Geo::kStages) & 1, abort_flag, p.err, kErrDecodeWait))
+      if (!warp_wait_bounded(&full[slot], (s / Geo::kStages) & 1, abort_flag, p.err,
+                             kErrDecodeWait))
         break;
       const int key0 = it.k_begin + s * Geo::kStageKeys + warp * 16;
       if (key0 < it.k_end) {

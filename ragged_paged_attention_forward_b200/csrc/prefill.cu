@@ -1,13 +1,467 @@
-// Tensor-core (tcgen05/TMEM) paged prefill kernel.
+// Causal paged prefill on the 5th-generation tensor cores (tcgen05 + TMEM), fed by TMA through
+// the block table; also the sparse mode that walks per-group block tables.
+//
+// What it computes: for a tile of 128 query tokens of one sequence and one query head, exact
+// softmax attention over the keys the tokens may see -- 0 .. past + i when causal (bottom-right
+// alignment: "[WebGPU] Optimized PagedAttention implementation (2/n)", commit "FlashAttention:
+// optional seqlens_q input"), restricted in sparse mode to the KV blocks listed in the table of
+// the head's KV group ("CompactAttention: Accelerating Chunked Prefill with Block-Union KV
+// Selection", Fig. 3: the paged kernel reads the selected pages in place).  This is the fused
+// paged prefill of the WebGPU page ("What's shipped": FlashAttentionPagedPrefillProgram, one
+// block-table lookup per K/V tile) and the prefill specialisation of "Ragged Paged Attention:
+// A High-Performance and Flexible LLM Inference Kernel for TPU" (Key ideas).
+//
+// B200 design (one CTA per (query tile, query head), 256 threads):
+//   warp 0     TMA producer: Q once, then K and V tiles of 128 keys, page by page (boxes of
+//              [min(P,128) slots x 64 dims], 128-byte swizzle) into a 2-stage ring;
+//   warp 1     allocates TMEM; lane 0 issues the MMAs:
+//                S_j = Q K_j^T   (M=128 queries, N=128 keys, K=D; A,B from shared memory)
+//                O  += P_j V_j   (M=128, N=D, K=128 keys; A = P_j from TMEM, B = V_j MN-major)
+//              S is double-buffered in TMEM so S_{j+1} runs while the softmax works on S_j;
+//              the warp zeroes V rows past the last real key before P_j V_j;
+//   warps 4-7  softmax: thread r owns query row r (TMEM lane r): loads S_j, masks, online
+//              softmax in fp32 (exp2), writes P_j as bf16 over S_j, rescales O in TMEM, and
+//              finally normalises O and stores the bf16 row and its log-sum-exp.
+// TMEM columns: S0 [0,128) S1 [128,256) O [256,256+D).  Every wait is bounded.
+#include <cuda_bf16.h>
+#include <math_constants.h>
+
+#include "ptx.cuh"
 #include "rpa_internal.h"
 
 namespace rpa {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kStagesPF = 2;
+constexpr int kRows = kPrefillTileRows;  // 128
+constexpr int kKeys = kPrefillTileKeys;  // 128
+constexpr uint32_t kTmemCols = 512;
+
+template <int D>
+struct PfGeom {
+  static constexpr int kHalves = D / 64;
+  static constexpr int kHalfBytes = 128 * 128;             // 128 rows x 128 B
+  static constexpr int kTileBytes = kHalves * kHalfBytes;  // Q, K or V tile
+  static constexpr int kQOff = 0;
+  static constexpr int kKOff = kTileBytes;
+  static constexpr int kVOff = kKOff + kStagesPF * kTileBytes;
+  static constexpr int kBarOff = kVOff + kStagesPF * kTileBytes;
+  // q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_ready, o_done, mma_done
+  static constexpr int kNumBars = 1 + 3 * kStagesPF + 2 + 3;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kBytes = kMiscOff + 64;
+  // at least 120 KB so that a second CTA never shares the SM (and its 512 TMEM columns)
+  static constexpr int kAlloc = kBytes + 1024 > 120 * 1024 ? kBytes + 1024 : 120 * 1024;
+  static_assert(kKOff % 1024 == 0 && kVOff % 1024 == 0 && kTileBytes % 1024 == 0,
+                "TMA destinations with 128-byte swizzle start on 1024-byte boundaries");
+  static_assert(kBarOff % 8 == 0 && kMiscOff % 8 == 0, "mbarrier alignment");
+};
+
+struct alignas(16) U4 {
+  uint32_t x, y, z, w;
+};
+
+// Key tiles: dense tiles are 128 consecutive positions; in sparse mode a tile holds the next
+// 128/P entries of the block-union table (ascending logical blocks of P keys).
+struct KeyMap {
+  const int32_t* table;  // sparse: ascending logical block ids, or null when dense
+  int n_entries;         // sparse: entries whose block starts before the visible limit
+  int P;
+  int log2P;
+};
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+    prefill_kernel(const __grid_constant__ CUtensorMap qmap,
+                   const __grid_constant__ CUtensorMap kmap,
+                   const __grid_constant__ CUtensorMap vmap, PrefillLaunch p) {
+  using Geo = PfGeom<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* Qs = smem + Geo::kQOff;
+  uint8_t* Ks = smem + Geo::kKOff;
+  uint8_t* Vs = smem + Geo::kVOff;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Geo::kBarOff);
+  uint64_t* q_full = bars;
+  uint64_t* k_full = bars + 1;
+  uint64_t* v_full = k_full + kStagesPF;
+  uint64_t* kv_empty = v_full + kStagesPF;
+  uint64_t* s_full = kv_empty + kStagesPF;  // [2]
+  uint64_t* p_ready = s_full + 2;
+  uint64_t* o_done = p_ready + 1;
+  uint64_t* mma_done = o_done + 1;
+  uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(smem + Geo::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Geo::kMiscOff + 8);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int Hq = p.num_q_heads;
+  const int tile_idx = blockIdx.x / Hq;
+  const int hq = blockIdx.x - tile_idx * Hq;
+  const PrefillTile tile = p.tiles[tile_idx];
+  const int G = Hq / p.num_kv_heads;
+  const int h = hq / G;
+  const int P = p.kv.page_size;
+  const int log2P = p.kv.log2_page;
+  const int past = tile.kv_len - tile.q_len;
+  const int q_end = min(tile.q_len, tile.q_start + kRows);  // local, exclusive
+  const int kv_hi = p.causal ? min(tile.kv_len, past + q_end) : tile.kv_len;
+
+  KeyMap km;
+  km.table = nullptr;
+  km.n_entries = 0;
+  km.P = P;
+  km.log2P = log2P;
+  int n_tiles;
+  if (p.group_table) {
+    const size_t row = (size_t)tile.seq * p.num_kv_heads + h;
+    km.table = p.group_table + row * p.kv.max_blocks;
+    const int cnt = min(__ldg(p.group_count + row), p.kv.max_blocks);
+    int lo = 0, hi = max(cnt, 0);  // entries whose block starts before kv_hi (ascending table)
+    while (lo < hi) {
+      const int mid = (lo + hi) >> 1;
+      if ((__ldg(km.table + mid) << log2P) < kv_hi) lo = mid + 1; else hi = mid;
+    }
+    km.n_entries = lo;
+    const int per = kKeys >> log2P;
+    n_tiles = (km.n_entries + per - 1) / per;
+  } else {
+    n_tiles = (kv_hi + kKeys - 1) / kKeys;
+  }
+
+  if (threadIdx.x == 0) {
+    mbar_init(q_full, 1);
+    for (int s = 0; s < kStagesPF; ++s) {
+      mbar_init(&k_full[s], 1);
+      mbar_init(&v_full[s], 1);
+      mbar_init(&kv_empty[s], 1);
+    }
+    mbar_init(&s_full[0], 1);
+    mbar_init(&s_full[1], 1);
+    mbar_init(p_ready, 128);
+    mbar_init(o_done, 1);
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_sh;
+  const uint32_t tmem_o = tmem + 256;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ TMA producer
+    if (lane == 0 && n_tiles > 0) {
+      tma_prefetch_desc(&qmap);
+      tma_prefetch_desc(&kmap);
+      tma_prefetch_desc(&vmap);
+      mbar_arrive_expect_tx(q_full, Geo::kTileBytes);
+#pragma unroll
+      for (int half = 0; half < Geo::kHalves; ++half)
+        tma_load_3d(Qs + half * Geo::kHalfBytes, &qmap, half * 64, hq, tile.t0 + tile.q_start,
+                    q_full);
+      const int32_t* bt_row =
+          p.kv.layout == 0
+              ? p.kv.block_table + (size_t)tile.seq * p.kv.max_blocks
+              : p.kv.block_table + ((size_t)tile.seq * p.kv.num_kv_heads + h) * p.kv.max_blocks;
+      const int hcoord = p.kv.layout == 0 ? h : 0;
+      const int box_rows = P < kKeys ? P : kKeys;
+      const uint32_t box_bytes = (uint32_t)box_rows * 128u * Geo::kHalves;
+      int issued = 0;
+      for (int j = 0; j < n_tiles; ++j) {
+        const int slot = j % kStagesPF;
+        if (j >= kStagesPF && !wait_bounded(&kv_empty[slot], ((j / kStagesPF) - 1) & 1,
+                                            abort_flag, p.err, kErrPrefillWait))
+          break;
+        // boxes of tile j: (page, first slot in the page, destination row in the tile)
+        int nbox, first_blk = 0, slot0 = 0;
+        if (km.table) {
+          nbox = min(kKeys >> log2P, km.n_entries - j * (kKeys >> log2P));
+        } else if (P >= kKeys) {
+          nbox = 1;
+          first_blk = (j * kKeys) >> log2P;
+          slot0 = (j * kKeys) & (P - 1);
+        } else {
+          first_blk = (j * kKeys) >> log2P;
+          nbox = ((min(j * kKeys + kKeys, kv_hi) - 1) >> log2P) - first_blk + 1;
+        }
+        mbar_arrive_expect_tx(&k_full[slot], box_bytes * nbox);
+        mbar_arrive_expect_tx(&v_full[slot], box_bytes * nbox);
+        for (int i = 0; i < nbox; ++i) {
+          const int blk = km.table ? __ldg(km.table + j * (kKeys >> log2P) + i) : first_blk + i;
+          int page = -1;  // out-of-range coordinates make TMA fill zeros: no stray access
+          if (blk >= 0 && blk < p.kv.max_blocks)
+            page = __ldg(bt_row + blk);
+          else
+            atomicOr(p.err, kErrBadIndex);
+          const int drow = i * box_rows;
+#pragma unroll
+          for (int half = 0; half < Geo::kHalves; ++half) {
+            const int off = slot * Geo::kTileBytes + half * Geo::kHalfBytes + drow * 128;
+            tma_load_4d(Ks + off, &kmap, half * 64, hcoord, slot0, page, &k_full[slot]);
+            tma_load_4d(Vs + off, &vmap, half * 64, hcoord, slot0, page, &v_full[slot]);
+          }
+        }
+        ++issued;
+      }
+      if (*abort_flag) {  // let copies in flight land before shared memory goes away
+        wait_bounded(q_full, 0, abort_flag, nullptr, 0, kWaitTimeoutNs / 8);
+        for (int j = max(0, issued - kStagesPF); j < issued; ++j) {
+          wait_bounded(&k_full[j % kStagesPF], (j / kStagesPF) & 1, abort_flag, nullptr, 0,
+                       kWaitTimeoutNs / 8);
+          wait_bounded(&v_full[j % kStagesPF], (j / kStagesPF) & 1, abort_flag, nullptr, 0,
+                       kWaitTimeoutNs / 8);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (n_tiles > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKeys, false, false);
+      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+      const uint32_t q_addr = smem_u32(Qs);
+      bool ok = warp_wait_bounded(q_full, 0, abort_flag, p.err, kErrPrefillWait);
+      auto issue_s = [&](int j) -> bool {
+        const int slot = j % kStagesPF;
+        if (!warp_wait_bounded(&k_full[slot], (j / kStagesPF) & 1, abort_flag, p.err,
+                               kErrPrefillWait))
+          return false;
+        if (lane == 0) {
+          tc_fence_after();
+          const uint32_t k_addr = smem_u32(Ks + slot * Geo::kTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * Geo::kHalfBytes + (kk & 3) * 32;
+            umma_ss(tmem + (j & 1) * 128, smem_desc_sw128(q_addr + off, 16, 1024),
+                    smem_desc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          }
+          umma_commit(&s_full[j & 1]);
+        }
+        __syncwarp();
+        return true;
+      };
+      if (ok) ok = issue_s(0);
+      for (int j = 0; ok && j < n_tiles; ++j) {
+        if (j + 1 < n_tiles && !issue_s(j + 1)) break;
+        const int slot = j % kStagesPF;
+        if (!warp_wait_bounded(&v_full[slot], (j / kStagesPF) & 1, abort_flag, p.err,
+                               kErrPrefillWait))
+          break;
+        // V rows past the last real key may hold anything (NaN tail slots, a stale tile):
+        // P = 0 there does not cancel a NaN in the product, so the rows are zeroed.
+        int nvalid;
+        if (km.table) {
+          const int per = kKeys >> log2P;
+          const int ne = min(per, km.n_entries - j * per);
+          const int last = __ldg(km.table + j * per + ne - 1);
+          nvalid = (ne - 1) * P + min(P, tile.kv_len - (last << log2P));
+        } else {
+          const int covered = min(tile.kv_len, ((kv_hi + P - 1) >> log2P) << log2P);
+          nvalid = min(kKeys, covered - j * kKeys);
+        }
+        if (nvalid < kKeys) {
+          uint8_t* vt = Vs + slot * Geo::kTileBytes;
+          const int n16 = (kKeys - nvalid) * Geo::kHalves * 8;
+          for (int i = lane; i < n16; i += 32) {
+            const int row = nvalid + i / (Geo::kHalves * 8);
+            const int rem = i % (Geo::kHalves * 8);
+            *reinterpret_cast<U4*>(vt + (rem >> 3) * Geo::kHalfBytes + row * 128 +
+                                   (rem & 7) * 16) = U4{0, 0, 0, 0};
+          }
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
+        if (!warp_wait_bounded(p_ready, j & 1, abort_flag, p.err, kErrPrefillWait)) break;
+        if (lane == 0) {
+          tc_fence_after();
+          const uint32_t v_addr = smem_u32(Vs + slot * Geo::kTileBytes);
+#pragma unroll
+          for (int kk = 0; kk < kKeys / 16; ++kk)
+            umma_ts(tmem_o, tmem + (j & 1) * 128 + kk * 8,
+                    smem_desc_sw128(v_addr + kk * 2048, Geo::kHalfBytes, 1024), idesc_o,
+                    (j > 0 || kk > 0) ? 1u : 0u);
+          umma_commit(o_done);
+          umma_commit(&kv_empty[slot]);
+        }
+        __syncwarp();
+      }
+      // every MMA issued so far must finish before TMEM is released
+      if (lane == 0) umma_commit(mma_done);
+      __syncwarp();
+      warp_wait_bounded(mma_done, 0, abort_flag, nullptr, 0, kWaitTimeoutNs / 8);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------------ softmax
+    const int r = (warp - 4) * 32 + lane;  // query row == TMEM lane
+    const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+    const int q_local = tile.q_start + r;
+    const int pos = past + q_local;        // absolute position of this row
+    const int lim = p.causal ? min(tile.kv_len, pos + 1) : tile.kv_len;
+    const float sc = p.scale_log2;
+    float m = -CUDART_INF_F, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_tiles; ++j) {
+      const uint32_t ts = tmem + (j & 1) * 128 + lane_off;
+      if (!warp_wait_bounded(&s_full[j & 1], (j >> 1) & 1, abort_flag, p.err,
+                             kErrPrefillWait)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      uint32_t sr[kKeys];
+#pragma unroll
+      for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(ts + c * 32, sr + c * 32);
+      tmem_wait_ld();
+      // first key position of each column group: dense -> j*128; sparse -> lane e holds the
+      // start of the tile's e-th table block (missing entries map past every limit)
+      int ent = j * kKeys;
+      int tile_last;  // last key position the tile may hold
+      bool partial = false;
+      if (km.table) {
+        const int per = kKeys >> log2P;
+        const int e0 = j * per;
+        const int ne = min(per, km.n_entries - e0);
+        ent = 0x3fff0000;
+        if (lane < ne) ent = __ldg(km.table + e0 + lane) << log2P;
+        tile_last = __shfl_sync(0xffffffffu, ent, ne - 1) + P - 1;
+        partial = ne < per;
+      } else {
+        tile_last = j * kKeys + kKeys - 1;
+      }
+      const bool need_mask = partial || tile_last >= tile.kv_len ||
+                             (p.causal && tile_last > past + tile.q_start);
+      float mx = -CUDART_INF_F;
+      if (need_mask) {
+#pragma unroll
+        for (int c = 0; c < kKeys; ++c) {
+          const int kp = km.table ? __shfl_sync(0xffffffffu, ent, c >> log2P) + (c & (P - 1))
+                                  : ent + c;
+          const float v = kp < lim ? __uint_as_float(sr[c]) * sc : -CUDART_INF_F;
+          sr[c] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < kKeys; ++c) {
+          const float v = __uint_as_float(sr[c]) * sc;
+          sr[c] = __float_as_uint(v);
+          mx = fmaxf(mx, v);
+        }
+      }
+      const float m_new = fmaxf(m, mx);
+      const float m_use = m_new == -CUDART_INF_F ? 0.f : m_new;
+      const float alpha = fast_exp2(m - m_use);
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < kKeys; c += 2) {
+        const float p0 = fast_exp2(__uint_as_float(sr[c]) - m_use);
+        const float p1 = fast_exp2(__uint_as_float(sr[c + 1]) - m_use);
+        rs += p0 + p1;
+        sr[c >> 1] = pack_bf16(p0, p1);  // P_j as bf16 pairs, over the consumed S values
+      }
+      l = l * alpha + rs;
+      m = m_new;
+#pragma unroll
+      for (int c = 0; c < kKeys / 64; ++c) tmem_st32(ts + c * 32, sr + c * 32);
+      if (j > 0) {
+        // O += P_{j-1} V_{j-1} must be complete before O is rescaled
+        if (!warp_wait_bounded(o_done, (j - 1) & 1, abort_flag, p.err, kErrPrefillWait)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tmem_o + lane_off + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
+            tmem_st32(tmem_o + lane_off + c * 32, o);
+          }
+        }
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(p_ready);
+    }
+    // ---- epilogue: O / l -> bf16 (a row that saw no key gets 0 and lse = -inf)
+    if (ok && n_tiles > 0) {
+      ok = warp_wait_bounded(o_done, (n_tiles - 1) & 1, abort_flag, p.err, kErrPrefillWait);
+      tc_fence_after();
+    }
+    if (ok) {
+      const int t = tile.t0 + q_local;
+      const bool write = q_local < tile.q_len;
+      uint16_t* orow = p.out + ((size_t)t * Hq + hq) * D;
+      const float inv = l > 0.f ? 1.f / l : 0.f;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t o[32];
+        if (n_tiles > 0) {
+          tmem_ld32(tmem_o + lane_off + c * 32, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) o[i] = 0u;
+        }
+        if (write) {
+#pragma unroll
+          for (int i = 0; i < 32; i += 8) {
+            U4 v;
+            v.x = pack_bf16(__uint_as_float(o[i + 0]) * inv, __uint_as_float(o[i + 1]) * inv);
+            v.y = pack_bf16(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+            v.z = pack_bf16(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+            v.w = pack_bf16(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+            *reinterpret_cast<U4*>(orow + c * 32 + i) = v;
+          }
+        }
+      }
+      if (write && p.lse)
+        p.lse[(size_t)t * Hq + hq] =
+            l > 0.f ? (m + fast_log2(l)) * 0.69314718055994531f : -CUDART_INF_F;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace
 
 cudaError_t launch_prefill(const PrefillLaunch& p, cudaStream_t stream) {
-  (void)stream;
   if (p.num_tiles <= 0) return cudaSuccess;
-  set_last_error("prefill kernel not built yet");
-  return cudaErrorNotSupported;
+  CUtensorMap qmap, kmap, vmap;
+  cudaError_t e = encode_q_map(&qmap, p.q, p.num_tokens, p.num_q_heads, p.head_dim, kRows);
+  if (e != cudaSuccess) return e;
+  e = encode_kv_map(&kmap, p.kv.k_pool, p.kv, p.head_dim, kKeys);
+  if (e != cudaSuccess) return e;
+  e = encode_kv_map(&vmap, p.kv.v_pool, p.kv, p.head_dim, kKeys);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)p.num_tiles * (unsigned)p.num_q_heads);
+  if (p.head_dim == 128) {
+    e = ensure_smem_attr(reinterpret_cast<const void*>(prefill_kernel<128>),
+                         PfGeom<128>::kAlloc);
+    if (e != cudaSuccess) return e;
+    prefill_kernel<128><<<grid, kThreads, PfGeom<128>::kAlloc, stream>>>(qmap, kmap, vmap, p);
+  } else {
+    e = ensure_smem_attr(reinterpret_cast<const void*>(prefill_kernel<64>), PfGeom<64>::kAlloc);
+    if (e != cudaSuccess) return e;
+    prefill_kernel<64><<<grid, kThreads, PfGeom<64>::kAlloc, stream>>>(qmap, kmap, vmap, p);
+  }
+  return cudaGetLastError();
 }
 
 }  // namespace rpa

@@ -1,0 +1,201 @@
+"""GPU parity of the tensor-core (tcgen05/TMEM) paged prefill path, the mixed batches and the
+sparse block-union mode against the fp64 oracle, through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import rpa_oracle as orc
+from ragged_paged_attention_forward_b200 import api
+from ragged_paged_attention_forward_b200 import workloads as wl
+from tests.rpa_testing import (assert_close, assert_lse_close, oracle_forward, run_forward)
+
+pytestmark = pytest.mark.gpu
+
+
+def _sample_rows(batch, n, seed):
+    g = np.random.default_rng(seed)
+    T, Hq = batch.num_tokens, batch.num_q_heads
+    rows = {(int(t), int(h)) for t, h in zip(g.integers(0, T, n), g.integers(0, Hq, n))}
+    # always include each sequence's first and last token
+    cu = batch.cu_seqlens_q.tolist()
+    for b in range(batch.num_seqs):
+        if cu[b + 1] > cu[b]:
+            rows.add((cu[b], int(g.integers(0, Hq))))
+            rows.add((cu[b + 1] - 1, int(g.integers(0, Hq))))
+    return sorted(rows)
+
+
+def test_prefill_small_no_past():
+    b = wl.ragged_batch([200, 64], [200, 64], 8, 2, 128, 64, seed=51)
+    ref, ref_lse, kp, vp = oracle_forward(b)
+    out, lse, gk, gv, plan = run_forward(b)
+    assert plan.info().batch_class == api.CLASS_PREFILL
+    assert_close(out, ref)
+    assert_lse_close(lse, ref_lse)
+    assert np.array_equal(orc.bits16(gk), kp) and np.array_equal(orc.bits16(gv), vp)
+
+
+@pytest.mark.parametrize("page", [16, 32, 64, 128, 256])
+def test_chunked_prefill_with_past(page):
+    b = wl.ragged_batch([430, 170, 1000], [130, 40, 257], 8, 2, 128, page, seed=52 + page)
+    ref, ref_lse, _, _ = oracle_forward(b)
+    out, lse, _, _, plan = run_forward(b)
+    assert plan.info().num_prefill_tiles > 0
+    assert_close(out, ref)
+    assert_lse_close(lse, ref_lse)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+@pytest.mark.parametrize("Hq,Hkv", [(4, 4), (8, 2), (8, 1)])
+def test_prefill_heads_and_dims(D, Hq, Hkv):
+    b = wl.ragged_batch([300, 129], [150, 129], Hq, Hkv, D, 16, seed=53 + D + Hq)
+    ref, ref_lse, _, _ = oracle_forward(b)
+    out, lse, _, _, _ = run_forward(b)
+    assert_close(out, ref)
+    assert_lse_close(lse, ref_lse)
+
+
+def test_varlen_regression_case_forced_on_tensor_cores():
+    # B=2, q_lens (32, 16), head size 128, MHA (the fused varlen prefill regression shape of
+    # the WebGPU page's test list) -- every row through the tensor-core kernel
+    b = wl.ragged_batch([32, 16], [32, 16], 4, 4, 128, 16, seed=54)
+    ref, ref_lse, _, _ = oracle_forward(b)
+    out, lse, _, _, plan = run_forward(b, plan_opts=dict(force_class=api.CLASS_PREFILL))
+    assert plan.info().num_decode_items == 0
+    assert_close(out, ref)
+    assert_lse_close(lse, ref_lse)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_mixed_q_len_with_past(causal):
+    # the failing WebGPU case: mixed q_len with past > 0
+    b = wl.ragged_batch([16, 40, 300, 77, 1000], [16, 4, 300, 1, 33], 4, 2, 128, 16, seed=55,
+                        causal=causal)
+    ref, ref_lse, _, _ = oracle_forward(b)
+    out, lse, _, _, plan = run_forward(b)
+    info = plan.info()
+    assert info.batch_class == api.CLASS_MIXED
+    assert info.num_prefill_tiles > 0 and info.num_decode_items > 0
+    assert_close(out, ref)
+    assert_lse_close(lse, ref_lse)
+    forced = run_forward(b, plan_opts=dict(force_class=api.CLASS_PREFILL))
+    assert_close(forced[0], ref)
+
+
+@pytest.mark.parametrize("scale", [0.0, 0.02, -0.09])
+def test_prefill_explicit_scale(scale):
+    b = wl.ragged_batch([260], [200], 4, 2, 64, 64, seed=56)
+    ref, ref_lse, _, _ = oracle_forward(b, scale=scale)
+    out, lse, _, _, _ = run_forward(b, scale=scale)
+    assert_close(out, ref)
+    assert_lse_close(lse, ref_lse)
+
+
+def test_prefill_head_major_equals_seq_major():
+    b = wl.ragged_batch([333, 128], [200, 128], 8, 2, 128, 64, seed=57)
+    o1 = run_forward(b)[0]
+    o2 = run_forward(wl.to_head_major(b))[0]
+    ref, _, _, _ = oracle_forward(b)
+    assert_close(o1, ref)
+    assert_close(o2, ref)
+
+
+def test_prefill_page_permutation_gives_identical_output():
+    b = wl.ragged_batch([500, 260], [300, 260], 8, 2, 128, 16, seed=58)
+    o1 = run_forward(b)[0]
+    o2 = run_forward(wl.permute_pages(b, seed=3))[0]
+    assert torch.equal(o1, o2)
+
+
+def test_prefill_config_full_size_sampled():
+    b = wl.prefill()
+    out, lse, gk, gv, plan = run_forward(b)
+    assert plan.info().batch_class == api.CLASS_PREFILL
+    rows = _sample_rows(b, 96, seed=1)
+    ref, ref_lse, kp, vp = oracle_forward(b, rows=rows)
+    assert_close(out, ref, rows=rows)
+    assert_lse_close(lse, ref_lse, rows=rows)
+    assert np.array_equal(orc.bits16(gk), kp) and np.array_equal(orc.bits16(gv), vp)
+    assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("shuffle", [False, True])
+def test_mixed_config_full_size_sampled(shuffle):
+    b = wl.mixed(shuffle=shuffle)
+    out, lse, _, _, plan = run_forward(b)
+    info = plan.info()
+    assert info.num_prefill_tiles > 0 and info.num_decode_items > 0
+    rows = _sample_rows(b, 96, seed=2)
+    # every decode row too (one head each)
+    cu = b.cu_seqlens_q.tolist()
+    rows = sorted(set(rows) | {(cu[i], i % 32) for i in range(b.num_seqs)
+                                if cu[i + 1] - cu[i] == 1})
+    ref, ref_lse, _, _ = oracle_forward(b, rows=rows)
+    assert_close(out, ref, rows=rows)
+    assert_lse_close(lse, ref_lse, rows=rows)
+    assert torch.isfinite(out.float()).all()
+
+
+# ------------------------------------------------------------------ sparse block-union mode
+
+def _sparse_case(kv_len, chunk, page, seed, density=None, Hq=8, Hkv=2, D=128):
+    b = wl.ragged_batch([kv_len], [chunk], Hq, Hkv, D, page, seed=seed, layout=wl.HEAD_MAJOR)
+    nqb = -(-chunk // page)
+    nkb = b.max_blocks
+    if density is None:
+        mask = wl.structured_block_mask(1, Hq, Hkv, nqb, nkb, seed=seed + 1,
+                                        past_blocks=(kv_len - chunk) // page)
+    else:
+        mask = wl.iid_block_mask(1, Hq, nqb, nkb, seed=seed + 1, density=density)
+    table, count = orc.build_group_tables(mask, Hkv)
+    return b, torch.from_numpy(table), torch.from_numpy(count)
+
+
+@pytest.mark.parametrize("page", [16, 64, 128])
+def test_sparse_small(page):
+    b, table, count = _sparse_case(1500, 300, page, seed=60 + page)
+    ref, ref_lse, _, _ = oracle_forward(b, group_table=table.numpy(), group_count=count.numpy())
+    out, lse, _, _, plan = run_forward(b, group_table=table, group_count=count)
+    assert plan.info().num_decode_items == 0
+    assert_close(out, ref)
+    assert_lse_close(lse, ref_lse)
+
+
+def test_sparse_all_ones_equals_dense():
+    b, table, count = _sparse_case(900, 200, 64, seed=61, density=1.0)
+    dense = run_forward(b)[0]
+    sp = run_forward(b, group_table=table, group_count=count)[0]
+    ref, _, _, _ = oracle_forward(b)
+    assert_close(dense, ref)
+    assert_close(sp, ref)
+
+
+def test_sparse_rows_without_visible_blocks():
+    b = wl.ragged_batch([256], [256], 4, 1, 64, 64, seed=62, layout=wl.HEAD_MAJOR)
+    mask = np.zeros((1, 4, 4, 4), dtype=np.uint8)
+    mask[..., 2:] = 1             # rows before position 128 see nothing
+    table, count = orc.build_group_tables(mask, 1)
+    ref, ref_lse, _, _ = oracle_forward(b, group_table=table, group_count=count)
+    out, lse, _, _, _ = run_forward(b, group_table=torch.from_numpy(table),
+                                    group_count=torch.from_numpy(count))
+    assert torch.all(out[:128] == 0)
+    assert torch.all(torch.isneginf(lse[:128]))
+    assert_close(out, ref)
+    assert_lse_close(lse, ref_lse)
+
+
+def test_sparse_config_full_size_sampled():
+    b, mask = wl.sparse()
+    m = mask.cuda()
+    nkb = mask.shape[-1]
+    table = torch.empty(1, 8, nkb, dtype=torch.int32, device="cuda")
+    count = torch.empty(1, 8, dtype=torch.int32, device="cuda")
+    api.rpa_build_group_tables(m, 8, table, count)
+    torch.cuda.synchronize()
+    rt, rc = orc.build_group_tables(mask, 8)
+    assert np.array_equal(table.cpu().numpy(), rt) and np.array_equal(count.cpu().numpy(), rc)
+    out, lse, _, _, _ = run_forward(b, group_table=table, group_count=count)
+    rows = _sample_rows(b, 24, seed=3)
+    ref, ref_lse, _, _ = oracle_forward(b, group_table=rt, group_count=rc, rows=rows)
+    assert_close(out, ref, rows=rows)
+    assert_lse_close(lse, ref_lse, rows=rows)
