@@ -1,0 +1,643 @@
+#!/usr/bin/env python
+"""Benchmark of ragged paged attention on B200 through the library's C ABI.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload decode|prefill|mixed|sparse] [--no-secondary]
+
+A step is one pass of the whole hot path over one synthetic batch: the fused call
+(KV-cache write + attention, with the decode splits merged), plus the block-union table
+build for the sparse workload.  Inputs are resident in HBM; L2 (126 MB) is flushed with a
+256 MB write before every timed step and the flush is not timed.  Each step is timed with
+CUDA events on the stream the kernels run on.  The headline line is the decode workload
+(Llama-3-8B attention, batch 64, kv_len ~ U[512, 8192]) in HBM GB/s; the prefill, mixed and
+sparse workloads are reported as secondary objects on the same line.
+
+Multi-GPU (torchrun, one process per GPU): every rank runs its own independent batch (a
+different seed) with no collective on the data path -- weak scaling; the elapsed time is the
+max over ranks.  ``--impl reference`` times the fp64 CPU oracle instead, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "paged-attn decode HBM GB/s (% peak) + prefill TFLOP/s (% bf16 peak), 1×B200"
+
+WORKLOAD_TEXT = {
+    "decode": "decode-only Llama-3-8B attention: batch 64, q_len=1, Hq=32, Hkv=8, D=128, "
+              "page_size=16, kv_len uniform 512-8192, bf16 N(0,1), shuffled pages, 1 new K/V "
+              "token written per seq",
+    "prefill": "prefill-only: 4 seqs x 4096 prompt tokens, causal, Hq=32, Hkv=8, D=128, "
+               "page_size=64, bf16 N(0,1), new K/V for all 16384 tokens scattered into "
+               "shuffled pages",
+    "mixed": "mixed continuous batch (token budget 2048): 48 decode seqs (kv_len 1024-16384 "
+             "uniform) + 2 prefill chunks of 512+976 tokens with prior context 1024 and 8192; "
+             "Hq=32, Hkv=8, D=128, page 16, bf16",
+    "sparse": "sparse chunked prefill: 1 seq, 2048-query chunk at 128K context, Hq=32, Hkv=8, "
+              "D=128, KV-head-major pages of 64, random 64x64 per-head block masks keeping "
+              "~25% blocks, Q-block+intra-group union tables",
+}
+
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------------------------
+# Algorithmic work (bytes that must move, flops that must be done) per workload
+# ------------------------------------------------------------------------------------
+
+def visible_pairs(batch, table=None, count=None):
+    """Sum over query rows of the number of keys each row sees, per query head."""
+    cu = batch.cu_seqlens_q.tolist()
+    kv = batch.kv_lens()
+    total = 0
+    if table is None:
+        for b in range(batch.num_seqs):
+            q_len = cu[b + 1] - cu[b]
+            past = kv[b] - q_len
+            if batch.causal:
+                total += q_len * past + q_len * (q_len + 1) // 2
+            else:
+                total += q_len * kv[b]
+        return total * batch.num_q_heads
+    G = batch.num_q_heads // batch.num_kv_heads
+    P = batch.page_size
+    for b in range(batch.num_seqs):
+        q_len = cu[b + 1] - cu[b]
+        past = kv[b] - q_len
+        pos = past + np.arange(q_len)
+        for g in range(batch.num_kv_heads):
+            blocks = np.asarray(table[b, g, :int(count[b, g])], dtype=np.int64)
+            starts = blocks * P
+            ends = np.minimum(starts + P, kv[b])
+            # keys of block k visible to position p: clip(p + 1 - start, 0, end - start)
+            vis = np.clip(pos[:, None] + 1 - starts[None, :], 0, (ends - starts)[None, :])
+            total += int(vis.sum()) * G
+    return total
+
+
+def work(batch, table=None, count=None):
+    D, Hq, Hkv = batch.head_dim, batch.num_q_heads, batch.num_kv_heads
+    T = batch.num_tokens
+    el = 2  # bf16
+    pairs = visible_pairs(batch, table, count)
+    flops = 4.0 * D * pairs
+    q_o = 2.0 * T * Hq * D * el
+    new_kv = 2.0 * 2 * T * Hkv * D * el              # read k_new/v_new + write into the pool
+    if table is None:
+        kv_read = float(sum(batch.kv_lens())) * Hkv * D * 2 * el
+    else:
+        kv_read = 0.0
+        cnt = np.asarray(count)
+        for b, kvl in enumerate(batch.kv_lens()):
+            for g in range(Hkv):
+                n = int(cnt[b, g])
+                blocks = np.asarray(table[b, g, :n], dtype=np.int64)
+                keys = np.minimum(blocks * batch.page_size + batch.page_size, kvl) - \
+                    blocks * batch.page_size
+                kv_read += float(keys.sum()) * D * 2 * el
+    return {"flops": flops, "attn_bytes": kv_read + q_o, "step_bytes": kv_read + q_o + new_kv}
+
+
+# ------------------------------------------------------------------------------------
+# Clocks during the timed region (NVML: the counters nvidia-smi prints)
+# ------------------------------------------------------------------------------------
+
+class ClockSampler:
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+               "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
+
+    def __init__(self, device_index: int, period_s: float = 0.005):
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._period = period_s
+        self._dev = device_index
+        self._thr = None
+        self._ok = False
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+            self._ok = True
+        except Exception:
+            self._ok = False
+
+    def _sample(self):
+        n = self._nvml
+        mhz = n.nvmlDeviceGetClockInfo(self._h, n.NVML_CLOCK_SM)
+        try:
+            rs = n.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+        except Exception:
+            rs = n.nvmlDeviceGetCurrentClocksThrottleReasons(self._h)
+        self.samples.append(mhz)
+        for name, bit in self.REASONS.items():
+            if rs & bit:
+                self.reasons.add(name)
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self._sample()
+            except Exception:
+                pass
+            time.sleep(self._period)
+
+    def start(self):
+        if self._ok:
+            self._thr = threading.Thread(target=self._run, daemon=True)
+            self._thr.start()
+        return self
+
+    def stop(self):
+        if self._thr is not None:
+            self._stop.set()
+            self._thr.join()
+        if self._ok and not self.samples:
+            try:
+                self._sample()
+            except Exception:
+                pass
+        return self
+
+    def summary(self):
+        if not self._ok:
+            return self._nvidia_smi_once()
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples), "source": "nvml"}
+
+    def _nvidia_smi_once(self):
+        try:
+            out = subprocess.run(
+                ["nvidia-smi", f"--id={self._dev}",
+                 "--query-gpu=clocks.sm,clocks.max.sm", "--format=csv,noheader,nounits"],
+                capture_output=True, text=True, timeout=10).stdout.strip().split(",")
+            return {"sm_mhz": float(out[0]), "sm_max_mhz": float(out[1]), "reasons": [],
+                    "samples": 1, "source": "nvidia-smi"}
+        except Exception:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+
+
+# ------------------------------------------------------------------------------------
+# GPU side
+# ------------------------------------------------------------------------------------
+
+def make_workload(name: str, seed_offset: int = 0):
+    from ragged_paged_attention_forward_b200 import workloads as wl
+    seeds = {"decode": 1002, "prefill": 1003, "mixed": 1004, "sparse": 1005}
+    seed = seeds[name] + seed_offset
+    if name == "decode":
+        return wl.decode(seed=seed, poison=False, keep_logical=False), None
+    if name == "prefill":
+        return wl.prefill(seed=seed, poison=False, keep_logical=False), None
+    if name == "mixed":
+        return wl.mixed(seed=seed, poison=False, keep_logical=False), None
+    return wl.sparse(seed=seed, poison=False)
+
+
+class Runner:
+    """Holds one batch on the device and runs steps through the C ABI."""
+
+    def __init__(self, name, batch, mask):
+        from ragged_paged_attention_forward_b200 import api
+        self.api = api
+        self.name = name
+        self.batch = batch
+        self.mask = mask
+        b = batch
+        self.d = {k: getattr(b, k).cuda().contiguous() for k in (
+            "q", "k_new", "v_new", "k_pool", "v_pool", "block_table", "cu_seqlens_q",
+            "seq_lens_k")}
+        self.out = torch.empty_like(self.d["q"])
+        self.lse = torch.empty(b.num_tokens, b.num_q_heads, dtype=torch.float32, device="cuda")
+        self.sparse = mask is not None
+        if self.sparse:
+            self.mask_d = mask.cuda()
+            nkb = mask.shape[-1]
+            assert nkb == b.max_blocks
+            self.table = torch.empty(b.num_seqs, b.num_kv_heads, nkb, dtype=torch.int32,
+                                     device="cuda")
+            self.count = torch.empty(b.num_seqs, b.num_kv_heads, dtype=torch.int32,
+                                     device="cuda")
+        else:
+            self.table = self.count = None
+        self.plan = self.make_plan()
+        self.ws = torch.empty(max(self.plan.workspace_bytes, 256), dtype=torch.uint8,
+                              device="cuda")
+        info = self.plan.info()
+        self.launches_step = info.launches_forward + (1 if self.sparse else 0)
+        self.info = info
+
+    def make_plan(self):
+        b = self.batch
+        return self.api.rpa_plan(
+            num_seqs=b.num_seqs, num_tokens=b.num_tokens, num_q_heads=b.num_q_heads,
+            num_kv_heads=b.num_kv_heads, head_dim=b.head_dim, page_size=b.page_size,
+            num_pages=b.num_pages, max_blocks_per_seq=b.max_blocks, layout=b.layout,
+            causal=b.causal, cu_seqlens_q=b.cu_seqlens_q, seq_lens_k=b.seq_lens_k,
+            sparse=self.sparse)
+
+    def tables(self, stream=None):
+        if self.sparse:
+            self.api.rpa_build_group_tables(self.mask_d, self.batch.num_kv_heads, self.table,
+                                            self.count, stream)
+
+    def step(self, fused=True, stream=None):
+        d = self.d
+        self.tables(stream)
+        self.api.rpa_forward(self.plan, d["q"], d["k_new"] if fused else None,
+                             d["v_new"] if fused else None, d["k_pool"], d["v_pool"],
+                             d["block_table"], d["cu_seqlens_q"], d["seq_lens_k"], self.table,
+                             self.count, self.batch.scale, self.out, self.lse, self.ws, stream)
+
+    def host_tables(self):
+        if not self.sparse:
+            return None, None
+        self.tables()
+        torch.cuda.synchronize()
+        return self.table.cpu().numpy(), self.count.cpu().numpy()
+
+
+def timed_loop(fn, steps, warmup, flush):
+    """Per-step CUDA-event durations (ms) of fn(), L2 flushed (untimed) before each step."""
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        flush.zero_()
+        fn()
+    torch.cuda.synchronize()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(steps)]
+    for s, e in evs:
+        flush.zero_()
+        s.record(stream)
+        fn()
+        e.record(stream)
+    torch.cuda.synchronize()
+    return [s.elapsed_time(e) for s, e in evs]
+
+
+def e2e_loop(runner, steps, warmup):
+    """End to end through the public API: plan on the host, copy the step's inputs from
+    pinned host memory, run the fused step, read the output back.  Returns (ms list, h2d
+    bytes, d2h bytes)."""
+    b = runner.batch
+    names = ["q", "k_new", "v_new", "block_table", "cu_seqlens_q", "seq_lens_k"]
+    host = {k: getattr(b, k).contiguous().pin_memory() for k in names}
+    out_host = torch.empty(runner.out.shape, dtype=runner.out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_host.numel() * out_host.element_size()
+    if runner.sparse:
+        mask_host = runner.mask.contiguous().pin_memory()
+        h2d += mask_host.numel()
+    stream = torch.cuda.current_stream()
+
+    def one():
+        plan = runner.make_plan()
+        for k in names:
+            runner.d[k].copy_(host[k], non_blocking=True)
+        if runner.sparse:
+            runner.mask_d.copy_(mask_host, non_blocking=True)
+        runner.tables()
+        d = runner.d
+        runner.api.rpa_forward(plan, d["q"], d["k_new"], d["v_new"], d["k_pool"], d["v_pool"],
+                               d["block_table"], d["cu_seqlens_q"], d["seq_lens_k"],
+                               runner.table, runner.count, b.scale, runner.out, runner.lse,
+                               runner.ws)
+        out_host.copy_(runner.out, non_blocking=True)
+        return plan
+
+    for _ in range(warmup):
+        one()
+    torch.cuda.synchronize()
+    ms = []
+    for _ in range(steps):
+        s = torch.cuda.Event(enable_timing=True)
+        e = torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        plan = one()
+        e.record(stream)
+        e.synchronize()
+        ms.append(s.elapsed_time(e))
+        del plan
+    return ms, h2d, d2h
+
+
+def profile_traffic(kernel_file: str, key: str):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel source it was taken
+    from is unchanged (sha256 of the source file)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    src = os.path.join(ROOT, "ragged_paged_attention_forward_b200", "csrc", kernel_file)
+    try:
+        with open(path) as f:
+            d = json.load(f)[key]
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+        if d.get("source_sha256") != sha:
+            return None
+        return float(d["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+def measure(name, runner, steps, warmup, flush, peaks):
+    b = runner.batch
+    table, count = runner.host_tables()
+    w = work(b, table, count)
+    step_ms = timed_loop(lambda: runner.step(True), steps, warmup, flush)
+    attn_ms = timed_loop(lambda: runner.step(False), steps, warmup, flush)
+    ms = statistics.mean(step_ms)
+    ams = statistics.mean(attn_ms)
+    res = {"workload": WORKLOAD_TEXT[name], "ms_per_step": ms, "attn_ms": ams,
+           "tokens_per_s": b.num_tokens / (ms * 1e-3),
+           "step_GBps": w["step_bytes"] / (ms * 1e-3) / 1e9,
+           "attn_GBps": w["attn_bytes"] / (ams * 1e-3) / 1e9,
+           "attn_TFLOPs": w["flops"] / (ams * 1e-3) / 1e12,
+           "flops": w["flops"], "attn_bytes": w["attn_bytes"], "step_bytes": w["step_bytes"],
+           "launches_per_step": runner.launches_step,
+           "batch_class": int(runner.info.batch_class)}
+    t_mem = w["attn_bytes"] / (peaks["hbm_gbs"] * 1e9)
+    t_flop = w["flops"] / (peaks["bf16_tflops"] * 1e12)
+    res["roofline_frac"] = max(t_mem, t_flop) / (ams * 1e-3)
+    res["bound"] = "hbm" if t_mem >= t_flop else "tensor"
+    return res
+
+
+def cpu_oracle_baseline(name, batch, target_s=12.0, table=None, count=None):
+    """Time the fp64 oracle, as it stands, on a bounded sample of the workload: whole
+    sequences (all query heads) until about target_s of CPU work."""
+    from oracle import rpa_oracle as orc
+    try:
+        from threadpoolctl import threadpool_info
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        threads = os.cpu_count() or 1
+    cu = batch.cu_seqlens_q.tolist()
+    kvl = batch.kv_lens()
+    done_bytes = done_flops = 0.0
+    elapsed = 0.0
+    nseq = 0
+    rows_done = 0
+    D, Hq, Hkv = batch.head_dim, batch.num_q_heads, batch.num_kv_heads
+    for b in range(batch.num_seqs):
+        q_len = cu[b + 1] - cu[b]
+        if q_len == 0:
+            continue
+        # rows of this sequence (capped so one sequence stays bounded)
+        nrows = min(q_len, 8)
+        rows = [(cu[b] + i, h) for i in range(q_len - nrows, q_len) for h in range(Hq)]
+        t0 = time.perf_counter()
+        orc.attention(batch.q, batch.k_pool, batch.v_pool, batch.block_table,
+                      batch.cu_seqlens_q, batch.seq_lens_k, scale=batch.scale,
+                      causal=batch.causal, page_size=batch.page_size, layout=batch.layout,
+                      num_kv_heads=Hkv, group_table=table, group_count=count, rows=rows)
+        elapsed += time.perf_counter() - t0
+        past = kvl[b] - q_len
+        keys = sum(min(kvl[b], past + i + 1) for i in range(q_len - nrows, q_len))
+        done_flops += 4.0 * D * keys * Hq
+        done_bytes += float(kvl[b]) * Hkv * D * 2 * 2 + 2.0 * nrows * Hq * D * 2
+        nseq += 1
+        rows_done += len(rows)
+        if elapsed >= target_s:
+            break
+    return {"elapsed_s": elapsed, "bytes": done_bytes, "flops": done_flops, "threads": threads,
+            "sample": f"{nseq} sequences x {Hq} query heads, last <=8 query rows each "
+                      f"({rows_done} rows), oracle fp64 numpy"}
+
+
+def run_gpu(args):
+    from ragged_paged_attention_forward_b200 import api  # noqa: F401  (fails loudly if unbuilt)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local_rank)
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    peaks, peak_src = load_peaks()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+
+    name = args.workload
+    batch, mask = make_workload(name, seed_offset=1000 * rank)
+    runner = Runner(name, batch, mask)
+    table, count = runner.host_tables()
+    w = work(batch, table, count)
+
+    # headline: the fused step, K timed steps after W warm-up steps, clocks sampled meanwhile
+    for _ in range(args.warmup):
+        flush.zero_()
+        runner.step(True)
+    torch.cuda.synchronize()
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(torch.cuda.current_device()).start()
+    stream = torch.cuda.current_stream()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(args.steps)]
+    t_wall0 = time.perf_counter()
+    for s, e in evs:
+        flush.zero_()
+        s.record(stream)
+        runner.step(True)
+        e.record(stream)
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall0
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler.stop()
+    step_ms = [s.elapsed_time(e) for s, e in evs]
+    total_ms = sum(step_ms)
+    if dist:
+        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    units = w["step_bytes"] if w["flops"] / max(w["step_bytes"], 1) < 300 else w["flops"]
+    value = world * w["step_bytes"] / (ms_per_step * 1e-3) / 1e9
+
+    # dominant kernel: the attention call alone (decode split + merge for this workload)
+    attn_ms = statistics.mean(timed_loop(lambda: runner.step(False), args.steps, 2, flush))
+    attn_gbps = w["attn_bytes"] / (attn_ms * 1e-3) / 1e9
+    kernel_file = "decode.cu" if name in ("decode", "mixed") else "prefill.cu"
+    bound = "hbm" if name in ("decode", "mixed") else "tensor"
+    if bound == "hbm":
+        roof = {"bound": "hbm", "achieved": attn_gbps, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": attn_gbps / peaks["hbm_gbs"],
+                "traffic": profile_traffic(kernel_file, name),
+                "algorithmic_bytes_per_launch": w["attn_bytes"],
+                "kernel": "rpa_forward attention (split-KV decode + LSE merge)",
+                "peak_source": f"{peak_src} (copy bandwidth)"}
+    else:
+        tf = w["flops"] / (attn_ms * 1e-3) / 1e12
+        roof = {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"],
+                "frac_of_sustained": tf / peaks["bf16_tflops_sustained"],
+                "traffic": profile_traffic(kernel_file, name),
+                "algorithmic_flops_per_launch": w["flops"],
+                "kernel": "rpa_forward attention (tcgen05 prefill)",
+                "peak_source": f"{peak_src} (cuBLAS bf16 burst)"}
+
+    # end to end through the public API with host buffers
+    e2e_ms, h2d, d2h = e2e_loop(runner, args.steps, 2)
+    e2e_ms_mean = statistics.mean(e2e_ms)
+    if dist:
+        t = torch.tensor([e2e_ms_mean], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms_mean = float(t.item())
+    e2e_val = world * w["step_bytes"] / (e2e_ms_mean * 1e-3) / 1e9
+
+    # planner host time
+    t0 = time.perf_counter()
+    for _ in range(20):
+        runner.make_plan()
+    planner_us = (time.perf_counter() - t0) / 20 * 1e6
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT[name], "per_rank_batch": "independent seed per rank",
+                   "l2": "256 MB write between timed steps (untimed); KV pool > L2",
+                   "step": "rpa_forward fused (KV write + attention + LSE merge)"
+                           + (" + group-table build" if runner.sparse else ""),
+                   "tokens_per_step": batch.num_tokens * world,
+                   "tokens_per_s": world * batch.num_tokens / (ms_per_step * 1e-3),
+                   "hbm_frac_of_step": value / world / peaks["hbm_gbs"],
+                   "planner_host_us": planner_us},
+        "roofline": roof,
+        "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms_mean,
+                "includes": "host planner + pinned H2D of q/k_new/v_new/tables + fused step + "
+                            "D2H of out"},
+        "gpu_launches": runner.launches_step * args.steps,
+        "clocks": sampler.summary(),
+        "wall_s_timed_region": t_wall,
+    }
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = cpu_oracle_baseline(name, batch, target_s=args.cpu_seconds, table=table,
+                                 count=count)
+        line["cpu_baseline"] = {"value": cb["bytes"] / cb["elapsed_s"] / 1e9, "unit": "GB/s",
+                                "cores": cb["threads"], "kind": "oracle", "sample": cb["sample"],
+                                "elapsed_s": cb["elapsed_s"],
+                                "gflops": cb["flops"] / cb["elapsed_s"] / 1e9}
+
+    if not args.no_secondary and world == 1:
+        secondary = {}
+        del runner
+        torch.cuda.empty_cache()
+        for other in ("prefill", "mixed", "sparse"):
+            if other == name:
+                continue
+            b2, m2 = make_workload(other)
+            r2 = Runner(other, b2, m2)
+            res = measure(other, r2, args.steps, args.warmup, flush, peaks)
+            if other in ("prefill", "sparse"):
+                res["frac_of_bf16_peak"] = res["attn_TFLOPs"] / peaks["bf16_tflops"]
+                res["frac_of_bf16_sustained"] = res["attn_TFLOPs"] / peaks[
+                    "bf16_tflops_sustained"]
+            secondary[other] = res
+            del r2, b2
+            torch.cuda.empty_cache()
+        line["secondary"] = secondary
+        if "prefill" in secondary:
+            line["prefill_TFLOPs"] = secondary["prefill"]["attn_TFLOPs"]
+            line["prefill_frac_of_bf16_peak"] = secondary["prefill"]["frac_of_bf16_peak"]
+    line["peaks"] = dict(peaks, source=peak_src)
+    line["hbm_frac"] = value / world / peaks["hbm_gbs"]
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_reference(args):
+    """The fp64 CPU oracle, as it stands, on the host cores: each step a bounded sample of
+    the workload (rank 0 only)."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    name = args.workload
+    batch, mask = make_workload(name)
+    table = count = None
+    if mask is not None:
+        from oracle import rpa_oracle as orc
+        table, count = orc.build_group_tables(mask, batch.num_kv_heads)
+    per_step = max(0.2, min(1.5, 120.0 / max(1, args.steps + args.warmup)))
+    for _ in range(args.warmup):
+        cpu_oracle_baseline(name, batch, target_s=per_step, table=table, count=count)
+    tot_bytes = tot_s = 0.0
+    last = None
+    for _ in range(args.steps):
+        last = cpu_oracle_baseline(name, batch, target_s=per_step, table=table, count=count)
+        tot_bytes += last["bytes"]
+        tot_s += last["elapsed_s"]
+    value = tot_bytes / tot_s / 1e9
+    line = {"metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": tot_s / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "impl": "reference",
+            "config": {"workload": WORKLOAD_TEXT[name]},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": last["threads"],
+                             "kind": "oracle", "sample": last["sample"]},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", default="decode", choices=list(WORKLOAD_TEXT))
+    ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

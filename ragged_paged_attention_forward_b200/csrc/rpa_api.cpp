@@ -310,7 +310,7 @@ rpa_status rpa_plan(const rpa_shape* shape, const int32_t* cu_seqlens_q,
            plan->pf_tiles.size() * sizeof(PrefillTile));
 
   plan->launches_write = T > 0 ? 1 : 0;
-  plan->launches_forward = (plan->dec_items.empty() ? 0 : 1) +
+  plan->launches_forward = plan->launches_write + (plan->dec_items.empty() ? 0 : 1) +
                            (plan->merge_rows.empty() ? 0 : 1) +
                            (plan->pf_tiles.empty() ? 0 : 1);
   *out_plan = plan;
