@@ -186,6 +186,37 @@ RPA_API rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new
                        void* stream);
 
 /*
+ * rpa_forward_no_alloc -- rpa_forward for callers that cannot allocate device memory.
+ * No counterpart in the pages: this is a convenience of this library.
+ *
+ * Who needs it: a host framework that owns all device memory -- a serving engine whose
+ * allocator reserved the pool at start-up, or a plugin interface that passes the operator
+ * only its inputs and outputs -- cannot hand rpa_forward a workspace, and a cudaMalloc on the
+ * step's path would stall the stream or fail.  This entry point allocates nothing: the
+ * step's scratch (the work lists copied from the plan and the split-KV decode partials) lives
+ * in a fixed array of RPA_NO_ALLOC_WORKSPACE_BYTES that the library holds on every device
+ * that loads it, until the process exits.
+ *
+ * Arguments, results and errors are those of rpa_forward minus the workspace.  A plan whose
+ * rpa_plan workspace size exceeds RPA_NO_ALLOC_WORKSPACE_BYTES is rejected with
+ * RPA_ERR_WORKSPACE_TOO_SMALL (use rpa_forward with a workspace for such batches).
+ * The first call on a device looks up the array's device address (once per device, with
+ * that device current); make that first call before any stream capture.
+ * All calls share the one array: calls whose work overlaps on the GPU (different streams,
+ * or different host threads on one device) race and must be serialised by the caller.  The
+ * array keeps the last call's contents; nothing in it needs to start at zero, because every
+ * call rewrites its work lists and every partial result before reading them.
+ */
+#define RPA_NO_ALLOC_WORKSPACE_BYTES ((size_t)8 << 20)
+
+RPA_API rpa_status rpa_forward_no_alloc(rpa_plan_t plan, const void* q, const void* k_new,
+                                        const void* v_new, void* k_pool, void* v_pool,
+                                        const int32_t* block_table, const int32_t* cu_seqlens_q,
+                                        const int32_t* seq_lens_k, const int32_t* group_table,
+                                        const int32_t* group_count, float scale, void* out,
+                                        float* lse, void* stream);
+
+/*
  * rpa_build_group_tables -- block-union KV selection (CompactAttention, Core claim and
  * Fig. 3): for every sequence b and KV group g, the ascending list of KV blocks kb such
  * that some query head hq of the group (hq / (Hq/Hkv) == g) selects kb in some query

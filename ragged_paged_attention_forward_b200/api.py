@@ -82,6 +82,9 @@ def lib() -> ctypes.CDLL:
         L.rpa_forward.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_float,
                                   _P, _P, _P, ctypes.c_size_t, _P]
         L.rpa_forward.restype = ctypes.c_int
+        L.rpa_forward_no_alloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                           ctypes.c_float, _P, _P, _P]
+        L.rpa_forward_no_alloc.restype = ctypes.c_int
         L.rpa_build_group_tables.argtypes = [_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                              ctypes.c_int32, ctypes.c_int32, _P, _P, _P]
         L.rpa_build_group_tables.restype = ctypes.c_int
@@ -190,6 +193,21 @@ def rpa_forward(plan: Plan, q, k_new, v_new, k_pool, v_pool, block_table, cu_seq
         _ptr(block_table), _ptr(cu_seqlens_q), _ptr(seq_lens_k), _ptr(group_table),
         _ptr(group_count), ctypes.c_float(scale), _ptr(out), _ptr(lse), _ptr(workspace), nbytes,
         _stream(stream)))
+
+
+NO_ALLOC_WORKSPACE_BYTES = 8 << 20
+
+
+def rpa_forward_no_alloc(plan: Plan, q, k_new, v_new, k_pool, v_pool, block_table,
+                         cu_seqlens_q, seq_lens_k, group_table, group_count, scale: float, out,
+                         lse, stream=None):
+    """rpa_forward without a workspace argument, for callers that cannot allocate device
+    memory: the scratch lives in the library's fixed per-device array (see include/rpa.h).
+    Calls that overlap on the GPU share that array and must be serialised by the caller."""
+    _check("rpa_forward_no_alloc", lib().rpa_forward_no_alloc(
+        plan.handle, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool),
+        _ptr(block_table), _ptr(cu_seqlens_q), _ptr(seq_lens_k), _ptr(group_table),
+        _ptr(group_count), ctypes.c_float(scale), _ptr(out), _ptr(lse), _stream(stream)))
 
 
 def rpa_build_group_tables(mask, num_kv_heads: int, table, count, stream=None):
