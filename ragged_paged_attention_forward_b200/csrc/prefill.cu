@@ -11,18 +11,21 @@
 // block-table lookup per K/V tile) and the prefill specialisation of "Ragged Paged Attention:
 // A High-Performance and Flexible LLM Inference Kernel for TPU" (Key ideas).
 //
-// B200 design (one CTA per (query tile, query head), 256 threads):
-//   warp 0     TMA producer: Q once, then K and V tiles of 128 keys, page by page (boxes of
-//              [min(P,128) slots x 64 dims], 128-byte swizzle) into a 2-stage ring;
-//   warp 1     allocates TMEM; lane 0 issues the MMAs:
-//                S_j = Q K_j^T   (M=128 queries, N=128 keys, K=D; A,B from shared memory)
-//                O  += P_j V_j   (M=128, N=D, K=128 keys; A = P_j from TMEM, B = V_j MN-major)
-//              S is double-buffered in TMEM so S_{j+1} runs while the softmax works on S_j;
-//              the warp zeroes V rows past the last real key before P_j V_j;
-//   warps 4-7  softmax: thread r owns query row r (TMEM lane r): loads S_j, masks, online
-//              softmax in fp32 (exp2), writes P_j as bf16 over S_j, rescales O in TMEM, and
-//              finally normalises O and stores the bf16 row and its log-sum-exp.
-// TMEM columns: S0 [0,128) S1 [128,256) O [256,256+D).  Every wait is bounded.
+// B200 design.  One CTA per (128-query tile, pair of query heads of one KV group) -- the two
+// heads share every K/V tile and the same causal mask -- with 384 threads:
+//   warp 0      TMA producer: both Q tiles once, then K and V tiles of 128 keys, page by page
+//               (boxes of [min(P,128) slots x 64 dims], 128-byte swizzle), 2-stage ring;
+//   warp 1      allocates TMEM; one thread issues the MMAs, interleaving the two heads so the
+//               tensor pipe works on one head while the other head's softmax runs:
+//                 S_h = Q_h K_j^T   (M=128 queries, N=128 keys, K=D; SMEM descriptors)
+//                 O_h += P_h V_j    (M=128, N=D, K=128 keys; P_h read from TMEM, V MN-major)
+//   warps 4-7   softmax of head A, warps 8-11 softmax of head B: thread r owns query row r
+//               (TMEM lane r); it loads S, masks, takes exp2 against a running reference max,
+//               writes P as bf16 over S and arrives.  The reference max only moves when a row's
+//               max grows by more than 2^8; only then is O rescaled in TMEM (after the previous
+//               P.V finished), so the softmax never waits on P.V otherwise.
+// TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+D) O_B [384,384+D).  Bounded waits.
+// An odd GQA group size runs with head B switched off.
 #include <cuda_bf16.h>
 #include <math_constants.h>
 
@@ -32,23 +35,24 @@
 namespace rpa {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 384;
 constexpr int kStagesPF = 2;
 constexpr int kRows = kPrefillTileRows;  // 128
 constexpr int kKeys = kPrefillTileKeys;  // 128
 constexpr uint32_t kTmemCols = 512;
+constexpr float kRescaleThreshold = 8.0f;  // log2 domain: P may grow up to 2^8 before O rescales
 
 template <int D>
 struct PfGeom {
   static constexpr int kHalves = D / 64;
   static constexpr int kHalfBytes = 128 * 128;             // 128 rows x 128 B
-  static constexpr int kTileBytes = kHalves * kHalfBytes;  // Q, K or V tile
-  static constexpr int kQOff = 0;
-  static constexpr int kKOff = kTileBytes;
+  static constexpr int kTileBytes = kHalves * kHalfBytes;  // a Q, K or V tile
+  static constexpr int kQOff = 0;                          // Q_A, Q_B
+  static constexpr int kKOff = 2 * kTileBytes;
   static constexpr int kVOff = kKOff + kStagesPF * kTileBytes;
   static constexpr int kBarOff = kVOff + kStagesPF * kTileBytes;
-  // q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_ready, o_done, mma_done
-  static constexpr int kNumBars = 1 + 3 * kStagesPF + 2 + 3;
+  // q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_ready[2], o_done[2], mma_done
+  static constexpr int kNumBars = 1 + 3 * kStagesPF + 6 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 64;
   // at least 120 KB so that a second CTA never shares the SM (and its 512 TMEM columns)
@@ -56,19 +60,11 @@ struct PfGeom {
   static_assert(kKOff % 1024 == 0 && kVOff % 1024 == 0 && kTileBytes % 1024 == 0,
                 "TMA destinations with 128-byte swizzle start on 1024-byte boundaries");
   static_assert(kBarOff % 8 == 0 && kMiscOff % 8 == 0, "mbarrier alignment");
+  static_assert(kAlloc <= 227 * 1024, "shared memory per CTA");
 };
 
 struct alignas(16) U4 {
   uint32_t x, y, z, w;
-};
-
-// Key tiles: dense tiles are 128 consecutive positions; in sparse mode a tile holds the next
-// 128/P entries of the block-union table (ascending logical blocks of P keys).
-struct KeyMap {
-  const int32_t* table;  // sparse: ascending logical block ids, or null when dense
-  int n_entries;         // sparse: entries whose block starts before the visible limit
-  int P;
-  int log2P;
 };
 
 template <int D>
@@ -88,45 +84,45 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* k_full = bars + 1;
   uint64_t* v_full = k_full + kStagesPF;
   uint64_t* kv_empty = v_full + kStagesPF;
-  uint64_t* s_full = kv_empty + kStagesPF;  // [2]
-  uint64_t* p_ready = s_full + 2;
-  uint64_t* o_done = p_ready + 1;
-  uint64_t* mma_done = o_done + 1;
+  uint64_t* s_full = kv_empty + kStagesPF;  // [2] per head
+  uint64_t* p_ready = s_full + 2;           // [2]
+  uint64_t* o_done = p_ready + 2;           // [2]
+  uint64_t* mma_done = o_done + 2;
   uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(smem + Geo::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Geo::kMiscOff + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int Hq = p.num_q_heads;
-  const int tile_idx = blockIdx.x / Hq;
-  const int hq = blockIdx.x - tile_idx * Hq;
-  const PrefillTile tile = p.tiles[tile_idx];
   const int G = Hq / p.num_kv_heads;
-  const int h = hq / G;
+  const int hpc = (G & 1) == 0 ? 2 : 1;            // query heads per CTA
+  const int groups = Hq / hpc;
+  const int tile_idx = blockIdx.x / groups;
+  const int hq0 = (blockIdx.x - tile_idx * groups) * hpc;
+  const PrefillTile tile = p.tiles[tile_idx];
+  const int h = hq0 / G;                            // KV head (shared by the pair)
   const int P = p.kv.page_size;
   const int log2P = p.kv.log2_page;
   const int past = tile.kv_len - tile.q_len;
   const int q_end = min(tile.q_len, tile.q_start + kRows);  // local, exclusive
   const int kv_hi = p.causal ? min(tile.kv_len, past + q_end) : tile.kv_len;
 
-  KeyMap km;
-  km.table = nullptr;
-  km.n_entries = 0;
-  km.P = P;
-  km.log2P = log2P;
+  // key tiles: dense -> ceil(kv_hi/128); sparse -> visible table entries, 128/P per tile
+  const int32_t* table = nullptr;
+  int n_entries = 0;
   int n_tiles;
   if (p.group_table) {
     const size_t row = (size_t)tile.seq * p.num_kv_heads + h;
-    km.table = p.group_table + row * p.kv.max_blocks;
+    table = p.group_table + row * p.kv.max_blocks;
     const int cnt = min(__ldg(p.group_count + row), p.kv.max_blocks);
-    int lo = 0, hi = max(cnt, 0);  // entries whose block starts before kv_hi (ascending table)
+    int lo = 0, hi = max(cnt, 0);  // entries whose block starts before kv_hi (ascending)
     while (lo < hi) {
       const int mid = (lo + hi) >> 1;
-      if ((__ldg(km.table + mid) << log2P) < kv_hi) lo = mid + 1; else hi = mid;
+      if ((__ldg(table + mid) << log2P) < kv_hi) lo = mid + 1; else hi = mid;
     }
-    km.n_entries = lo;
+    n_entries = lo;
     const int per = kKeys >> log2P;
-    n_tiles = (km.n_entries + per - 1) / per;
+    n_tiles = (n_entries + per - 1) / per;
   } else {
     n_tiles = (kv_hi + kKeys - 1) / kKeys;
   }
@@ -138,10 +134,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&v_full[s], 1);
       mbar_init(&kv_empty[s], 1);
     }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(p_ready, 128);
-    mbar_init(o_done, 1);
+    for (int x = 0; x < 2; ++x) {
+      mbar_init(&s_full[x], 1);
+      mbar_init(&p_ready[x], 128);
+      mbar_init(&o_done[x], 1);
+    }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -154,7 +151,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_base_sh;
-  const uint32_t tmem_o = tmem + 256;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
@@ -162,11 +158,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
-      mbar_arrive_expect_tx(q_full, Geo::kTileBytes);
+      mbar_arrive_expect_tx(q_full, Geo::kTileBytes * hpc);
+      for (int x = 0; x < hpc; ++x)
 #pragma unroll
-      for (int half = 0; half < Geo::kHalves; ++half)
-        tma_load_3d(Qs + half * Geo::kHalfBytes, &qmap, half * 64, hq, tile.t0 + tile.q_start,
-                    q_full);
+        for (int half = 0; half < Geo::kHalves; ++half)
+          tma_load_3d(Qs + x * Geo::kTileBytes + half * Geo::kHalfBytes, &qmap, half * 64,
+                      hq0 + x, tile.t0 + tile.q_start, q_full);
       const int32_t* bt_row =
           p.kv.layout == 0
               ? p.kv.block_table + (size_t)tile.seq * p.kv.max_blocks
@@ -180,10 +177,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (j >= kStagesPF && !wait_bounded(&kv_empty[slot], ((j / kStagesPF) - 1) & 1,
                                             abort_flag, p.err, kErrPrefillWait))
           break;
-        // boxes of tile j: (page, first slot in the page, destination row in the tile)
         int nbox, first_blk = 0, slot0 = 0;
-        if (km.table) {
-          nbox = min(kKeys >> log2P, km.n_entries - j * (kKeys >> log2P));
+        if (table) {
+          nbox = min(kKeys >> log2P, n_entries - j * (kKeys >> log2P));
         } else if (P >= kKeys) {
           nbox = 1;
           first_blk = (j * kKeys) >> log2P;
@@ -194,19 +190,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         mbar_arrive_expect_tx(&k_full[slot], box_bytes * nbox);
         mbar_arrive_expect_tx(&v_full[slot], box_bytes * nbox);
-        for (int i = 0; i < nbox; ++i) {
-          const int blk = km.table ? __ldg(km.table + j * (kKeys >> log2P) + i) : first_blk + i;
-          int page = -1;  // out-of-range coordinates make TMA fill zeros: no stray access
-          if (blk >= 0 && blk < p.kv.max_blocks)
-            page = __ldg(bt_row + blk);
-          else
-            atomicOr(p.err, kErrBadIndex);
-          const int drow = i * box_rows;
+        // K boxes first (S needs them first), then V
+        for (int kv = 0; kv < 2; ++kv) {
+          uint8_t* dst_base = (kv == 0 ? Ks : Vs) + slot * Geo::kTileBytes;
+          const CUtensorMap* map = kv == 0 ? &kmap : &vmap;
+          uint64_t* bar = kv == 0 ? &k_full[slot] : &v_full[slot];
+          for (int i = 0; i < nbox; ++i) {
+            const int blk = table ? __ldg(table + j * (kKeys >> log2P) + i) : first_blk + i;
+            int page = -1;  // out-of-range coordinates make TMA fill zeros: no stray access
+            if (blk >= 0 && blk < p.kv.max_blocks)
+              page = __ldg(bt_row + blk);
+            else if (kv == 0)
+              atomicOr(p.err, kErrBadIndex);
 #pragma unroll
-          for (int half = 0; half < Geo::kHalves; ++half) {
-            const int off = slot * Geo::kTileBytes + half * Geo::kHalfBytes + drow * 128;
-            tma_load_4d(Ks + off, &kmap, half * 64, hcoord, slot0, page, &k_full[slot]);
-            tma_load_4d(Vs + off, &vmap, half * 64, hcoord, slot0, page, &v_full[slot]);
+            for (int half = 0; half < Geo::kHalves; ++half)
+              tma_load_4d(dst_base + half * Geo::kHalfBytes + i * box_rows * 128, map, half * 64,
+                          hcoord, slot0, page, bar);
           }
         }
         ++issued;
@@ -227,30 +226,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (n_tiles > 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKeys, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
-      const uint32_t q_addr = smem_u32(Qs);
-      bool ok = warp_wait_bounded(q_full, 0, abort_flag, p.err, kErrPrefillWait);
-      auto issue_s = [&](int j) -> bool {
+      auto issue_s = [&](int x, int j) {  // S_x = Q_x K_j^T into TMEM columns [128x, +128)
         const int slot = j % kStagesPF;
-        if (!warp_wait_bounded(&k_full[slot], (j / kStagesPF) & 1, abort_flag, p.err,
-                               kErrPrefillWait))
-          return false;
-        if (lane == 0) {
-          tc_fence_after();
-          const uint32_t k_addr = smem_u32(Ks + slot * Geo::kTileBytes);
+        const uint32_t q_addr = smem_u32(Qs + x * Geo::kTileBytes);
+        const uint32_t k_addr = smem_u32(Ks + slot * Geo::kTileBytes);
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * Geo::kHalfBytes + (kk & 3) * 32;
-            umma_ss(tmem + (j & 1) * 128, smem_desc_sw128(q_addr + off, 16, 1024),
-                    smem_desc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
-          }
-          umma_commit(&s_full[j & 1]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * Geo::kHalfBytes + (kk & 3) * 32;
+          umma_ss(tmem + x * 128, smem_desc_sw128(q_addr + off, 16, 1024),
+                  smem_desc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
         }
-        __syncwarp();
-        return true;
+        umma_commit(&s_full[x]);
       };
-      if (ok) ok = issue_s(0);
+      auto issue_o = [&](int x, int j) {  // O_x += P_x V_j
+        const int slot = j % kStagesPF;
+        const uint32_t v_addr = smem_u32(Vs + slot * Geo::kTileBytes);
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk)
+          umma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8,
+                  smem_desc_sw128(v_addr + kk * 2048, Geo::kHalfBytes, 1024), idesc_o,
+                  (j > 0 || kk > 0) ? 1u : 0u);
+        umma_commit(&o_done[x]);
+      };
+      bool ok = warp_wait_bounded(q_full, 0, abort_flag, p.err, kErrPrefillWait) &&
+                warp_wait_bounded(&k_full[0], 0, abort_flag, p.err, kErrPrefillWait);
+      if (ok && lane == 0) {
+        tc_fence_after();
+        for (int x = 0; x < hpc; ++x) issue_s(x, 0);
+      }
+      __syncwarp();
       for (int j = 0; ok && j < n_tiles; ++j) {
-        if (j + 1 < n_tiles && !issue_s(j + 1)) break;
         const int slot = j % kStagesPF;
         if (!warp_wait_bounded(&v_full[slot], (j / kStagesPF) & 1, abort_flag, p.err,
                                kErrPrefillWait))
@@ -258,10 +263,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // V rows past the last real key may hold anything (NaN tail slots, a stale tile):
         // P = 0 there does not cancel a NaN in the product, so the rows are zeroed.
         int nvalid;
-        if (km.table) {
+        if (table) {
           const int per = kKeys >> log2P;
-          const int ne = min(per, km.n_entries - j * per);
-          const int last = __ldg(km.table + j * per + ne - 1);
+          const int ne = min(per, n_entries - j * per);
+          const int last = __ldg(table + j * per + ne - 1);
           nvalid = (ne - 1) * P + min(P, tile.kv_len - (last << log2P));
         } else {
           const int covered = min(tile.kv_len, ((kv_hi + P - 1) >> log2P) << log2P);
@@ -279,18 +284,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
         }
-        if (!warp_wait_bounded(p_ready, j & 1, abort_flag, p.err, kErrPrefillWait)) break;
-        if (lane == 0) {
-          tc_fence_after();
-          const uint32_t v_addr = smem_u32(Vs + slot * Geo::kTileBytes);
-#pragma unroll
-          for (int kk = 0; kk < kKeys / 16; ++kk)
-            umma_ts(tmem_o, tmem + (j & 1) * 128 + kk * 8,
-                    smem_desc_sw128(v_addr + kk * 2048, Geo::kHalfBytes, 1024), idesc_o,
-                    (j > 0 || kk > 0) ? 1u : 0u);
-          umma_commit(o_done);
-          umma_commit(&kv_empty[slot]);
+        const bool more = j + 1 < n_tiles;
+        if (more && !warp_wait_bounded(&k_full[(j + 1) % kStagesPF], ((j + 1) / kStagesPF) & 1,
+                                       abort_flag, p.err, kErrPrefillWait))
+          break;
+        for (int x = 0; x < hpc; ++x) {
+          if (!warp_wait_bounded(&p_ready[x], j & 1, abort_flag, p.err, kErrPrefillWait)) {
+            ok = false;
+            break;
+          }
+          if (lane == 0) {
+            tc_fence_after();
+            issue_o(x, j);
+            if (more) issue_s(x, j + 1);  // after O_x += P_x V_j consumed P_x (in order)
+          }
+          __syncwarp();
         }
+        if (!ok) break;
+        if (lane == 0) umma_commit(&kv_empty[slot]);
         __syncwarp();
       }
       // every MMA issued so far must finish before TMEM is released
@@ -298,20 +309,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       warp_wait_bounded(mma_done, 0, abort_flag, nullptr, 0, kWaitTimeoutNs / 8);
     }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------------ softmax
-    const int r = (warp - 4) * 32 + lane;  // query row == TMEM lane
-    const uint32_t lane_off = (uint32_t)((warp - 4) * 32) << 16;
+  } else if (warp >= 4 && (warp - 4) / 4 < hpc) {
+    // ------------------------------------------------------------------ softmax (head x)
+    const int x = (warp - 4) / 4;
+    const int hq = hq0 + x;
+    const int wq = warp & 3;                        // TMEM lane quarter of this warp
+    const int r = wq * 32 + lane;                   // query row == TMEM lane
+    const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
+    const uint32_t ts = tmem + x * 128 + lane_off;
+    const uint32_t to = tmem + 256 + x * 128 + lane_off;
     const int q_local = tile.q_start + r;
-    const int pos = past + q_local;        // absolute position of this row
+    const int pos = past + q_local;                 // absolute position of this row
     const int lim = p.causal ? min(tile.kv_len, pos + 1) : tile.kv_len;
     const float sc = p.scale_log2;
-    float m = -CUDART_INF_F, l = 0.f;
+    float m_ref = -CUDART_INF_F, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
-      const uint32_t ts = tmem + (j & 1) * 128 + lane_off;
-      if (!warp_wait_bounded(&s_full[j & 1], (j >> 1) & 1, abort_flag, p.err,
-                             kErrPrefillWait)) {
+      if (!warp_wait_bounded(&s_full[x], j & 1, abort_flag, p.err, kErrPrefillWait)) {
         ok = false;
         break;
       }
@@ -319,18 +333,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t sr[kKeys];
 #pragma unroll
       for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(ts + c * 32, sr + c * 32);
-      tmem_wait_ld();
       // first key position of each column group: dense -> j*128; sparse -> lane e holds the
       // start of the tile's e-th table block (missing entries map past every limit)
       int ent = j * kKeys;
       int tile_last;  // last key position the tile may hold
       bool partial = false;
-      if (km.table) {
+      if (table) {
         const int per = kKeys >> log2P;
         const int e0 = j * per;
-        const int ne = min(per, km.n_entries - e0);
+        const int ne = min(per, n_entries - e0);
         ent = 0x3fff0000;
-        if (lane < ne) ent = __ldg(km.table + e0 + lane) << log2P;
+        if (lane < ne) ent = __ldg(table + e0 + lane) << log2P;
         tile_last = __shfl_sync(0xffffffffu, ent, ne - 1) + P - 1;
         partial = ne < per;
       } else {
@@ -338,12 +351,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const bool need_mask = partial || tile_last >= tile.kv_len ||
                              (p.causal && tile_last > past + tile.q_start);
+      tmem_wait_ld();
       float mx = -CUDART_INF_F;
       if (need_mask) {
 #pragma unroll
         for (int c = 0; c < kKeys; ++c) {
-          const int kp = km.table ? __shfl_sync(0xffffffffu, ent, c >> log2P) + (c & (P - 1))
-                                  : ent + c;
+          const int kp = table ? __shfl_sync(0xffffffffu, ent, c >> log2P) + (c & (P - 1))
+                               : ent + c;
           const float v = kp < lim ? __uint_as_float(sr[c]) * sc : -CUDART_INF_F;
           sr[c] = __float_as_uint(v);
           mx = fmaxf(mx, v);
@@ -356,47 +370,53 @@ __global__ void __launch_bounds__(kThreads, 1)
           mx = fmaxf(mx, v);
         }
       }
-      const float m_new = fmaxf(m, mx);
-      const float m_use = m_new == -CUDART_INF_F ? 0.f : m_new;
-      const float alpha = fast_exp2(m - m_use);
+      // reference max: moves only when the row max grows by more than the threshold
+      float fac = 1.f;
+      bool rescale = false;
+      if (m_ref == -CUDART_INF_F) {
+        m_ref = mx;  // nothing accumulated yet (O and l are zero for this row)
+      } else if (mx > m_ref + kRescaleThreshold) {
+        fac = fast_exp2(m_ref - mx);
+        m_ref = mx;
+        rescale = true;
+      }
+      const float m_use = m_ref == -CUDART_INF_F ? 0.f : m_ref;
       float rs = 0.f;
 #pragma unroll
       for (int c = 0; c < kKeys; c += 2) {
         const float p0 = fast_exp2(__uint_as_float(sr[c]) - m_use);
         const float p1 = fast_exp2(__uint_as_float(sr[c + 1]) - m_use);
         rs += p0 + p1;
-        sr[c >> 1] = pack_bf16(p0, p1);  // P_j as bf16 pairs, over the consumed S values
+        sr[c >> 1] = pack_bf16(p0, p1);  // P as bf16 pairs, over the consumed S values
       }
-      l = l * alpha + rs;
-      m = m_new;
+      l = l * fac + rs;
 #pragma unroll
       for (int c = 0; c < kKeys / 64; ++c) tmem_st32(ts + c * 32, sr + c * 32);
-      if (j > 0) {
-        // O += P_{j-1} V_{j-1} must be complete before O is rescaled
-        if (!warp_wait_bounded(o_done, (j - 1) & 1, abort_flag, p.err, kErrPrefillWait)) {
+      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+        // O += P V of the previous tile must be complete before O is rescaled
+        if (!warp_wait_bounded(&o_done[x], (j - 1) & 1, abort_flag, p.err, kErrPrefillWait)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            uint32_t o[32];
-            tmem_ld32(tmem_o + lane_off + c * 32, o);
-            tmem_wait_ld();
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t o[32];
+          tmem_ld32(to + c * 32, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * alpha);
-            tmem_st32(tmem_o + lane_off + c * 32, o);
-          }
+          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * fac);
+          tmem_st32(to + c * 32, o);
         }
       }
       tmem_wait_st();
       tc_fence_before();
-      mbar_arrive(p_ready);
+      mbar_arrive(&p_ready[x]);
     }
     // ---- epilogue: O / l -> bf16 (a row that saw no key gets 0 and lse = -inf)
     if (ok && n_tiles > 0) {
-      ok = warp_wait_bounded(o_done, (n_tiles - 1) & 1, abort_flag, p.err, kErrPrefillWait);
+      ok = warp_wait_bounded(&o_done[x], (n_tiles - 1) & 1, abort_flag, p.err,
+                             kErrPrefillWait);
       tc_fence_after();
     }
     if (ok) {
@@ -408,7 +428,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];
         if (n_tiles > 0) {
-          tmem_ld32(tmem_o + lane_off + c * 32, o);
+          tmem_ld32(to + c * 32, o);
           tmem_wait_ld();
         } else {
 #pragma unroll
@@ -428,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (write && p.lse)
         p.lse[(size_t)t * Hq + hq] =
-            l > 0.f ? (m + fast_log2(l)) * 0.69314718055994531f : -CUDART_INF_F;
+            l > 0.f ? (m_ref + fast_log2(l)) * 0.69314718055994531f : -CUDART_INF_F;
     }
   }
   tc_fence_before();
@@ -450,7 +470,9 @@ cudaError_t launch_prefill(const PrefillLaunch& p, cudaStream_t stream) {
   if (e != cudaSuccess) return e;
   e = encode_kv_map(&vmap, p.kv.v_pool, p.kv, p.head_dim, kKeys);
   if (e != cudaSuccess) return e;
-  const dim3 grid((unsigned)p.num_tiles * (unsigned)p.num_q_heads);
+  const int G = p.num_q_heads / p.num_kv_heads;
+  const int hpc = (G & 1) == 0 ? 2 : 1;
+  const dim3 grid((unsigned)p.num_tiles * (unsigned)(p.num_q_heads / hpc));
   if (p.head_dim == 128) {
     e = ensure_smem_attr(reinterpret_cast<const void*>(prefill_kernel<128>),
                          PfGeom<128>::kAlloc);
