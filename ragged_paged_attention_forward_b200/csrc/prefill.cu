@@ -41,6 +41,12 @@ constexpr int kRows = kPrefillTileRows;  // 128
 constexpr int kKeys = kPrefillTileKeys;  // 128
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 domain: P may grow up to 2^8 before O rescales
+// Registers: the CTA launches with kLaunchRegs per thread (3 warpgroups); the producer/MMA
+// warpgroup gives most of its share to the two softmax warpgroups.
+constexpr int kLaunchRegs = 168;
+constexpr int kRegsControl = 64;
+constexpr int kRegsSoftmax = 216;
+static_assert(kRegsControl + 2 * kRegsSoftmax <= 3 * kLaunchRegs, "register split");
 
 template <int D>
 struct PfGeom {
@@ -51,8 +57,9 @@ struct PfGeom {
   static constexpr int kKOff = 2 * kTileBytes;
   static constexpr int kVOff = kKOff + kStagesPF * kTileBytes;
   static constexpr int kBarOff = kVOff + kStagesPF * kTileBytes;
-  // q_full, k_full[S], v_full[S], kv_empty[S], s_full[2], p_ready[2], o_done[2], mma_done
-  static constexpr int kNumBars = 1 + 3 * kStagesPF + 6 + 1;
+  // q_full, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], p_ready[2], o_done[2],
+  // mma_done
+  static constexpr int kNumBars = 1 + 4 * kStagesPF + 6 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 64;
   // at least 120 KB so that a second CTA never shares the SM (and its 512 TMEM columns)
@@ -83,8 +90,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
   uint64_t* v_full = k_full + kStagesPF;
-  uint64_t* kv_empty = v_full + kStagesPF;
-  uint64_t* s_full = kv_empty + kStagesPF;  // [2] per head
+  uint64_t* k_empty = v_full + kStagesPF;   // K slot free: both heads' S MMAs done
+  uint64_t* v_empty = k_empty + kStagesPF;  // V slot free: both heads' P.V MMAs done
+  uint64_t* s_full = v_empty + kStagesPF;   // [2] per head
   uint64_t* p_ready = s_full + 2;           // [2]
   uint64_t* o_done = p_ready + 2;           // [2]
   uint64_t* mma_done = o_done + 2;
@@ -132,7 +140,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < kStagesPF; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&v_full[s], 1);
-      mbar_init(&kv_empty[s], 1);
+      mbar_init(&k_empty[s], 1);
+      mbar_init(&v_empty[s], 1);
     }
     for (int x = 0; x < 2; ++x) {
       mbar_init(&s_full[x], 1);
@@ -152,6 +161,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_base_sh;
 
+  // Registers are rebalanced at the top of each warpgroup's branch: the control warpgroup
+  // (producer, MMA issuer, two idle warps) gives registers to the softmax warpgroups, whose
+  // threads each hold a 128-value S row.
+  if (warp < 4) {
+    regs_dealloc<kRegsControl>();
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0 && n_tiles > 0) {
@@ -171,12 +185,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int hcoord = p.kv.layout == 0 ? h : 0;
       const int box_rows = P < kKeys ? P : kKeys;
       const uint32_t box_bytes = (uint32_t)box_rows * 128u * Geo::kHalves;
-      int issued = 0;
+      int issued[2] = {0, 0};  // K and V tiles whose copies were started
       for (int j = 0; j < n_tiles; ++j) {
         const int slot = j % kStagesPF;
-        if (j >= kStagesPF && !wait_bounded(&kv_empty[slot], ((j / kStagesPF) - 1) & 1,
-                                            abort_flag, p.err, kErrPrefillWait))
-          break;
         int nbox, first_blk = 0, slot0 = 0;
         if (table) {
           nbox = min(kKeys >> log2P, n_entries - j * (kKeys >> log2P));
@@ -188,10 +199,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           first_blk = (j * kKeys) >> log2P;
           nbox = ((min(j * kKeys + kKeys, kv_hi) - 1) >> log2P) - first_blk + 1;
         }
-        mbar_arrive_expect_tx(&k_full[slot], box_bytes * nbox);
-        mbar_arrive_expect_tx(&v_full[slot], box_bytes * nbox);
-        // K boxes first (S needs them first), then V
+        // K first (S needs it first), then V; each waits for its own slot to be released
+        bool stop = false;
         for (int kv = 0; kv < 2; ++kv) {
+          uint64_t* empty = kv == 0 ? &k_empty[slot] : &v_empty[slot];
+          if (j >= kStagesPF && !wait_bounded(empty, ((j / kStagesPF) - 1) & 1, abort_flag,
+                                              p.err, kErrPrefillWait)) {
+            stop = true;
+            break;
+          }
+          mbar_arrive_expect_tx(kv == 0 ? &k_full[slot] : &v_full[slot], box_bytes * nbox);
           uint8_t* dst_base = (kv == 0 ? Ks : Vs) + slot * Geo::kTileBytes;
           const CUtensorMap* map = kv == 0 ? &kmap : &vmap;
           uint64_t* bar = kv == 0 ? &k_full[slot] : &v_full[slot];
@@ -207,17 +224,16 @@ __global__ void __launch_bounds__(kThreads, 1)
               tma_load_4d(dst_base + half * Geo::kHalfBytes + i * box_rows * 128, map, half * 64,
                           hcoord, slot0, page, bar);
           }
+          issued[kv] = j + 1;
         }
-        ++issued;
+        if (stop) break;
       }
       if (*abort_flag) {  // let copies in flight land before shared memory goes away
         wait_bounded(q_full, 0, abort_flag, nullptr, 0, kWaitTimeoutNs / 8);
-        for (int j = max(0, issued - kStagesPF); j < issued; ++j) {
-          wait_bounded(&k_full[j % kStagesPF], (j / kStagesPF) & 1, abort_flag, nullptr, 0,
-                       kWaitTimeoutNs / 8);
-          wait_bounded(&v_full[j % kStagesPF], (j / kStagesPF) & 1, abort_flag, nullptr, 0,
-                       kWaitTimeoutNs / 8);
-        }
+        for (int kv = 0; kv < 2; ++kv)
+          for (int j = max(0, issued[kv] - kStagesPF); j < issued[kv]; ++j)
+            wait_bounded(kv == 0 ? &k_full[j % kStagesPF] : &v_full[j % kStagesPF],
+                         (j / kStagesPF) & 1, abort_flag, nullptr, 0, kWaitTimeoutNs / 8);
       }
     }
     __syncwarp();
@@ -253,6 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok && lane == 0) {
         tc_fence_after();
         for (int x = 0; x < hpc; ++x) issue_s(x, 0);
+        umma_commit(&k_empty[0]);  // K_0 is free once both S MMAs finish
       }
       __syncwarp();
       for (int j = 0; ok && j < n_tiles; ++j) {
@@ -284,10 +301,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           fence_proxy_async_smem();
           __syncwarp();
         }
+        // per head: O_x += P_x V_j as soon as P_x is ready, then S_x for the next tile (it
+        // overwrites P_x in TMEM, so it must follow the P.V MMA, which tcgen05 keeps in order)
         const bool more = j + 1 < n_tiles;
-        if (more && !warp_wait_bounded(&k_full[(j + 1) % kStagesPF], ((j + 1) / kStagesPF) & 1,
-                                       abort_flag, p.err, kErrPrefillWait))
-          break;
+        const int nslot = (j + 1) % kStagesPF;
         for (int x = 0; x < hpc; ++x) {
           if (!warp_wait_bounded(&p_ready[x], j & 1, abort_flag, p.err, kErrPrefillWait)) {
             ok = false;
@@ -296,21 +313,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) {
             tc_fence_after();
             issue_o(x, j);
-            if (more) issue_s(x, j + 1);  // after O_x += P_x V_j consumed P_x (in order)
+            if (x == hpc - 1) umma_commit(&v_empty[slot]);
           }
           __syncwarp();
+          if (more) {
+            if (!warp_wait_bounded(&k_full[nslot], ((j + 1) / kStagesPF) & 1, abort_flag, p.err,
+                                   kErrPrefillWait)) {
+              ok = false;
+              break;
+            }
+            if (lane == 0) {
+              tc_fence_after();
+              issue_s(x, j + 1);
+              if (x == hpc - 1) umma_commit(&k_empty[nslot]);
+            }
+            __syncwarp();
+          }
         }
         if (!ok) break;
-        if (lane == 0) umma_commit(&kv_empty[slot]);
-        __syncwarp();
       }
       // every MMA issued so far must finish before TMEM is released
       if (lane == 0) umma_commit(mma_done);
       __syncwarp();
       warp_wait_bounded(mma_done, 0, abort_flag, nullptr, 0, kWaitTimeoutNs / 8);
     }
-  } else if (warp >= 4 && (warp - 4) / 4 < hpc) {
+  }
+  } else if ((warp - 4) / 4 < hpc) {
     // ------------------------------------------------------------------ softmax (head x)
+    regs_alloc<kRegsSoftmax>();
     const int x = (warp - 4) / 4;
     const int hq = hq0 + x;
     const int wq = warp & 3;                        // TMEM lane quarter of this warp
@@ -450,6 +480,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         p.lse[(size_t)t * Hq + hq] =
             l > 0.f ? (m_ref + fast_log2(l)) * 0.69314718055994531f : -CUDART_INF_F;
     }
+  } else {
+    regs_dealloc<kRegsControl>();  // head B's warpgroup when the group size is odd
   }
   tc_fence_before();
   __syncthreads();
@@ -473,6 +505,20 @@ cudaError_t launch_prefill(const PrefillLaunch& p, cudaStream_t stream) {
   const int G = p.num_q_heads / p.num_kv_heads;
   const int hpc = (G & 1) == 0 ? 2 : 1;
   const dim3 grid((unsigned)p.num_tiles * (unsigned)(p.num_q_heads / hpc));
+  // the register rebalancing inside the kernel needs exactly the launch budget it was
+  // written for; refuse to launch otherwise (a short budget would stall setmaxnreg.inc)
+  {
+    cudaFuncAttributes fa;
+    const void* k = p.head_dim == 128 ? reinterpret_cast<const void*>(prefill_kernel<128>)
+                                      : reinterpret_cast<const void*>(prefill_kernel<64>);
+    e = cudaFuncGetAttributes(&fa, k);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != kLaunchRegs) {
+      set_last_error("prefill kernel built with %d registers per thread, expected %d",
+                     fa.numRegs, kLaunchRegs);
+      return cudaErrorInvalidConfiguration;
+    }
+  }
   if (p.head_dim == 128) {
     e = ensure_smem_attr(reinterpret_cast<const void*>(prefill_kernel<128>),
                          PfGeom<128>::kAlloc);

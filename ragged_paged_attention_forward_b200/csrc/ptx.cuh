@@ -184,6 +184,17 @@ __device__ __forceinline__ float fast_log2(float x) {
   return y;
 }
 
+// Per-warpgroup register budget (all four warps of a warpgroup execute it).  The sum over the
+// CTA's warpgroups must not exceed the registers the CTA was launched with.
+template <int N>
+__device__ __forceinline__ void regs_dealloc() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_alloc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ------------------------------------------------------------------------------------
 // tcgen05: tensor memory and the 5th-generation tensor-core MMA
 // ------------------------------------------------------------------------------------
