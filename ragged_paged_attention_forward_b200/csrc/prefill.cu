@@ -382,22 +382,44 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool need_mask = partial || tile_last >= tile.kv_len ||
                              (p.causal && tile_last > past + tile.q_start);
       tmem_wait_ld();
-      float mx = -CUDART_INF_F;
+      // Row max of scale*S over the visible columns, with 8 independent accumulators so the
+      // reduction is a short tree, not a 128-long dependency chain.
+      float mx;
+      uint32_t vis[kKeys / 32];  // visibility bits (masked tiles only)
       if (need_mask) {
+        float acc[8];
+#pragma unroll
+        for (int k = 0; k < 8; ++k) acc[k] = -CUDART_INF_F;
+#pragma unroll
+        for (int w = 0; w < kKeys / 32; ++w) vis[w] = 0u;
 #pragma unroll
         for (int c = 0; c < kKeys; ++c) {
           const int kp = table ? __shfl_sync(0xffffffffu, ent, c >> log2P) + (c & (P - 1))
                                : ent + c;
-          const float v = kp < lim ? __uint_as_float(sr[c]) * sc : -CUDART_INF_F;
-          sr[c] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
+          const bool v = kp < lim;
+          vis[c >> 5] |= (v ? 1u : 0u) << (c & 31);
+          acc[c & 7] = fmaxf(acc[c & 7], v ? __uint_as_float(sr[c]) * sc : -CUDART_INF_F);
         }
+        mx = fmaxf(fmaxf(fmaxf(acc[0], acc[1]), fmaxf(acc[2], acc[3])),
+                   fmaxf(fmaxf(acc[4], acc[5]), fmaxf(acc[6], acc[7])));
       } else {
+        // scale*max(S) for a non-negative scale, scale*min(S) for a negative one
+        // 3-input max/min: two new values per instruction, four independent accumulators
+        float acc[4];
 #pragma unroll
-        for (int c = 0; c < kKeys; ++c) {
-          const float v = __uint_as_float(sr[c]) * sc;
-          sr[c] = __float_as_uint(v);
-          mx = fmaxf(mx, v);
+        for (int k = 0; k < 4; ++k) acc[k] = __uint_as_float(sr[k]);
+        if (sc >= 0.f) {
+#pragma unroll
+          for (int c = 4; c < kKeys; c += 2)
+            acc[(c >> 1) & 3] = fmax3(acc[(c >> 1) & 3], __uint_as_float(sr[c]),
+                                      __uint_as_float(sr[c + 1]));
+          mx = fmaxf(fmax3(acc[0], acc[1], acc[2]), acc[3]) * sc;
+        } else {
+#pragma unroll
+          for (int c = 4; c < kKeys; c += 2)
+            acc[(c >> 1) & 3] = fmin3(acc[(c >> 1) & 3], __uint_as_float(sr[c]),
+                                      __uint_as_float(sr[c + 1]));
+          mx = fminf(fmin3(acc[0], acc[1], acc[2]), acc[3]) * sc;
         }
       }
       // reference max: moves only when the row max grows by more than the threshold
@@ -410,14 +432,34 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_ref = mx;
         rescale = true;
       }
-      const float m_use = m_ref == -CUDART_INF_F ? 0.f : m_ref;
-      float rs = 0.f;
+      const float neg_m = m_ref == -CUDART_INF_F ? 0.f : -m_ref;
+      // P = exp2(scale*S - m): one packed FFMA per pair of elements and one EX2 per element;
+      // the row sum is kept in four packed partial sums
+      const uint64_t sc2 = f2_pack(sc, sc);
+      const uint64_t nm2 = f2_pack(neg_m, neg_m);
+      uint64_t rsum2[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) rsum2[k] = 0ull;
 #pragma unroll
       for (int c = 0; c < kKeys; c += 2) {
-        const float p0 = fast_exp2(__uint_as_float(sr[c]) - m_use);
-        const float p1 = fast_exp2(__uint_as_float(sr[c + 1]) - m_use);
-        rs += p0 + p1;
+        float t0, t1;
+        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2),
+                  t0, t1);
+        float p0 = fast_exp2(t0);
+        float p1 = fast_exp2(t1);
+        if (need_mask) {
+          p0 = (vis[c >> 5] >> (c & 31)) & 1u ? p0 : 0.f;
+          p1 = (vis[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u ? p1 : 0.f;
+        }
+        rsum2[(c >> 1) & 3] = f2_add(rsum2[(c >> 1) & 3], f2_pack(p0, p1));
         sr[c >> 1] = pack_bf16(p0, p1);  // P as bf16 pairs, over the consumed S values
+      }
+      float rs = 0.f;
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        float a, b;
+        f2_unpack(rsum2[k], a, b);
+        rs += a + b;
       }
       l = l * fac + rs;
 #pragma unroll
