@@ -36,7 +36,8 @@ namespace rpa {
 namespace {
 
 constexpr int kThreads = 384;
-constexpr int kStagesPF = 2;
+constexpr int kStagesK = 2;  // K tiles in flight
+constexpr int kStagesV = 2;  // V tiles in flight
 constexpr int kRows = kPrefillTileRows;  // 128
 constexpr int kKeys = kPrefillTileKeys;  // 128
 constexpr uint32_t kTmemCols = 512;
@@ -55,11 +56,11 @@ struct PfGeom {
   static constexpr int kTileBytes = kHalves * kHalfBytes;  // a Q, K or V tile
   static constexpr int kQOff = 0;                          // Q_A, Q_B
   static constexpr int kKOff = 2 * kTileBytes;
-  static constexpr int kVOff = kKOff + kStagesPF * kTileBytes;
-  static constexpr int kBarOff = kVOff + kStagesPF * kTileBytes;
+  static constexpr int kVOff = kKOff + kStagesK * kTileBytes;
+  static constexpr int kBarOff = kVOff + kStagesV * kTileBytes;
   // q_full, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], p_ready[2], o_done[2],
   // mma_done
-  static constexpr int kNumBars = 1 + 4 * kStagesPF + 6 + 1;
+  static constexpr int kNumBars = 1 + 2 * kStagesK + 2 * kStagesV + 6 + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 64;
   // at least 120 KB so that a second CTA never shares the SM (and its 512 TMEM columns)
@@ -89,10 +90,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Geo::kBarOff);
   uint64_t* q_full = bars;
   uint64_t* k_full = bars + 1;
-  uint64_t* v_full = k_full + kStagesPF;
-  uint64_t* k_empty = v_full + kStagesPF;   // K slot free: both heads' S MMAs done
-  uint64_t* v_empty = k_empty + kStagesPF;  // V slot free: both heads' P.V MMAs done
-  uint64_t* s_full = v_empty + kStagesPF;   // [2] per head
+  uint64_t* v_full = k_full + kStagesK;
+  uint64_t* k_empty = v_full + kStagesV;   // K slot free: both heads' S MMAs done
+  uint64_t* v_empty = k_empty + kStagesK;  // V slot free: both heads' P.V MMAs done
+  uint64_t* s_full = v_empty + kStagesV;   // [2] per head
   uint64_t* p_ready = s_full + 2;           // [2]
   uint64_t* o_done = p_ready + 2;           // [2]
   uint64_t* mma_done = o_done + 2;
@@ -137,10 +138,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < kStagesPF; ++s) {
+    for (int s = 0; s < kStagesK; ++s) {
       mbar_init(&k_full[s], 1);
-      mbar_init(&v_full[s], 1);
       mbar_init(&k_empty[s], 1);
+    }
+    for (int s = 0; s < kStagesV; ++s) {
+      mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
     for (int x = 0; x < 2; ++x) {
@@ -187,7 +190,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t box_bytes = (uint32_t)box_rows * 128u * Geo::kHalves;
       int issued[2] = {0, 0};  // K and V tiles whose copies were started
       for (int j = 0; j < n_tiles; ++j) {
-        const int slot = j % kStagesPF;
         int nbox, first_blk = 0, slot0 = 0;
         if (table) {
           nbox = min(kKeys >> log2P, n_entries - j * (kKeys >> log2P));
@@ -202,9 +204,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         // K first (S needs it first), then V; each waits for its own slot to be released
         bool stop = false;
         for (int kv = 0; kv < 2; ++kv) {
+          const int ns = kv == 0 ? kStagesK : kStagesV;
+          const int slot = j % ns;
           uint64_t* empty = kv == 0 ? &k_empty[slot] : &v_empty[slot];
-          if (j >= kStagesPF && !wait_bounded(empty, ((j / kStagesPF) - 1) & 1, abort_flag,
-                                              p.err, kErrPrefillWait)) {
+          if (j >= ns && !wait_bounded(empty, ((j / ns) - 1) & 1, abort_flag, p.err,
+                                       kErrPrefillWait)) {
             stop = true;
             break;
           }
@@ -230,10 +234,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (*abort_flag) {  // let copies in flight land before shared memory goes away
         wait_bounded(q_full, 0, abort_flag, nullptr, 0, kWaitTimeoutNs / 8);
-        for (int kv = 0; kv < 2; ++kv)
-          for (int j = max(0, issued[kv] - kStagesPF); j < issued[kv]; ++j)
-            wait_bounded(kv == 0 ? &k_full[j % kStagesPF] : &v_full[j % kStagesPF],
-                         (j / kStagesPF) & 1, abort_flag, nullptr, 0, kWaitTimeoutNs / 8);
+        for (int kv = 0; kv < 2; ++kv) {
+          const int ns = kv == 0 ? kStagesK : kStagesV;
+          for (int j = max(0, issued[kv] - ns); j < issued[kv]; ++j)
+            wait_bounded(kv == 0 ? &k_full[j % ns] : &v_full[j % ns], (j / ns) & 1, abort_flag,
+                         nullptr, 0, kWaitTimeoutNs / 8);
+        }
       }
     }
     __syncwarp();
@@ -242,26 +248,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (n_tiles > 0) {
       constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKeys, false, false);
       constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+      // Descriptors are built once; an MMA's operands differ from the base only in the start
+      // address field (bits 0..13, in 16-byte units, no carry for addresses below 256 KB), so
+      // each MMA needs one add per operand instead of rebuilding a 64-bit descriptor.
+      const uint64_t dq0 = smem_desc_sw128(smem_u32(Qs), 16, 1024);
+      const uint64_t dk0 = smem_desc_sw128(smem_u32(Ks), 16, 1024);
+      const uint64_t dv0 = smem_desc_sw128(smem_u32(Vs), Geo::kHalfBytes, 1024);
       auto issue_s = [&](int x, int j) {  // S_x = Q_x K_j^T into TMEM columns [128x, +128)
-        const int slot = j % kStagesPF;
-        const uint32_t q_addr = smem_u32(Qs + x * Geo::kTileBytes);
-        const uint32_t k_addr = smem_u32(Ks + slot * Geo::kTileBytes);
+        const uint64_t a0 = dq0 + (uint64_t)((x * Geo::kTileBytes) >> 4);
+        const uint64_t b0 = dk0 + (uint64_t)(((j % kStagesK) * Geo::kTileBytes) >> 4);
+        const uint32_t d = tmem + x * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * Geo::kHalfBytes + (kk & 3) * 32;
-          umma_ss(tmem + x * 128, smem_desc_sw128(q_addr + off, 16, 1024),
-                  smem_desc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+          const uint64_t off = (uint64_t)(((kk >> 2) * Geo::kHalfBytes + (kk & 3) * 32) >> 4);
+          umma_ss(d, a0 + off, b0 + off, idesc_s, kk > 0 ? 1u : 0u);
         }
         umma_commit(&s_full[x]);
       };
       auto issue_o = [&](int x, int j) {  // O_x += P_x V_j
-        const int slot = j % kStagesPF;
-        const uint32_t v_addr = smem_u32(Vs + slot * Geo::kTileBytes);
+        const uint64_t b0 = dv0 + (uint64_t)(((j % kStagesV) * Geo::kTileBytes) >> 4);
+        const uint32_t d = tmem + 256 + x * 128;
+        const uint32_t a = tmem + x * 128;
+        const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk)
-          umma_ts(tmem + 256 + x * 128, tmem + x * 128 + kk * 8,
-                  smem_desc_sw128(v_addr + kk * 2048, Geo::kHalfBytes, 1024), idesc_o,
-                  (j > 0 || kk > 0) ? 1u : 0u);
+          umma_ts(d, a + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : acc0);
         umma_commit(&o_done[x]);
       };
       bool ok = warp_wait_bounded(q_full, 0, abort_flag, p.err, kErrPrefillWait) &&
@@ -273,8 +284,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       __syncwarp();
       for (int j = 0; ok && j < n_tiles; ++j) {
-        const int slot = j % kStagesPF;
-        if (!warp_wait_bounded(&v_full[slot], (j / kStagesPF) & 1, abort_flag, p.err,
+        const int slot = j % kStagesV;
+        if (!warp_wait_bounded(&v_full[slot], (j / kStagesV) & 1, abort_flag, p.err,
                                kErrPrefillWait))
           break;
         // V rows past the last real key may hold anything (NaN tail slots, a stale tile):
@@ -304,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // per head: O_x += P_x V_j as soon as P_x is ready, then S_x for the next tile (it
         // overwrites P_x in TMEM, so it must follow the P.V MMA, which tcgen05 keeps in order)
         const bool more = j + 1 < n_tiles;
-        const int nslot = (j + 1) % kStagesPF;
+        const int nslot = (j + 1) % kStagesK;
         for (int x = 0; x < hpc; ++x) {
           if (!warp_wait_bounded(&p_ready[x], j & 1, abort_flag, p.err, kErrPrefillWait)) {
             ok = false;
@@ -317,7 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           __syncwarp();
           if (more) {
-            if (!warp_wait_bounded(&k_full[nslot], ((j + 1) / kStagesPF) & 1, abort_flag, p.err,
+            if (!warp_wait_bounded(&k_full[nslot], ((j + 1) / kStagesK) & 1, abort_flag, p.err,
                                    kErrPrefillWait)) {
               ok = false;
               break;
