@@ -107,6 +107,20 @@ cudaError_t ensure_smem_attr(const void* kernel, int bytes) {
   return cudaSuccess;
 }
 
+cudaError_t side_stream(cudaStream_t* stream) {
+  static cudaStream_t streams[kMaxDevices] = {nullptr};
+  static std::mutex mu;
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!streams[dev]) {
+    cudaError_t e = cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking);
+    if (e != cudaSuccess) return e;
+  }
+  *stream = streams[dev];
+  return cudaSuccess;
+}
+
 int device_sm_count() {
   static int counts[kMaxDevices] = {0};
   const int dev = current_device();

@@ -67,6 +67,13 @@ struct rpa_plan_s {
   std::vector<uint8_t> meta;  // host image of the metadata region
   int launches_forward = 0;
   int launches_write = 0;
+  // fork/join events of a mixed batch (created on first use, on the device of that call)
+  cudaEvent_t fork_ev = nullptr;
+  cudaEvent_t join_ev = nullptr;
+  ~rpa_plan_s() {
+    if (fork_ev) cudaEventDestroy(fork_ev);
+    if (join_ev) cudaEventDestroy(join_ev);
+  }
 };
 
 #define RPA_FAIL(code, ...)            \
@@ -451,6 +458,28 @@ rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const 
   kv.num_pages = s.num_pages;
   const float scale_log2 = scale * 1.4426950408889634f;
 
+  // A mixed batch runs the tensor-core kernel on the library's side stream, concurrently with
+  // the split-KV decode kernel on the caller's stream: the decode CTAs fill the SMs that the
+  // long prefill CTAs leave free.  The caller's stream waits for both before it goes on.
+  const bool fork = !plan->pf_tiles.empty() && !plan->dec_items.empty();
+  cudaStream_t pf_stream = stream;
+  if (fork) {
+    st = check_cuda(side_stream(&pf_stream), "side stream");
+    if (st != RPA_OK) return st;
+    if (!plan->fork_ev) {
+      st = check_cuda(cudaEventCreateWithFlags(&plan->fork_ev, cudaEventDisableTiming),
+                      "event create");
+      if (st != RPA_OK) return st;
+      st = check_cuda(cudaEventCreateWithFlags(&plan->join_ev, cudaEventDisableTiming),
+                      "event create");
+      if (st != RPA_OK) return st;
+    }
+    st = check_cuda(cudaEventRecord(plan->fork_ev, stream), "fork record");
+    if (st != RPA_OK) return st;
+    st = check_cuda(cudaStreamWaitEvent(pf_stream, plan->fork_ev, 0), "fork wait");
+    if (st != RPA_OK) return st;
+  }
+
   if (!plan->pf_tiles.empty()) {
     PrefillLaunch p;
     p.tiles = reinterpret_cast<const PrefillTile*>(ws + plan->off_pf);
@@ -468,7 +497,7 @@ rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const 
     p.group_count = group_count;
     p.err = err;
     p.kv = kv;
-    st = check_cuda(launch_prefill(p, stream), "prefill launch");
+    st = check_cuda(launch_prefill(p, pf_stream), "prefill launch");
     if (st != RPA_OK) return st;
   }
   if (!plan->dec_items.empty()) {
@@ -505,6 +534,12 @@ rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const 
       st = check_cuda(launch_merge(m, stream), "merge launch");
       if (st != RPA_OK) return st;
     }
+  }
+  if (fork) {
+    st = check_cuda(cudaEventRecord(plan->join_ev, pf_stream), "join record");
+    if (st != RPA_OK) return st;
+    st = check_cuda(cudaStreamWaitEvent(stream, plan->join_ev, 0), "join wait");
+    if (st != RPA_OK) return st;
   }
   return RPA_OK;
 }
