@@ -131,7 +131,7 @@ class ClockSampler:
     REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
                "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80}
 
-    def __init__(self, device_index: int, period_s: float = 0.005):
+    def __init__(self, device_index: int, period_s: float = 0.002):
         self.samples = []
         self.reasons = set()
         self.max_mhz = None
@@ -350,17 +350,27 @@ def e2e_loop(runner, steps, warmup):
     return ms, h2d, d2h
 
 
+KERNEL_SOURCES = ("ptx.cuh", "rpa_internal.h")
+
+
+def kernel_source_sha256(kernel_file: str) -> str:
+    """sha256 over the sources a kernel is compiled from (its .cu and the shared headers)."""
+    h = hashlib.sha256()
+    for name in (kernel_file,) + KERNEL_SOURCES:
+        with open(os.path.join(ROOT, "ragged_paged_attention_forward_b200", "csrc", name),
+                  "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def profile_traffic(kernel_file: str, key: str):
-    """DRAM bytes per launch from a committed ncu summary, if the kernel source it was taken
-    from is unchanged (sha256 of the source file)."""
+    """DRAM bytes per launch (scaled to the benchmark's workload) from the committed ncu
+    summary ``profiles/traffic.json``, or None when the kernel's sources changed since."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
-    src = os.path.join(ROOT, "ragged_paged_attention_forward_b200", "csrc", kernel_file)
     try:
         with open(path) as f:
             d = json.load(f)[key]
-        with open(src, "rb") as f:
-            sha = hashlib.sha256(f.read()).hexdigest()
-        if d.get("source_sha256") != sha:
+        if d.get("source_sha256") != kernel_source_sha256(kernel_file):
             return None
         return float(d["dram_bytes_per_launch"])
     except Exception:
@@ -432,6 +442,26 @@ def cpu_oracle_baseline(name, batch, target_s=12.0, table=None, count=None):
                       f"({rows_done} rows), oracle fp64 numpy"}
 
 
+def rank_seed_offset(rank: int) -> int:
+    """Seed offset of a rank's batch: every rank draws its own independent batch."""
+    return 1000 * rank
+
+
+def max_over_ranks(value: float, dist=None, device="cpu") -> float:
+    """The max of a per-rank number over all ranks (the job is as slow as its slowest rank)."""
+    if dist is None or not dist.is_available() or not dist.is_initialized():
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_gbps(world: int, bytes_per_rank_step: float, max_ms_per_step: float) -> float:
+    """Aggregate throughput of `world` ranks that each moved `bytes_per_rank_step` per step,
+    timed by the slowest rank."""
+    return world * bytes_per_rank_step / (max_ms_per_step * 1e-3) / 1e9
+
+
 def run_gpu(args):
     from ragged_paged_attention_forward_b200 import api  # noqa: F401  (fails loudly if unbuilt)
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -447,7 +477,7 @@ def run_gpu(args):
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
     name = args.workload
-    batch, mask = make_workload(name, seed_offset=1000 * rank)
+    batch, mask = make_workload(name, seed_offset=rank_seed_offset(rank))
     runner = Runner(name, batch, mask)
     table, count = runner.host_tables()
     w = work(batch, table, count)
@@ -477,14 +507,9 @@ def run_gpu(args):
     torch.cuda.synchronize()
     sampler.stop()
     step_ms = [s.elapsed_time(e) for s, e in evs]
-    total_ms = sum(step_ms)
-    if dist:
-        t = torch.tensor([total_ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), dist, "cuda")
     ms_per_step = total_ms / args.steps
-    units = w["step_bytes"] if w["flops"] / max(w["step_bytes"], 1) < 300 else w["flops"]
-    value = world * w["step_bytes"] / (ms_per_step * 1e-3) / 1e9
+    value = whole_job_gbps(world, w["step_bytes"], ms_per_step)
 
     # dominant kernel: the attention call alone (decode split + merge for this workload)
     attn_ms = statistics.mean(timed_loop(lambda: runner.step(False), args.steps, 2, flush))
@@ -510,12 +535,8 @@ def run_gpu(args):
 
     # end to end through the public API with host buffers
     e2e_ms, h2d, d2h = e2e_loop(runner, args.steps, 2)
-    e2e_ms_mean = statistics.mean(e2e_ms)
-    if dist:
-        t = torch.tensor([e2e_ms_mean], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms_mean = float(t.item())
-    e2e_val = world * w["step_bytes"] / (e2e_ms_mean * 1e-3) / 1e9
+    e2e_ms_mean = max_over_ranks(statistics.mean(e2e_ms), dist, "cuda")
+    e2e_val = whole_job_gbps(world, w["step_bytes"], e2e_ms_mean)
 
     # planner host time
     t0 = time.perf_counter()
@@ -623,8 +644,8 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=50)
-    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", default="decode", choices=list(WORKLOAD_TEXT))
     ap.add_argument("--no-secondary", action="store_true")

@@ -111,12 +111,31 @@ def _check(func: str, status: int):
         raise RPAError(func, status, last_error())
 
 
-def _host_i32(x) -> ctypes.Array:
+def _host_i32(x):
+    """A host int32 array for the C ABI: contiguous int32 CPU tensors and numpy arrays are
+    passed by pointer (the returned object keeps them alive for the call)."""
     if isinstance(x, torch.Tensor):
+        if x.device.type == "cpu" and x.dtype == torch.int32 and x.is_contiguous():
+            return _Keep(x, ctypes.cast(ctypes.c_void_p(x.data_ptr()), _I32P))
         x = x.detach().cpu().to(torch.int32).tolist()
     else:
+        try:
+            import numpy as np
+            if isinstance(x, np.ndarray) and x.dtype == np.int32 and x.flags.c_contiguous:
+                return _Keep(x, x.ctypes.data_as(_I32P))
+        except ImportError:  # pragma: no cover
+            pass
         x = [int(v) for v in x]
-    return (ctypes.c_int32 * max(1, len(x)))(*x)
+    arr = (ctypes.c_int32 * max(1, len(x)))(*x)
+    return _Keep(arr, ctypes.cast(arr, _I32P))
+
+
+class _Keep:
+    """A ctypes pointer argument that holds a reference to the buffer it points into."""
+
+    def __init__(self, owner, ptr):
+        self.owner = owner
+        self._as_parameter_ = ptr
 
 
 def _ptr(t: Optional[torch.Tensor]):
