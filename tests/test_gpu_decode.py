@@ -140,3 +140,12 @@ def test_group_tables_bit_exact_sparse_config_mask():
     assert np.array_equal(t, rt) and np.array_equal(c, rc)
     density = rc.sum() / (8 * mask.shape[-1])
     assert 0.15 < density < 0.35
+
+
+@pytest.mark.parametrize("nkb,nqb,density", [(16, 1, 0.5), (2048, 32, 0.02), (4128, 3, 0.3),
+                                              (4096, 2, 0.0), (64, 5, 1.0)])
+def test_group_tables_bit_exact_vector_path(nkb, nqb, density):
+    mask = wl.iid_block_mask(2, 8, nqb, nkb, seed=41 + nkb, density=density)
+    t, c = _tables_on_gpu(mask, 4)
+    rt, rc = orc.build_group_tables(mask, 4)
+    assert np.array_equal(t, rt) and np.array_equal(c, rc)
