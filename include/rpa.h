@@ -94,7 +94,7 @@ typedef struct rpa_plan_info {
   int32_t num_decode_items;    /* (sequence, key split) items of the decode kernel         */
   int32_t num_prefill_tiles;   /* (sequence, 128-query tile) items of the prefill kernel   */
   int32_t num_merge_rows;      /* query tokens whose decode splits need the LSE merge      */
-  int32_t launches_forward;    /* kernels rpa_forward launches (KV write included)         */
+  int32_t launches_forward;    /* kernels rpa_forward launches when given k_new/v_new      */
   int32_t launches_write;      /* kernels rpa_write_kv launches                            */
   int32_t decode_split_keys;   /* split size used                                          */
   int32_t reserved;

@@ -62,7 +62,8 @@ struct alignas(16) U4 {
 template <int D, int NT>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
-                        const __grid_constant__ CUtensorMap vmap, DecodeLaunch p) {
+                        const __grid_constant__ CUtensorMap vmap, DecodeLaunch p,
+                        const __grid_constant__ DecodeItemsInline inl) {
   using Geo = DecodeGeom<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -76,7 +77,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  const DecodeItem it = p.items[blockIdx.x];
+  const DecodeItem it = p.items ? p.items[blockIdx.x] : inl.v[blockIdx.x];
   const int h = blockIdx.y;
   const int Hq = p.num_q_heads;
   const int G = Hq / p.num_kv_heads;
@@ -87,6 +88,9 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   const int log2P = p.kv.log2_page;
 
   if (threadIdx.x == 0) {
+    // the merge kernel (launched with programmatic dependent launch) may get its CTAs onto
+    // the SMs now; it waits for this whole grid to finish before reading any partial result
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     for (int s = 0; s < Geo::kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kConsumerWarps);
@@ -107,6 +111,36 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             : p.kv.block_table + ((size_t)it.seq * p.kv.num_kv_heads + h) * p.kv.max_blocks;
     for (int j = lane; j < npg; j += 32) pages[j] = __ldg(bt_row + first_blk + j);
     __syncwarp();
+    if (p.k_new) {
+      // fused KV write: the new tokens (positions past .. kv_len-1) that fall in this CTA's key
+      // range are copied into their slots for KV head h before any page of the range is
+      // loaded; the proxy fence orders these plain stores before the TMA reads below.
+      const int lo = max(past, it.k_begin);
+      const int ntok = it.k_end - lo;
+      const int chunks = D / 8;  // 16-byte chunks per row
+      for (int idx = lane; idx < 2 * ntok * chunks; idx += 32) {
+        const int which = idx / (ntok * chunks);
+        const int rem = idx - which * ntok * chunks;
+        const int i = rem / chunks;
+        const int c = rem - i * chunks;
+        const int pos = lo + i;
+        const int tok = it.t0 + (pos - past);
+        const int page = pages[(pos >> log2P) - first_blk];
+        if (page < 0 || page >= p.kv.num_pages) {
+          atomicOr(p.err, kErrBadIndex);
+          continue;
+        }
+        const size_t row = p.kv.layout == 0
+                               ? ((size_t)page * P + (pos & (P - 1))) * p.num_kv_heads + h
+                               : (size_t)page * P + (pos & (P - 1));
+        const uint16_t* src = (which == 0 ? p.k_new : p.v_new) +
+                              ((size_t)tok * p.num_kv_heads + h) * D + c * 8;
+        uint16_t* dst = (which == 0 ? p.k_pool_w : p.v_pool_w) + row * D + c * 8;
+        *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
+      }
+      asm volatile("fence.proxy.async.global;" ::: "memory");
+      __syncwarp();
+    }
     if (lane == 0) {
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
@@ -347,7 +381,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 }
 
 template <int D>
-__global__ void __launch_bounds__(128) merge_kernel(MergeLaunch p) {
+__global__ void __launch_bounds__(128) merge_kernel(MergeLaunch p,
+                                                    const __grid_constant__ MergeRowsInline inl) {
+  // launched early (programmatic dependent launch): wait until the decode grid has finished
+  // and its partial results are visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const int Hq = p.num_q_heads;
@@ -355,7 +393,7 @@ __global__ void __launch_bounds__(128) merge_kernel(MergeLaunch p) {
   const int r = gw / Hq;
   const int hq = gw - r * Hq;
   const int G = Hq / p.num_kv_heads;
-  const MergeRow mr = p.rows[r];
+  const MergeRow mr = p.rows ? p.rows[r] : inl.v[r];
   const int h = hq / G;
   const int col = mr.local * G + (hq - h * G);
   constexpr int E = D / 32;
@@ -393,7 +431,8 @@ __global__ void __launch_bounds__(128) merge_kernel(MergeLaunch p) {
 }
 
 template <int D, int NT>
-cudaError_t launch_decode_t(const DecodeLaunch& p, cudaStream_t stream) {
+cudaError_t launch_decode_t(const DecodeLaunch& p, const DecodeItemsInline* inl,
+                            cudaStream_t stream) {
   using Geo = DecodeGeom<D>;
   // 4-D box over the pool: (dims, kv head, slot, page); head-major pools use one "head".
   CUtensorMap kmap, vmap;
@@ -405,33 +444,40 @@ cudaError_t launch_decode_t(const DecodeLaunch& p, cudaStream_t stream) {
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), Geo::kAlloc);
   if (e != cudaSuccess) return e;
   dim3 grid(p.num_items, p.num_kv_heads);
-  kern<<<grid, kDecodeThreads, Geo::kAlloc, stream>>>(kmap, vmap, p);
+  kern<<<grid, kDecodeThreads, Geo::kAlloc, stream>>>(kmap, vmap, p, *inl);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_decode(const DecodeLaunch& p, int nt, cudaStream_t stream) {
+cudaError_t launch_decode(const DecodeLaunch& p, const DecodeItemsInline* inl, int nt,
+                          cudaStream_t stream) {
   if (p.num_items <= 0) return cudaSuccess;
   if (p.head_dim == 128) {
-    if (nt == 1) return launch_decode_t<128, 1>(p, stream);
-    if (nt == 2) return launch_decode_t<128, 2>(p, stream);
-    return launch_decode_t<128, 4>(p, stream);
+    if (nt == 1) return launch_decode_t<128, 1>(p, inl, stream);
+    if (nt == 2) return launch_decode_t<128, 2>(p, inl, stream);
+    return launch_decode_t<128, 4>(p, inl, stream);
   }
-  if (nt == 1) return launch_decode_t<64, 1>(p, stream);
-  if (nt == 2) return launch_decode_t<64, 2>(p, stream);
-  return launch_decode_t<64, 4>(p, stream);
+  if (nt == 1) return launch_decode_t<64, 1>(p, inl, stream);
+  if (nt == 2) return launch_decode_t<64, 2>(p, inl, stream);
+  return launch_decode_t<64, 4>(p, inl, stream);
 }
 
-cudaError_t launch_merge(const MergeLaunch& p, cudaStream_t stream) {
+cudaError_t launch_merge(const MergeLaunch& p, const MergeRowsInline* inl, cudaStream_t stream) {
   if (p.num_rows <= 0) return cudaSuccess;
   const long warps = (long)p.num_rows * p.num_q_heads;
-  const int blocks = (int)((warps + 3) / 4);
-  if (p.head_dim == 128)
-    merge_kernel<128><<<blocks, 128, 0, stream>>>(p);
-  else
-    merge_kernel<64><<<blocks, 128, 0, stream>>>(p);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)((warps + 3) / 4));
+  cfg.blockDim = dim3(128);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (p.head_dim == 128) return cudaLaunchKernelEx(&cfg, merge_kernel<128>, p, *inl);
+  return cudaLaunchKernelEx(&cfg, merge_kernel<64>, p, *inl);
 }
 
 }  // namespace rpa

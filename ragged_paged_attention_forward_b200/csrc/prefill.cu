@@ -79,7 +79,8 @@ template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap,
                    const __grid_constant__ CUtensorMap kmap,
-                   const __grid_constant__ CUtensorMap vmap, PrefillLaunch p) {
+                   const __grid_constant__ CUtensorMap vmap, PrefillLaunch p,
+                   const __grid_constant__ PrefillTilesInline inl) {
   using Geo = PfGeom<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -108,7 +109,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int groups = Hq / hpc;
   const int tile_idx = blockIdx.x / groups;
   const int hq0 = (blockIdx.x - tile_idx * groups) * hpc;
-  const PrefillTile tile = p.tiles[tile_idx];
+  const PrefillTile tile = p.tiles ? p.tiles[tile_idx] : inl.v[tile_idx];
   const int h = hq0 / G;                            // KV head (shared by the pair)
   const int P = p.kv.page_size;
   const int log2P = p.kv.log2_page;
@@ -546,7 +547,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-cudaError_t launch_prefill(const PrefillLaunch& p, cudaStream_t stream) {
+cudaError_t launch_prefill(const PrefillLaunch& p, const PrefillTilesInline* inl,
+                           cudaStream_t stream) {
   if (p.num_tiles <= 0) return cudaSuccess;
   CUtensorMap qmap, kmap, vmap;
   cudaError_t e = encode_q_map(&qmap, p.q, p.num_tokens, p.num_q_heads, p.head_dim, kRows);
@@ -576,11 +578,13 @@ cudaError_t launch_prefill(const PrefillLaunch& p, cudaStream_t stream) {
     e = ensure_smem_attr(reinterpret_cast<const void*>(prefill_kernel<128>),
                          PfGeom<128>::kAlloc);
     if (e != cudaSuccess) return e;
-    prefill_kernel<128><<<grid, kThreads, PfGeom<128>::kAlloc, stream>>>(qmap, kmap, vmap, p);
+    prefill_kernel<128><<<grid, kThreads, PfGeom<128>::kAlloc, stream>>>(qmap, kmap, vmap, p,
+                                                                        *inl);
   } else {
     e = ensure_smem_attr(reinterpret_cast<const void*>(prefill_kernel<64>), PfGeom<64>::kAlloc);
     if (e != cudaSuccess) return e;
-    prefill_kernel<64><<<grid, kThreads, PfGeom<64>::kAlloc, stream>>>(qmap, kmap, vmap, p);
+    prefill_kernel<64><<<grid, kThreads, PfGeom<64>::kAlloc, stream>>>(qmap, kmap, vmap, p,
+                                                                      *inl);
   }
   return cudaGetLastError();
 }

@@ -65,6 +65,13 @@ struct rpa_plan_s {
   size_t off_dec = 0, off_merge = 0, off_pf = 0, meta_bytes = 0;
   size_t off_part_o = 0, off_part_lse = 0, ws_bytes = 0;
   std::vector<uint8_t> meta;  // host image of the metadata region
+  // every list short enough to travel as kernel parameters: no work-list copy at all
+  bool inline_lists = false;
+  DecodeItemsInline dec_inline;
+  MergeRowsInline merge_inline;
+  PrefillTilesInline pf_inline;
+  // pure decode plans fold the KV write into the decode kernel
+  bool fuse_write = false;
   int launches_forward = 0;
   int launches_write = 0;
   // fork/join events of a mixed batch (created on first use, on the device of that call)
@@ -316,8 +323,21 @@ rpa_status rpa_plan(const rpa_shape* shape, const int32_t* cu_seqlens_q,
     memcpy(plan->meta.data() + plan->off_pf, plan->pf_tiles.data(),
            plan->pf_tiles.size() * sizeof(PrefillTile));
 
+  plan->inline_lists = plan->dec_items.size() <= (size_t)kInlineItems &&
+                       plan->merge_rows.size() <= (size_t)kInlineItems &&
+                       plan->pf_tiles.size() <= (size_t)kInlineItems;
+  memset(&plan->dec_inline, 0, sizeof(plan->dec_inline));
+  memset(&plan->merge_inline, 0, sizeof(plan->merge_inline));
+  memset(&plan->pf_inline, 0, sizeof(plan->pf_inline));
+  if (plan->inline_lists) {
+    std::copy(plan->dec_items.begin(), plan->dec_items.end(), plan->dec_inline.v);
+    std::copy(plan->merge_rows.begin(), plan->merge_rows.end(), plan->merge_inline.v);
+    std::copy(plan->pf_tiles.begin(), plan->pf_tiles.end(), plan->pf_inline.v);
+  }
+  plan->fuse_write = plan->pf_tiles.empty() && !plan->dec_items.empty();
   plan->launches_write = T > 0 ? 1 : 0;
-  plan->launches_forward = plan->launches_write + (plan->dec_items.empty() ? 0 : 1) +
+  plan->launches_forward = (plan->fuse_write ? 0 : plan->launches_write) +
+                           (plan->dec_items.empty() ? 0 : 1) +
                            (plan->merge_rows.empty() ? 0 : 1) +
                            (plan->pf_tiles.empty() ? 0 : 1);
   *out_plan = plan;
@@ -430,13 +450,13 @@ rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const 
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     RPA_FAIL(RPA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
 
-  if (k_new) {
+  if (k_new && !plan->fuse_write) {
     st = write_kv_impl(plan, k_new, v_new, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k,
                        stream);
     if (st != RPA_OK) return st;
   }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
-  if (plan->meta_bytes > 0) {
+  if (plan->meta_bytes > 0 && !plan->inline_lists) {
     st = check_cuda(cudaMemcpyAsync(ws, plan->meta.data(), plan->meta_bytes,
                                     cudaMemcpyHostToDevice, stream),
                     "work-list copy");
@@ -482,7 +502,7 @@ rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const 
 
   if (!plan->pf_tiles.empty()) {
     PrefillLaunch p;
-    p.tiles = reinterpret_cast<const PrefillTile*>(ws + plan->off_pf);
+    p.tiles = plan->inline_lists ? nullptr : reinterpret_cast<const PrefillTile*>(ws + plan->off_pf);
     p.num_tiles = (int32_t)plan->pf_tiles.size();
     p.q = static_cast<const uint16_t*>(q);
     p.num_tokens = s.num_tokens;
@@ -497,12 +517,12 @@ rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const 
     p.group_count = group_count;
     p.err = err;
     p.kv = kv;
-    st = check_cuda(launch_prefill(p, pf_stream), "prefill launch");
+    st = check_cuda(launch_prefill(p, &plan->pf_inline, pf_stream), "prefill launch");
     if (st != RPA_OK) return st;
   }
   if (!plan->dec_items.empty()) {
     DecodeLaunch d;
-    d.items = reinterpret_cast<const DecodeItem*>(ws + plan->off_dec);
+    d.items = plan->inline_lists ? nullptr : reinterpret_cast<const DecodeItem*>(ws + plan->off_dec);
     d.num_items = (int32_t)plan->dec_items.size();
     d.rows_per_item = 8 * plan->decode_nt;
     d.q = static_cast<const uint16_t*>(q);
@@ -517,11 +537,16 @@ rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const 
     d.part_lse = reinterpret_cast<float*>(ws + plan->off_part_lse);
     d.err = err;
     d.kv = kv;
-    st = check_cuda(launch_decode(d, plan->decode_nt, stream), "decode launch");
+    const bool fused = k_new && plan->fuse_write;
+    d.k_new = fused ? static_cast<const uint16_t*>(k_new) : nullptr;
+    d.v_new = fused ? static_cast<const uint16_t*>(v_new) : nullptr;
+    d.k_pool_w = fused ? static_cast<uint16_t*>(k_pool) : nullptr;
+    d.v_pool_w = fused ? static_cast<uint16_t*>(v_pool) : nullptr;
+    st = check_cuda(launch_decode(d, &plan->dec_inline, plan->decode_nt, stream), "decode launch");
     if (st != RPA_OK) return st;
     if (!plan->merge_rows.empty()) {
       MergeLaunch m;
-      m.rows = reinterpret_cast<const MergeRow*>(ws + plan->off_merge);
+      m.rows = plan->inline_lists ? nullptr : reinterpret_cast<const MergeRow*>(ws + plan->off_merge);
       m.num_rows = (int32_t)plan->merge_rows.size();
       m.rows_per_item = d.rows_per_item;
       m.num_q_heads = s.num_q_heads;
@@ -531,7 +556,7 @@ rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const 
       m.part_lse = d.part_lse;
       m.out = d.out;
       m.lse = lse;
-      st = check_cuda(launch_merge(m, stream), "merge launch");
+      st = check_cuda(launch_merge(m, &plan->merge_inline, stream), "merge launch");
       if (st != RPA_OK) return st;
     }
   }

@@ -17,6 +17,10 @@ constexpr int kPrefillTileRows = 128;
 constexpr int kMaxSplitKeys = 4096;
 constexpr int kMinSplitKeys = 256;
 
+// Work lists of up to kInlineItems entries travel as kernel parameters (no host-to-device
+// copy); longer lists go through the workspace.
+constexpr int kInlineItems = 256;
+
 // Device error word codes (OR-ed together).
 enum DeviceErrorCode : int {
   kErrDecodeWait = 1 << 0,
@@ -57,6 +61,16 @@ struct PrefillTile {
 };
 static_assert(sizeof(PrefillTile) == 32, "PrefillTile layout");
 
+struct DecodeItemsInline {
+  DecodeItem v[kInlineItems];
+};
+struct MergeRowsInline {
+  MergeRow v[kInlineItems];
+};
+struct PrefillTilesInline {
+  PrefillTile v[kInlineItems];
+};
+
 struct PagedKV {
   const void* k_pool;
   const void* v_pool;
@@ -70,7 +84,7 @@ struct PagedKV {
 };
 
 struct DecodeLaunch {
-  const DecodeItem* items;
+  const DecodeItem* items;   // null: the items are the kernel's inline parameter list
   int32_t num_items;
   int32_t rows_per_item;     // 8 * NT: stride of the partial-result rows
   const uint16_t* q;         // bf16 [T, Hq, D]
@@ -85,10 +99,16 @@ struct DecodeLaunch {
   float* part_lse;           // [slots, Hkv, rows_per_item] (log2 domain)
   int* err;
   PagedKV kv;
+  // KV write fused into the decode kernel (pure decode batches): each CTA first writes the
+  // new tokens whose positions fall in its key range, for its KV head.  Null: no write.
+  const uint16_t* k_new;     // bf16 [T, Hkv, D]
+  const uint16_t* v_new;
+  uint16_t* k_pool_w;
+  uint16_t* v_pool_w;
 };
 
 struct MergeLaunch {
-  const MergeRow* rows;
+  const MergeRow* rows;      // null: inline parameter list
   int32_t num_rows;
   int32_t rows_per_item;
   int32_t num_q_heads;
@@ -101,7 +121,7 @@ struct MergeLaunch {
 };
 
 struct PrefillLaunch {
-  const PrefillTile* tiles;
+  const PrefillTile* tiles;  // null: inline parameter list
   int32_t num_tiles;
   const uint16_t* q;
   int32_t num_tokens;
@@ -139,9 +159,11 @@ struct WriteLaunch {
 
 // Launchers (return the cudaError_t of the launch).
 cudaError_t launch_write_kv(const WriteLaunch& p, cudaStream_t stream);
-cudaError_t launch_decode(const DecodeLaunch& p, int nt, cudaStream_t stream);
-cudaError_t launch_merge(const MergeLaunch& p, cudaStream_t stream);
-cudaError_t launch_prefill(const PrefillLaunch& p, cudaStream_t stream);
+cudaError_t launch_decode(const DecodeLaunch& p, const DecodeItemsInline* inl, int nt,
+                          cudaStream_t stream);
+cudaError_t launch_merge(const MergeLaunch& p, const MergeRowsInline* inl, cudaStream_t stream);
+cudaError_t launch_prefill(const PrefillLaunch& p, const PrefillTilesInline* inl,
+                           cudaStream_t stream);
 cudaError_t launch_group_tables(const uint8_t* mask, int B, int Hq, int Hkv, int nqb, int nkb,
                                 int32_t* table, int32_t* count, cudaStream_t stream);
 

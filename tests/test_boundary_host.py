@@ -73,7 +73,7 @@ def test_plan_classifies_and_sizes():
     assert info.num_decode_items == expect_items
     multi = sum(1 for kv in dec.kv_lens() if kv > split)
     assert info.num_merge_rows == multi
-    assert info.launches_forward == 2 + (1 if multi else 0)   # write + decode (+ merge)
+    assert info.launches_forward == 1 + (1 if multi else 0)   # decode (+ merge); write fused
 
     pf = wl.ragged_batch([300, 64], [300, 40], 8, 2, 64, 16, seed=1)
     info = plan_for(pf).info()
