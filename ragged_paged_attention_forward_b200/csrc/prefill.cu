@@ -20,10 +20,11 @@
 //                 S_h = Q_h K_j^T   (M=128 queries, N=128 keys, K=D; SMEM descriptors)
 //                 O_h += P_h V_j    (M=128, N=D, K=128 keys; P_h read from TMEM, V MN-major)
 //   warps 4-7   softmax of head A, warps 8-11 softmax of head B: thread r owns query row r
-//               (TMEM lane r); it loads S, masks, takes exp2 against a running reference max,
-//               writes P as bf16 over S and arrives.  The reference max only moves when a row's
-//               max grows by more than 2^8; only then is O rescaled in TMEM (after the previous
-//               P.V finished), so the softmax never waits on P.V otherwise.
+//               (TMEM lane r); it loads S, masks, takes exp2 against a reference max, writes P
+//               as bf16 over S and arrives.  The reference max is set by the first tile that
+//               shows the row a key and then held (no max pass per tile); only a tile whose row
+//               sum would pass 2^64 moves it, and only then is O rescaled in TMEM (after the
+//               previous P.V finished), so the softmax never waits on P.V otherwise.
 // TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+D) O_B [384,384+D).  Bounded waits.
 // An odd GQA group size runs with head B switched off.
 #include <cuda_bf16.h>
@@ -41,7 +42,7 @@ constexpr int kStagesV = 2;  // V tiles in flight
 constexpr int kRows = kPrefillTileRows;  // 128
 constexpr int kKeys = kPrefillTileKeys;  // 128
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleThreshold = 8.0f;  // log2 domain: P may grow up to 2^8 before O rescales
+constexpr float kMaxTileSum = 0x1p64f;  // a tile whose row sum passes this is redone
 // Registers: the CTA launches with kLaunchRegs per thread (3 warpgroups); the producer/MMA
 // warpgroup gives most of its share to the two softmax warpgroups.
 constexpr int kLaunchRegs = 168;
@@ -256,24 +257,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint64_t dk0 = smem_desc_sw128(smem_u32(Ks), 16, 1024);
       const uint64_t dv0 = smem_desc_sw128(smem_u32(Vs), Geo::kHalfBytes, 1024);
       auto issue_s = [&](int x, int j) {  // S_x = Q_x K_j^T into TMEM columns [128x, +128)
-        const uint64_t a0 = dq0 + (uint64_t)((x * Geo::kTileBytes) >> 4);
-        const uint64_t b0 = dk0 + (uint64_t)(((j % kStagesK) * Geo::kTileBytes) >> 4);
+        const uint32_t a_lo = (uint32_t)dq0 + (uint32_t)((x * Geo::kTileBytes) >> 4);
+        const uint32_t b_lo =
+            (uint32_t)dk0 + (uint32_t)(((j % kStagesK) * Geo::kTileBytes) >> 4);
+        const uint32_t a_hi = (uint32_t)(dq0 >> 32), b_hi = (uint32_t)(dk0 >> 32);
         const uint32_t d = tmem + x * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint64_t off = (uint64_t)(((kk >> 2) * Geo::kHalfBytes + (kk & 3) * 32) >> 4);
-          umma_ss(d, a0 + off, b0 + off, idesc_s, kk > 0 ? 1u : 0u);
+          const uint32_t off = (uint32_t)(((kk >> 2) * Geo::kHalfBytes + (kk & 3) * 32) >> 4);
+          if (kk == 0) umma_ss_lh<0>(d, a_lo + off, a_hi, b_lo + off, b_hi, idesc_s);
+          else umma_ss_lh<1>(d, a_lo + off, a_hi, b_lo + off, b_hi, idesc_s);
         }
         umma_commit(&s_full[x]);
       };
       auto issue_o = [&](int x, int j) {  // O_x += P_x V_j
-        const uint64_t b0 = dv0 + (uint64_t)(((j % kStagesV) * Geo::kTileBytes) >> 4);
+        const uint32_t b_lo =
+            (uint32_t)dv0 + (uint32_t)(((j % kStagesV) * Geo::kTileBytes) >> 4);
+        const uint32_t b_hi = (uint32_t)(dv0 >> 32);
         const uint32_t d = tmem + 256 + x * 128;
         const uint32_t a = tmem + x * 128;
         const uint32_t acc0 = j > 0 ? 1u : 0u;
 #pragma unroll
         for (int kk = 0; kk < kKeys / 16; ++kk)
-          umma_ts(d, a + kk * 8, b0 + (uint64_t)((kk * 2048) >> 4), idesc_o, kk > 0 ? 1u : acc0);
+          umma_ts_lh(d, a + kk * 8, b_lo + (uint32_t)((kk * 2048) >> 4), b_hi, idesc_o,
+                     kk > 0 ? 1u : acc0);
         umma_commit(&o_done[x]);
       };
       bool ok = warp_wait_bounded(q_full, 0, abort_flag, p.err, kErrPrefillWait) &&
@@ -394,84 +401,106 @@ __global__ void __launch_bounds__(kThreads, 1)
       const bool need_mask = partial || tile_last >= tile.kv_len ||
                              (p.causal && tile_last > past + tile.q_start);
       tmem_wait_ld();
-      // Row max of scale*S over the visible columns, with 8 independent accumulators so the
-      // reduction is a short tree, not a 128-long dependency chain.
-      float mx;
       uint32_t vis[kKeys / 32];  // visibility bits (masked tiles only)
       if (need_mask) {
-        float acc[8];
-#pragma unroll
-        for (int k = 0; k < 8; ++k) acc[k] = -CUDART_INF_F;
 #pragma unroll
         for (int w = 0; w < kKeys / 32; ++w) vis[w] = 0u;
 #pragma unroll
         for (int c = 0; c < kKeys; ++c) {
           const int kp = table ? __shfl_sync(0xffffffffu, ent, c >> log2P) + (c & (P - 1))
                                : ent + c;
-          const bool v = kp < lim;
-          vis[c >> 5] |= (v ? 1u : 0u) << (c & 31);
-          acc[c & 7] = fmaxf(acc[c & 7], v ? __uint_as_float(sr[c]) * sc : -CUDART_INF_F);
-        }
-        mx = fmaxf(fmaxf(fmaxf(acc[0], acc[1]), fmaxf(acc[2], acc[3])),
-                   fmaxf(fmaxf(acc[4], acc[5]), fmaxf(acc[6], acc[7])));
-      } else {
-        // scale*max(S) for a non-negative scale, scale*min(S) for a negative one
-        // 3-input max/min: two new values per instruction, four independent accumulators
-        float acc[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) acc[k] = __uint_as_float(sr[k]);
-        if (sc >= 0.f) {
-#pragma unroll
-          for (int c = 4; c < kKeys; c += 2)
-            acc[(c >> 1) & 3] = fmax3(acc[(c >> 1) & 3], __uint_as_float(sr[c]),
-                                      __uint_as_float(sr[c + 1]));
-          mx = fmaxf(fmax3(acc[0], acc[1], acc[2]), acc[3]) * sc;
-        } else {
-#pragma unroll
-          for (int c = 4; c < kKeys; c += 2)
-            acc[(c >> 1) & 3] = fmin3(acc[(c >> 1) & 3], __uint_as_float(sr[c]),
-                                      __uint_as_float(sr[c + 1]));
-          mx = fminf(fmin3(acc[0], acc[1], acc[2]), acc[3]) * sc;
+          vis[c >> 5] |= (kp < lim ? 1u : 0u) << (c & 31);
         }
       }
-      // reference max: moves only when the row max grows by more than the threshold
+      // The reference max m_ref comes from the first tile in which the row sees a key; later
+      // tiles take P against it with no max pass, so P may exceed 1.  That costs no precision
+      // (fp32 and bf16 are relative formats) until a tile's row sum passes 2^64; such a tile,
+      // rare in practice, is redone once against its own max, with O and l rescaled.
+      bool need_max = m_ref == -CUDART_INF_F;
       float fac = 1.f;
       bool rescale = false;
-      if (m_ref == -CUDART_INF_F) {
-        m_ref = mx;  // nothing accumulated yet (O and l are zero for this row)
-      } else if (mx > m_ref + kRescaleThreshold) {
-        fac = fast_exp2(m_ref - mx);
-        m_ref = mx;
-        rescale = true;
-      }
-      const float neg_m = m_ref == -CUDART_INF_F ? 0.f : -m_ref;
-      // P = exp2(scale*S - m): one packed FFMA per pair of elements and one EX2 per element;
-      // the row sum is kept in four packed partial sums
-      const uint64_t sc2 = f2_pack(sc, sc);
-      const uint64_t nm2 = f2_pack(neg_m, neg_m);
-      uint64_t rsum2[4];
+      float rs;
+#pragma unroll 1
+      for (int attempt = 0;; ++attempt) {
+        if (__any_sync(0xffffffffu, need_max)) {
+          // row max of scale*S over the visible columns: short trees of independent
+          // accumulators, not a 128-long dependency chain
+          float mx;
+          if (need_mask) {
+            float acc[8];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) rsum2[k] = 0ull;
+            for (int k = 0; k < 8; ++k) acc[k] = -CUDART_INF_F;
 #pragma unroll
-      for (int c = 0; c < kKeys; c += 2) {
-        float t0, t1;
-        f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2),
-                  t0, t1);
-        float p0 = fast_exp2(t0);
-        float p1 = fast_exp2(t1);
-        if (need_mask) {
-          p0 = (vis[c >> 5] >> (c & 31)) & 1u ? p0 : 0.f;
-          p1 = (vis[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u ? p1 : 0.f;
+            for (int c = 0; c < kKeys; ++c)
+              acc[c & 7] = fmaxf(acc[c & 7], (vis[c >> 5] >> (c & 31)) & 1u
+                                                 ? __uint_as_float(sr[c]) * sc
+                                                 : -CUDART_INF_F);
+            mx = fmaxf(fmaxf(fmaxf(acc[0], acc[1]), fmaxf(acc[2], acc[3])),
+                       fmaxf(fmaxf(acc[4], acc[5]), fmaxf(acc[6], acc[7])));
+          } else {
+            // scale*max(S) for a non-negative scale, scale*min(S) for a negative one;
+            // 3-input max/min: two new values per instruction, four accumulators
+            float acc[4];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[k] = __uint_as_float(sr[k]);
+            if (sc >= 0.f) {
+#pragma unroll
+              for (int c = 4; c < kKeys; c += 2)
+                acc[(c >> 1) & 3] = fmax3(acc[(c >> 1) & 3], __uint_as_float(sr[c]),
+                                          __uint_as_float(sr[c + 1]));
+              mx = fmaxf(fmax3(acc[0], acc[1], acc[2]), acc[3]) * sc;
+            } else {
+#pragma unroll
+              for (int c = 4; c < kKeys; c += 2)
+                acc[(c >> 1) & 3] = fmin3(acc[(c >> 1) & 3], __uint_as_float(sr[c]),
+                                          __uint_as_float(sr[c + 1]));
+              mx = fminf(fmin3(acc[0], acc[1], acc[2]), acc[3]) * sc;
+            }
+          }
+          if (need_max && mx > m_ref) {  // mx = -inf: still no visible key
+            if (m_ref != -CUDART_INF_F) {
+              fac = fast_exp2(m_ref - mx);
+              rescale = true;
+            }
+            m_ref = mx;
+          }
         }
-        rsum2[(c >> 1) & 3] = f2_add(rsum2[(c >> 1) & 3], f2_pack(p0, p1));
-        sr[c >> 1] = pack_bf16(p0, p1);  // P as bf16 pairs, over the consumed S values
-      }
-      float rs = 0.f;
+        const float neg_m = m_ref == -CUDART_INF_F ? 0.f : -m_ref;
+        // P = exp2(scale*S - m): one packed FFMA per pair of elements and one EX2 per
+        // element; the row sum is kept in four packed partial sums
+        const uint64_t sc2 = f2_pack(sc, sc);
+        const uint64_t nm2 = f2_pack(neg_m, neg_m);
+        uint64_t rsum2[4];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        float a, b;
-        f2_unpack(rsum2[k], a, b);
-        rs += a + b;
+        for (int k = 0; k < 4; ++k) rsum2[k] = 0ull;
+#pragma unroll
+        for (int c = 0; c < kKeys; c += 2) {
+          float t0, t1;
+          f2_unpack(
+              f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2), t0,
+              t1);
+          float p0 = fast_exp2(t0);
+          float p1 = fast_exp2(t1);
+          if (need_mask) {
+            p0 = (vis[c >> 5] >> (c & 31)) & 1u ? p0 : 0.f;
+            p1 = (vis[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u ? p1 : 0.f;
+          }
+          rsum2[(c >> 1) & 3] = f2_add(rsum2[(c >> 1) & 3], f2_pack(p0, p1));
+          sr[c >> 1] = pack_bf16(p0, p1);  // P as bf16 pairs, over the consumed S values
+        }
+        rs = 0.f;
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          float a, b;
+          f2_unpack(rsum2[k], a, b);
+          rs += a + b;
+        }
+        const bool over = !(rs <= kMaxTileSum);
+        if (attempt > 0 || !__any_sync(0xffffffffu, over)) break;
+        need_max = over;
+#pragma unroll
+        for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(ts + c * 32, sr + c * 32);
+        tmem_wait_ld();
       }
       l = l * fac + rs;
 #pragma unroll

@@ -180,8 +180,8 @@ rpa_status rpa_plan(const rpa_shape* shape, const int32_t* cu_seqlens_q,
              o.decode_split_keys, kDecodeStageKeys, kDecodeStageKeys, kMaxSplitKeys);
   if (o.sparse && s.layout != RPA_LAYOUT_HEAD_MAJOR)
     RPA_FAIL(RPA_ERR_UNSUPPORTED, "block-union tables need the KV-head-major layout");
-  if (o.sparse && s.page_size > kPrefillTileKeys)
-    RPA_FAIL(RPA_ERR_UNSUPPORTED, "block-union tables need page_size <= %d", kPrefillTileKeys);
+  if (o.sparse && s.page_size > kMaxSparsePage)
+    RPA_FAIL(RPA_ERR_UNSUPPORTED, "block-union tables need page_size <= %d", kMaxSparsePage);
 
   // ---- lengths
   if (B > 0) {

@@ -14,6 +14,7 @@ namespace rpa {
 constexpr int kDecodeStageKeys = 64;
 constexpr int kPrefillTileKeys = 128;
 constexpr int kPrefillTileRows = 128;
+constexpr int kMaxSparsePage = 128;  // block-union tables: largest page (= table block) size
 constexpr int kMaxSplitKeys = 4096;
 constexpr int kMinSplitKeys = 256;
 
