@@ -6,9 +6,11 @@
 
 A step is one pass of the whole hot path over one synthetic batch: the fused call
 (KV-cache write + attention, with the decode splits merged), plus the block-union table
-build for the sparse workload.  Inputs are resident in HBM; L2 (126 MB) is flushed with a
-256 MB write before every timed step and the flush is not timed.  Each step is timed with
-CUDA events on the stream the kernels run on.  The headline line is the decode workload
+build for the sparse workload.  Inputs are resident in HBM and larger than L2 (126 MB): the
+KV pool rotates over copies (at least three, and together more than twice L2), so that each
+step reads memory the previous steps did not touch.  K steps run back to back between two
+CUDA events on the stream the kernels run on, with a barrier and a synchronize on both
+sides.  The headline line is the decode workload
 (Llama-3-8B attention, batch 64, kv_len ~ U[512, 8192]) in HBM GB/s; the prefill, mixed and
 sparse workloads are reported as secondary objects on the same line.
 
@@ -223,6 +225,9 @@ def make_workload(name: str, seed_offset: int = 0):
     return wl.sparse(seed=seed, poison=False)
 
 
+L2_BYTES = 126 << 20
+
+
 class Runner:
     """Holds one batch on the device and runs steps through the C ABI."""
 
@@ -249,6 +254,12 @@ class Runner:
                                      device="cuda")
         else:
             self.table = self.count = None
+        # the KV pool and copies of it, so that consecutive steps read disjoint memory
+        pool_bytes = 2 * self.d["k_pool"].numel() * self.d["k_pool"].element_size()
+        n = max(3, -(-2 * L2_BYTES // pool_bytes) + 1)
+        self.pools = [(self.d["k_pool"], self.d["v_pool"])] + [
+            (self.d["k_pool"].clone(), self.d["v_pool"].clone()) for _ in range(n - 1)]
+        self.pool_bytes_total = n * pool_bytes
         self.plan = self.make_plan()
         self.ws = torch.empty(max(self.plan.workspace_bytes, 256), dtype=torch.uint8,
                               device="cuda")
@@ -270,11 +281,12 @@ class Runner:
             self.api.rpa_build_group_tables(self.mask_d, self.batch.num_kv_heads, self.table,
                                             self.count, stream)
 
-    def step(self, fused=True, stream=None):
+    def step(self, fused=True, stream=None, i=0):
         d = self.d
+        kp, vp = self.pools[i % len(self.pools)]
         self.tables(stream)
         self.api.rpa_forward(self.plan, d["q"], d["k_new"] if fused else None,
-                             d["v_new"] if fused else None, d["k_pool"], d["v_pool"],
+                             d["v_new"] if fused else None, kp, vp,
                              d["block_table"], d["cu_seqlens_q"], d["seq_lens_k"], self.table,
                              self.count, self.batch.scale, self.out, self.lse, self.ws, stream)
 
@@ -286,28 +298,28 @@ class Runner:
         return self.table.cpu().numpy(), self.count.cpu().numpy()
 
 
-def timed_loop(fn, steps, warmup, flush):
-    """Per-step CUDA-event durations (ms) of fn(), L2 flushed (untimed) before each step."""
+def timed_loop(fn, steps, warmup):
+    """Mean CUDA-event duration (ms) of fn(i) over `steps` calls run back to back on the
+    current stream after `warmup` untimed calls; fn(i) reads the i-th pool copy."""
     stream = torch.cuda.current_stream()
-    for _ in range(warmup):
-        flush.zero_()
-        fn()
+    for i in range(warmup):
+        fn(i)
     torch.cuda.synchronize()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(steps)]
-    for s, e in evs:
-        flush.zero_()
-        s.record(stream)
-        fn()
-        e.record(stream)
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for i in range(steps):
+        fn(warmup + i)
+    e.record(stream)
     torch.cuda.synchronize()
-    return [s.elapsed_time(e) for s, e in evs]
+    return s.elapsed_time(e) / steps
 
 
 def e2e_loop(runner, steps, warmup):
     """End to end through the public API: plan on the host, copy the step's inputs from one
-    pinned host buffer (one H2D copy), run the fused step, read the output back.  Returns
-    (ms list, h2d bytes, d2h bytes)."""
+    pinned host buffer (one H2D copy), run the fused step, read the output back; the KV pool
+    rotates over copies so that no step finds K/V in L2.  Returns (ms list, h2d bytes, d2h
+    bytes)."""
     b = runner.batch
     names = ["q", "k_new", "v_new", "block_table", "cu_seqlens_q", "seq_lens_k"]
     srcs = [getattr(b, k).contiguous() for k in names]
@@ -329,35 +341,118 @@ def e2e_loop(runner, steps, warmup):
     h2d = total
     d2h = out_host.numel() * out_host.element_size()
     stream = torch.cuda.current_stream()
-    d = runner.d
+    pools = runner.pools
 
-    def one():
+    def one(i):
+        kp, vp = pools[i % len(pools)]
         plan = runner.make_plan()
         dev.copy_(host, non_blocking=True)
         if runner.sparse:
             runner.api.rpa_build_group_tables(views["mask"], b.num_kv_heads, runner.table,
                                               runner.count)
-        runner.api.rpa_forward(plan, views["q"], views["k_new"], views["v_new"], d["k_pool"],
-                               d["v_pool"], views["block_table"], views["cu_seqlens_q"],
+        runner.api.rpa_forward(plan, views["q"], views["k_new"], views["v_new"], kp, vp,
+                               views["block_table"], views["cu_seqlens_q"],
                                views["seq_lens_k"], runner.table, runner.count, b.scale,
                                runner.out, runner.lse, runner.ws)
         out_host.copy_(runner.out, non_blocking=True)
         return plan
 
-    for _ in range(warmup):
-        one()
+    for i in range(warmup):
+        one(i)
     torch.cuda.synchronize()
     ms = []
-    for _ in range(steps):
+    for i in range(steps):
         s = torch.cuda.Event(enable_timing=True)
         e = torch.cuda.Event(enable_timing=True)
         s.record(stream)
-        plan = one()
+        plan = one(warmup + i)
         e.record(stream)
         e.synchronize()
         ms.append(s.elapsed_time(e))
         del plan
     return ms, h2d, d2h
+
+
+def e2e_pipelined(runner, steps, warmup):
+    """End to end as a serving loop runs it: every step plans on the host, copies its inputs
+    from pinned host memory (one H2D copy on a copy stream), runs the fused step on the
+    compute stream and copies the output back (D2H on a second copy stream).  Two device
+    input and output buffers let step i+1's H2D and step i-1's D2H overlap step i's kernels,
+    and the host plans ahead while the GPU works; the KV pool rotates over copies so that no
+    step finds K/V in L2.  Returns (ms per step, h2d bytes, d2h bytes): the time from the
+    first step's start to the last step's output landing on the host, divided by the number
+    of steps."""
+    b = runner.batch
+    names = ["q", "k_new", "v_new", "block_table", "cu_seqlens_q", "seq_lens_k"]
+    srcs = [getattr(b, k).contiguous() for k in names]
+    if runner.sparse:
+        names.append("mask")
+        srcs.append(runner.mask.contiguous())
+    offs, total = [], 0
+    for t in srcs:
+        offs.append(total)
+        total += (t.numel() * t.element_size() + 255) // 256 * 256
+    host = torch.empty(total, dtype=torch.uint8).pin_memory()
+    for t, o in zip(srcs, offs):
+        nb = t.numel() * t.element_size()
+        host[o:o + nb].copy_(t.view(torch.uint8).reshape(-1))
+    devs = [torch.empty(total, dtype=torch.uint8, device="cuda") for _ in range(2)]
+    views = []
+    for dev in devs:
+        v = {}
+        for k, t, o in zip(names, srcs, offs):
+            nb = t.numel() * t.element_size()
+            v[k] = dev[o:o + nb].view(t.dtype).view(t.shape)
+        views.append(v)
+    outs = [torch.empty_like(runner.out) for _ in range(2)]
+    outs_host = [torch.empty(runner.out.shape, dtype=runner.out.dtype).pin_memory()
+                 for _ in range(2)]
+    h2d = total
+    d2h = outs_host[0].numel() * outs_host[0].element_size()
+    compute = torch.cuda.current_stream()
+    up, down = torch.cuda.Stream(), torch.cuda.Stream()
+    h2d_done = [torch.cuda.Event() for _ in range(2)]
+    comp_done = [torch.cuda.Event() for _ in range(2)]
+    d2h_done = [torch.cuda.Event() for _ in range(2)]
+    pools = runner.pools
+
+    def one(i):
+        k = i & 1
+        kp, vp = pools[i % len(pools)]
+        plan = runner.make_plan()
+        up.wait_event(comp_done[k])          # step i-2 has finished reading devs[k]
+        with torch.cuda.stream(up):
+            devs[k].copy_(host, non_blocking=True)
+        h2d_done[k].record(up)
+        compute.wait_event(h2d_done[k])
+        compute.wait_event(d2h_done[k])      # step i-2's output has left outs[k]
+        v = views[k]
+        if runner.sparse:
+            runner.api.rpa_build_group_tables(v["mask"], b.num_kv_heads, runner.table,
+                                              runner.count)
+        runner.api.rpa_forward(plan, v["q"], v["k_new"], v["v_new"], kp, vp,
+                               v["block_table"], v["cu_seqlens_q"], v["seq_lens_k"],
+                               runner.table, runner.count, b.scale, outs[k], runner.lse,
+                               runner.ws)
+        comp_done[k].record(compute)
+        down.wait_event(comp_done[k])
+        with torch.cuda.stream(down):
+            outs_host[k].copy_(outs[k], non_blocking=True)
+        d2h_done[k].record(down)
+        return plan
+
+    plans = [one(i) for i in range(warmup)]
+    torch.cuda.synchronize()
+    plans.clear()
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(compute)
+    for i in range(steps):
+        plans.append(one(warmup + i))
+    down.wait_stream(compute)
+    end.record(down)
+    end.synchronize()
+    return start.elapsed_time(end) / steps, h2d, d2h
 
 
 KERNEL_SOURCES = ("ptx.cuh", "rpa_internal.h")
@@ -387,14 +482,12 @@ def profile_traffic(kernel_file: str, key: str):
         return None
 
 
-def measure(name, runner, steps, warmup, flush, peaks):
+def measure(name, runner, steps, warmup, peaks):
     b = runner.batch
     table, count = runner.host_tables()
     w = work(b, table, count)
-    step_ms = timed_loop(lambda: runner.step(True), steps, warmup, flush)
-    attn_ms = timed_loop(lambda: runner.step(False), steps, warmup, flush)
-    ms = statistics.mean(step_ms)
-    ams = statistics.mean(attn_ms)
+    ms = timed_loop(lambda i: runner.step(True, i=i), steps, warmup)
+    ams = timed_loop(lambda i: runner.step(False, i=i), steps, warmup)
     res = {"workload": WORKLOAD_TEXT[name], "ms_per_step": ms, "attn_ms": ams,
            "tokens_per_s": b.num_tokens / (ms * 1e-3),
            "step_GBps": w["step_bytes"] / (ms * 1e-3) / 1e9,
@@ -484,7 +577,6 @@ def run_gpu(args):
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     peaks, peak_src = load_peaks()
-    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
 
     name = args.workload
     batch, mask = make_workload(name, seed_offset=rank_seed_offset(rank))
@@ -493,36 +585,33 @@ def run_gpu(args):
     w = work(batch, table, count)
 
     # headline: the fused step, K timed steps after W warm-up steps, clocks sampled meanwhile
-    for _ in range(args.warmup):
-        flush.zero_()
-        runner.step(True)
+    for i in range(args.warmup):
+        runner.step(True, i=i)
     torch.cuda.synchronize()
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     sampler = ClockSampler(torch.cuda.current_device()).start()
     stream = torch.cuda.current_stream()
-    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
-           for _ in range(args.steps)]
+    ev_s = torch.cuda.Event(enable_timing=True)
+    ev_e = torch.cuda.Event(enable_timing=True)
     t_wall0 = time.perf_counter()
-    for s, e in evs:
-        flush.zero_()
-        s.record(stream)
-        runner.step(True)
-        e.record(stream)
+    ev_s.record(stream)
+    for i in range(args.steps):
+        runner.step(True, i=args.warmup + i)
+    ev_e.record(stream)
     torch.cuda.synchronize()
     t_wall = time.perf_counter() - t_wall0
     if dist:
         dist.barrier()
     torch.cuda.synchronize()
     sampler.stop()
-    step_ms = [s.elapsed_time(e) for s, e in evs]
-    total_ms = max_over_ranks(sum(step_ms), dist, "cuda")
+    total_ms = max_over_ranks(ev_s.elapsed_time(ev_e), dist, "cuda")
     ms_per_step = total_ms / args.steps
     value = whole_job_gbps(world, w["step_bytes"], ms_per_step)
 
     # dominant kernel: the attention call alone (decode split + merge for this workload)
-    attn_ms = statistics.mean(timed_loop(lambda: runner.step(False), args.steps, 2, flush))
+    attn_ms = timed_loop(lambda i: runner.step(False, i=i), args.steps, 2)
     attn_gbps = w["attn_bytes"] / (attn_ms * 1e-3) / 1e9
     kernel_file = "decode.cu" if name in ("decode", "mixed") else "prefill.cu"
     bound = "hbm" if name in ("decode", "mixed") else "tensor"
@@ -543,10 +632,14 @@ def run_gpu(args):
                 "kernel": "rpa_forward attention (tcgen05 prefill)",
                 "peak_source": f"{peak_src} (cuBLAS bf16 burst)"}
 
-    # end to end through the public API with host buffers
+    # end to end through the public API with host buffers: one step at a time (latency) and
+    # as a pipelined serving loop (throughput, the reported value)
     e2e_ms, h2d, d2h = e2e_loop(runner, args.steps, 2)
     e2e_ms_mean = max_over_ranks(statistics.mean(e2e_ms), dist, "cuda")
-    e2e_val = whole_job_gbps(world, w["step_bytes"], e2e_ms_mean)
+    e2e_serial = whole_job_gbps(world, w["step_bytes"], e2e_ms_mean)
+    e2e_pipe_ms, _, _ = e2e_pipelined(runner, args.steps, 4)
+    e2e_pipe_ms = max_over_ranks(e2e_pipe_ms, dist, "cuda")
+    e2e_val = whole_job_gbps(world, w["step_bytes"], e2e_pipe_ms)
 
     # planner host time
     t0 = time.perf_counter()
@@ -560,7 +653,10 @@ def run_gpu(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": {"workload": WORKLOAD_TEXT[name], "per_rank_batch": "independent seed per rank",
-                   "l2": "256 MB write between timed steps (untimed); KV pool > L2",
+                   "l2": f"inputs larger than L2: the KV pool rotates over "
+                         f"{len(runner.pools)} copies ({runner.pool_bytes_total / 1e9:.2f} GB), "
+                         f"so each step reads memory the previous steps did not touch; "
+                         f"steps run back to back, no flush",
                    "step": "rpa_forward fused (KV write + attention + LSE merge)"
                            + (" + group-table build" if runner.sparse else ""),
                    "tokens_per_step": batch.num_tokens * world,
@@ -569,9 +665,13 @@ def run_gpu(args):
                    "planner_host_us": planner_us},
         "roofline": roof,
         "e2e": {"value": e2e_val, "unit": "GB/s", "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms_mean,
-                "includes": "host planner + one pinned H2D copy of q/k_new/v_new/block "
-                            "table/lengths + fused step + D2H of out"},
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_pipe_ms,
+                "includes": "every step: host planner + one pinned H2D copy of q/k_new/v_new/"
+                            "block table/lengths + fused step + D2H of out, pipelined over "
+                            "two buffers (copy streams overlap the neighbouring steps' kernels)",
+                "serial_value": e2e_serial, "serial_ms_per_step": e2e_ms_mean,
+                "serial_includes": "the same, one step at a time (each step waits for the "
+                                   "previous one's output)"},
         "gpu_launches": runner.launches_step * args.steps,
         "clocks": sampler.summary(),
         "wall_s_timed_region": t_wall,
@@ -594,7 +694,7 @@ def run_gpu(args):
                 continue
             b2, m2 = make_workload(other)
             r2 = Runner(other, b2, m2)
-            res = measure(other, r2, args.steps, args.warmup, flush, peaks)
+            res = measure(other, r2, args.steps, args.warmup, peaks)
             if other in ("prefill", "sparse"):
                 res["frac_of_bf16_peak"] = res["attn_TFLOPs"] / peaks["bf16_tflops"]
                 res["frac_of_bf16_sustained"] = res["attn_TFLOPs"] / peaks[
