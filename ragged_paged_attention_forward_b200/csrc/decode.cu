@@ -74,6 +74,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + Geo::kBarOff);
   uint64_t* empty = full + Geo::kStages;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + Geo::kStages);
+  volatile int* never = abort_flag + 1;  // stays 0: time-bounded waits that ignore an abort
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -96,6 +97,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       mbar_init(&empty[s], kConsumerWarps);
     }
     *abort_flag = 0;
+    *never = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -177,7 +179,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       if (*abort_flag) {
         // let copies already in flight land before the CTA's shared memory goes away
         for (int s = max(0, issued - Geo::kStages); s < issued; ++s)
-          wait_bounded(&full[s % Geo::kStages], (s / Geo::kStages) & 1, abort_flag, nullptr, 0,
+          wait_bounded(&full[s % Geo::kStages], (s / Geo::kStages) & 1, never, nullptr, 0,
                        kWaitTimeoutNs / 8);
       }
     }

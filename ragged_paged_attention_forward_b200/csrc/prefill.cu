@@ -76,6 +76,26 @@ struct alignas(16) U4 {
   uint32_t x, y, z, w;
 };
 
+// Number of entries of the ascending list t[0, n) that are below `limit`, found by the whole
+// warp: each round probes 32 evenly spaced entries at once and keeps the one gap where the
+// answer lies, so a 2048-entry table takes three dependent loads instead of eleven.
+__device__ __forceinline__ int warp_count_below(const int32_t* t, int n, int limit) {
+  const int lane = threadIdx.x & 31;
+  int lo = 0, hi = n;  // t[i] < limit for i < lo; t[i] >= limit for i >= hi
+  while (hi - lo > 32) {
+    const int step = (hi - lo + 32) / 33;
+    const int idx = lo + (lane + 1) * step;
+    const bool below = idx < hi && __ldg(t + idx) < limit;
+    const int c = __popc(__ballot_sync(0xffffffffu, below));
+    const int nlo = c > 0 ? lo + c * step + 1 : lo;
+    const int nhi = (c < 32 && lo + (c + 1) * step < hi) ? lo + (c + 1) * step : hi;
+    lo = nlo;
+    hi = nhi;
+  }
+  const bool below = lo + lane < hi && __ldg(t + lo + lane) < limit;
+  return lo + __popc(__ballot_sync(0xffffffffu, below));
+}
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap,
@@ -101,6 +121,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* mma_done = o_done + 2;
   uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(smem + Geo::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Geo::kMiscOff + 8);
+  volatile int* never = reinterpret_cast<volatile int*>(smem + Geo::kMiscOff + 12);  // stays 0
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -126,12 +147,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const size_t row = (size_t)tile.seq * p.num_kv_heads + h;
     table = p.group_table + row * p.kv.max_blocks;
     const int cnt = min(__ldg(p.group_count + row), p.kv.max_blocks);
-    int lo = 0, hi = max(cnt, 0);  // entries whose block starts before kv_hi (ascending)
-    while (lo < hi) {
-      const int mid = (lo + hi) >> 1;
-      if ((__ldg(table + mid) << log2P) < kv_hi) lo = mid + 1; else hi = mid;
-    }
-    n_entries = lo;
+    // entries (ascending block ids) whose block starts before kv_hi; every warp of the CTA
+    // runs this search with all its lanes
+    n_entries = warp_count_below(table, max(cnt, 0), (kv_hi + P - 1) >> log2P);
     const int per = kKeys >> log2P;
     n_tiles = (n_entries + per - 1) / per;
   } else {
@@ -155,6 +173,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
+    *never = 0;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -234,12 +253,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (stop) break;
       }
-      if (*abort_flag) {  // let copies in flight land before shared memory goes away
-        wait_bounded(q_full, 0, abort_flag, nullptr, 0, kWaitTimeoutNs / 8);
+      if (*abort_flag) {
+        // let copies in flight land before shared memory goes away (time-bounded only: the
+        // raised abort flag must not cut these waits short)
+        wait_bounded(q_full, 0, never, nullptr, 0, kWaitTimeoutNs / 8);
         for (int kv = 0; kv < 2; ++kv) {
           const int ns = kv == 0 ? kStagesK : kStagesV;
           for (int j = max(0, issued[kv] - ns); j < issued[kv]; ++j)
-            wait_bounded(kv == 0 ? &k_full[j % ns] : &v_full[j % ns], (j / ns) & 1, abort_flag,
+            wait_bounded(kv == 0 ? &k_full[j % ns] : &v_full[j % ns], (j / ns) & 1, never,
                          nullptr, 0, kWaitTimeoutNs / 8);
         }
       }
@@ -354,7 +375,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // every MMA issued so far must finish before TMEM is released
       if (lane == 0) umma_commit(mma_done);
       __syncwarp();
-      warp_wait_bounded(mma_done, 0, abort_flag, nullptr, 0, kWaitTimeoutNs / 8);
+      warp_wait_bounded(mma_done, 0, never, nullptr, 0, kWaitTimeoutNs / 8);
     }
   }
   } else if ((warp - 4) / 4 < hpc) {

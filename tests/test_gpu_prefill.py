@@ -7,7 +7,8 @@ import torch
 from oracle import rpa_oracle as orc
 from ragged_paged_attention_forward_b200 import api
 from ragged_paged_attention_forward_b200 import workloads as wl
-from tests.rpa_testing import (assert_close, assert_lse_close, oracle_forward, run_forward)
+from tests.rpa_testing import (assert_close, assert_lse_close, oracle_forward, plan_for,
+                                run_forward, to_device)
 
 pytestmark = pytest.mark.gpu
 
@@ -150,6 +151,26 @@ def test_mixed_config_full_size_sampled(shuffle):
     assert_close(out, ref, rows=rows)
     assert_lse_close(lse, ref_lse, rows=rows)
     assert torch.isfinite(out.float()).all()
+
+
+def test_mixed_output_is_stream_ordered():
+    # The tensor-core kernel runs on the library's side stream beside the decode kernel: work
+    # queued on the caller's stream right after the call must see every output row.
+    b = wl.ragged_batch([700, 3000, 1500, 40], [300, 1, 1, 40], 8, 2, 128, 16, seed=62)
+    plan = plan_for(b)
+    assert plan.info().batch_class == api.CLASS_MIXED
+    d = to_device(b)
+    out = torch.full_like(d["q"], float("nan"))
+    ws = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device="cuda")
+    api.rpa_forward(plan, d["q"], d["k_new"], d["v_new"], d["k_pool"], d["v_pool"],
+                    d["block_table"], d["cu_seqlens_q"], d["seq_lens_k"], None, None, b.scale,
+                    out, None, ws)
+    snap = out.clone()  # queued on the same stream, no synchronisation in between
+    torch.cuda.synchronize()
+    assert api.rpa_device_error(clear=True) == 0
+    assert torch.equal(snap, out)
+    ref, _, _, _ = oracle_forward(b)
+    assert_close(out.cpu(), ref)
 
 
 # ------------------------------------------------------------------ sparse block-union mode
