@@ -153,6 +153,53 @@ RPA_API rpa_status rpa_write_kv(rpa_plan_t plan, const void* k_new, const void* 
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Rotary position embedding applied by rpa_rotary_write_kv ("[WebGPU] Optimized
+ * PagedAttention implementation (2/n)", commit "Phase 1b.2": the rotary program rotates Q and
+ * K before the K/V scatter, with position_id = past_b + s and dims >= rotary_dim copied
+ * unchanged; interleaved or split pairing).
+ *
+ *   cos_cache, sin_cache  device bf16 [max_position, rotary_dim / 2]: row p holds cos and
+ *                         sin of the angles of position p, one per rotated pair.
+ *   max_position          rows of the caches; every position must be below it.
+ *   rotary_dim            rotated dims per head: a multiple of 16, <= head_dim.
+ *   interleaved           1: pair j is (x[2j], x[2j+1]); 0: pair j is (x[j], x[j + rd/2]).
+ * Pair j of a row at position p becomes (x1 c - x2 s, x1 s + x2 c) with c = cos[p, j],
+ * s = sin[p, j]; arithmetic in fp32, results rounded to bf16 (nearest even).
+ */
+typedef struct rpa_rotary {
+  const void* cos_cache;
+  const void* sin_cache;
+  int32_t max_position;
+  int32_t rotary_dim;
+  int32_t interleaved;
+  int32_t reserved;            /* must be zero */
+} rpa_rotary;
+
+/*
+ * rpa_rotary_write_kv -- the step's input pass: take the new tokens' Q, K and V (separate, or
+ * packed per token as [Q | K | V] columns: "... (2/n)", packed-QKV commit), rotate Q and K
+ * by their positions (optional), write the queries to q_out and scatter K and V into their
+ * cache slots (rpa_write_kv's index rule).  rpa_forward then runs on q_out with
+ * k_new = v_new = NULL.  This pass is not in the pages' fused step; it is the "next" row
+ * that folds rotary and the packed-QKV split into the KV write.
+ *
+ *   q            device bf16 [T, Hq, D]; or, with k == v == NULL, the packed input
+ *                [T, (Hq + 2 Hkv) * D] (columns [0, Hq D) = Q, then K, then V).
+ *   k, v         device bf16 [T, Hkv, D], or both NULL (packed input).
+ *   rotary       host struct, read during the call; NULL = no rotation (a copy / split).
+ *   q_out        device bf16 [T, Hq, D]; must not overlap q.
+ *   k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k   as for rpa_write_kv.
+ * Pointers 16-byte aligned.  T == 0 returns RPA_OK and launches nothing.  Positions at or
+ * past max_position, and page ids outside [0, num_pages), are reported in the device error
+ * word (rpa_device_error) and nothing is written for the affected rows.
+ */
+RPA_API rpa_status rpa_rotary_write_kv(rpa_plan_t plan, const void* q, const void* k,
+                               const void* v, const rpa_rotary* rotary, void* q_out,
+                               void* k_pool, void* v_pool, const int32_t* block_table,
+                               const int32_t* cu_seqlens_q, const int32_t* seq_lens_k,
+                               void* stream);
+
+/*
  * rpa_forward -- the fused step: write the new tokens' K/V (when k_new/v_new are given)
  * and compute, for every query token t and query head hq,
  *     out[t, hq] = sum_j softmax_j(scale * q[t,hq] . K_j) V_j
@@ -235,7 +282,10 @@ RPA_API rpa_status rpa_build_group_tables(const uint8_t* mask, int32_t num_seqs,
 /*
  * rpa_device_error -- read (and optionally clear) the library's device error word on the
  * current device.  Kernels never spin without bound: a wait that runs out records a code
- * here and the kernel returns early.  Synchronizes the device.  *code = 0 means no error.
+ * here and the kernel returns early.  Synchronizes the device.  *code = 0 means no error;
+ * otherwise an OR of: 1 decode wait ran out, 2 prefill wait ran out, 4 a page id outside
+ * [0, num_pages) or a block index outside the table, 8 a position at or past the rotary
+ * caches' max_position.
  */
 RPA_API rpa_status rpa_device_error(int32_t* code, int32_t clear);
 

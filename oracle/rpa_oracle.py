@@ -25,6 +25,12 @@ What it computes (plain definitions, written out; no tiling, no fusion, no reord
   WebGPU page, "What's shipped").
 * ``build_group_tables`` -- Q-block union, then intra-group union, then the ascending list
   of selected KV blocks per (sequence, KV group) (CompactAttention, Core claim; Fig. 3).
+* ``rotate`` / ``rotary_write_kv`` -- the input pass with rotary position embedding: Q and
+  K rows rotated by their position ``past_b + s``, dims at or past ``rotary_dim`` unchanged,
+  pairs interleaved ``(2j, 2j+1)`` or split ``(j, j + rotary_dim/2)``; a packed input holds
+  per token the columns ``[Q | K | V]`` (same page, commits "Phase 1b.2" and the packed-QKV
+  commit).  Each rotated value is the exact ``x1 c - x2 s`` / ``x1 s + x2 c`` rounded once to
+  bf16 (nearest, ties to even).
 
 Inputs are bf16 bit patterns (numpy ``uint16``) or torch bf16 tensors; every bf16 value is
 widened exactly to fp64 before any arithmetic.  Cache writes move the bf16 bit patterns
@@ -298,3 +304,94 @@ def build_group_tables(mask, num_kv_heads: int):
             table[b, g, :len(sel)] = sel
             count[b, g] = len(sel)
     return table, count
+
+
+# --------------------------------------------------------------------------------------
+# Rotary position embedding and the packed-QKV split (the input pass)
+# --------------------------------------------------------------------------------------
+
+def round_bf16(x) -> np.ndarray:
+    """fp64 -> bf16 bit patterns, rounded once to nearest with ties to even (the plain
+    definition: 8 significant bits; below 2^-126 the spacing is fixed at 2^-133)."""
+    x = np.asarray(x, dtype=np.float64)
+    out = np.empty(x.shape, dtype=np.uint16)
+    flat = x.reshape(-1)
+    res = out.reshape(-1)
+    for i, v in enumerate(flat):
+        if v != v:
+            res[i] = 0x7FC0
+            continue
+        if v == 0.0 or math.isinf(v):
+            res[i] = np.array([v], dtype=np.float32).view(np.uint32)[0] >> 16
+            continue
+        m, e = math.frexp(v)              # v = m * 2^e, 0.5 <= |m| < 1
+        if e - 1 >= -126:                 # normal range: 8 significant bits
+            r = math.ldexp(float(np.rint(math.ldexp(m, 8))), e - 8)
+        else:                             # subnormal: multiples of 2^-133
+            r = math.ldexp(float(np.rint(math.ldexp(v, 133))), -133)
+        if abs(r) >= 2.0 ** 128:
+            r = math.copysign(math.inf, r)
+        res[i] = np.array([r], dtype=np.float32).view(np.uint32)[0] >> 16
+    return out
+
+
+def rotate(x: np.ndarray, pos, cos: np.ndarray, sin: np.ndarray, rotary_dim: int,
+           interleaved: bool) -> np.ndarray:
+    """Rotate the last axis of ``x`` (fp64 ``[..., D]``) by the angles of positions ``pos``
+    (integers broadcast to ``x.shape[:-1]``); ``cos``/``sin`` are fp64 ``[max_pos, rd/2]``."""
+    out = np.array(x, dtype=np.float64, copy=True)
+    half = rotary_dim // 2
+    c = cos[pos]
+    s = sin[pos]
+    if interleaved:
+        x1 = out[..., 0:rotary_dim:2].copy()
+        x2 = out[..., 1:rotary_dim:2].copy()
+        out[..., 0:rotary_dim:2] = x1 * c - x2 * s
+        out[..., 1:rotary_dim:2] = x1 * s + x2 * c
+    else:
+        x1 = out[..., :half].copy()
+        x2 = out[..., half:rotary_dim].copy()
+        out[..., :half] = x1 * c - x2 * s
+        out[..., half:rotary_dim] = x1 * s + x2 * c
+    return out
+
+
+def split_packed(qkv, num_q_heads: int, num_kv_heads: int, head_dim: int):
+    """Packed ``[T, (Hq + 2 Hkv) * D]`` bf16 bits -> Q ``[T, Hq, D]``, K, V ``[T, Hkv, D]``."""
+    a = bits16(qkv)
+    T = a.shape[0]
+    a = a.reshape(T, -1)
+    qd = num_q_heads * head_dim
+    kd = num_kv_heads * head_dim
+    return (a[:, :qd].reshape(T, num_q_heads, head_dim),
+            a[:, qd:qd + kd].reshape(T, num_kv_heads, head_dim),
+            a[:, qd + kd:qd + 2 * kd].reshape(T, num_kv_heads, head_dim))
+
+
+def token_positions(cu_seqlens_q, seq_lens_k) -> np.ndarray:
+    """Absolute position of every new token: ``past_b + i``."""
+    cu = ints(cu_seqlens_q)
+    out = np.zeros(int(cu[-1]), dtype=np.int64)
+    for t0, q_len, kv_len, past in seq_ranges(cu_seqlens_q, seq_lens_k):
+        out[t0:t0 + q_len] = past + np.arange(q_len)
+    return out
+
+
+def rotary_write_kv(q, k, v, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k,
+                    page_size: int, layout: int = SEQ_MAJOR, *, num_q_heads: int,
+                    num_kv_heads: int, head_dim: int, cos=None, sin=None,
+                    rotary_dim: int = 0, interleaved: bool = False):
+    """The input pass: returns (q_out bits [T, Hq, D], k_pool bits, v_pool bits)."""
+    if k is None:
+        qb, kb, vb = split_packed(q, num_q_heads, num_kv_heads, head_dim)
+    else:
+        qb, kb, vb = bits16(q), bits16(k), bits16(v)
+    if cos is not None:
+        pos = token_positions(cu_seqlens_q, seq_lens_k)
+        c = widen(bits16(cos))
+        s_ = widen(bits16(sin))
+        qb = round_bf16(rotate(widen(qb), pos[:, None], c, s_, rotary_dim, interleaved))
+        kb = round_bf16(rotate(widen(kb), pos[:, None], c, s_, rotary_dim, interleaved))
+    kp, vp = write_kv(k_pool, v_pool, kb, vb, block_table, cu_seqlens_q, seq_lens_k,
+                      page_size, layout)
+    return np.ascontiguousarray(qb), kp, vp

@@ -56,6 +56,12 @@ class RPAError(RuntimeError):
         self.status = status
 
 
+class Rotary(ctypes.Structure):
+    _fields_ = [("cos_cache", ctypes.c_void_p), ("sin_cache", ctypes.c_void_p),
+                ("max_position", ctypes.c_int32), ("rotary_dim", ctypes.c_int32),
+                ("interleaved", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
 _lib = None
 
 _P = ctypes.c_void_p
@@ -85,6 +91,9 @@ def lib() -> ctypes.CDLL:
         L.rpa_forward_no_alloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                            ctypes.c_float, _P, _P, _P]
         L.rpa_forward_no_alloc.restype = ctypes.c_int
+        L.rpa_rotary_write_kv.argtypes = [_P, _P, _P, _P, ctypes.POINTER(Rotary), _P, _P, _P,
+                                          _P, _P, _P, _P]
+        L.rpa_rotary_write_kv.restype = ctypes.c_int
         L.rpa_build_group_tables.argtypes = [_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                              ctypes.c_int32, ctypes.c_int32, _P, _P, _P]
         L.rpa_build_group_tables.restype = ctypes.c_int
@@ -227,6 +236,21 @@ def rpa_forward_no_alloc(plan: Plan, q, k_new, v_new, k_pool, v_pool, block_tabl
         plan.handle, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool),
         _ptr(block_table), _ptr(cu_seqlens_q), _ptr(seq_lens_k), _ptr(group_table),
         _ptr(group_count), ctypes.c_float(scale), _ptr(out), _ptr(lse), _stream(stream)))
+
+
+def rpa_rotary_write_kv(plan: Plan, q, k, v, q_out, k_pool, v_pool, block_table, cu_seqlens_q,
+                        seq_lens_k, cos_cache=None, sin_cache=None, rotary_dim: int = 0,
+                        interleaved: bool = False, stream=None):
+    """Rotate Q and K by position (when cos/sin caches are given), write Q to q_out and
+    scatter K, V into the pools.  k = v = None: q is the packed [T, (Hq + 2 Hkv) * D] input."""
+    rot = None
+    if cos_cache is not None:
+        rot = Rotary(cos_cache.data_ptr(), sin_cache.data_ptr(), int(cos_cache.shape[0]),
+                     int(rotary_dim or 2 * cos_cache.shape[1]), 1 if interleaved else 0, 0)
+    _check("rpa_rotary_write_kv", lib().rpa_rotary_write_kv(
+        plan.handle, _ptr(q), _ptr(k), _ptr(v), ctypes.byref(rot) if rot is not None else None,
+        _ptr(q_out), _ptr(k_pool), _ptr(v_pool), _ptr(block_table), _ptr(cu_seqlens_q),
+        _ptr(seq_lens_k), _stream(stream)))
 
 
 def rpa_build_group_tables(mask, num_kv_heads: int, table, count, stream=None):

@@ -417,6 +417,78 @@ rpa_status rpa_write_kv(rpa_plan_t plan, const void* k_new, const void* v_new, v
                        seq_lens_k, static_cast<cudaStream_t>(stream));
 }
 
+rpa_status rpa_rotary_write_kv(rpa_plan_t plan, const void* q, const void* k, const void* v,
+                               const rpa_rotary* rotary, void* q_out, void* k_pool,
+                               void* v_pool, const int32_t* block_table,
+                               const int32_t* cu_seqlens_q, const int32_t* seq_lens_k,
+                               void* stream) {
+  g_last_error.clear();
+  rpa_status st = check_common(plan, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k);
+  if (st != RPA_OK) return st;
+  const rpa_shape& s = plan->shape;
+  if (s.num_tokens == 0) return RPA_OK;
+  if (!q || !q_out) RPA_FAIL(RPA_ERR_INVALID_ARG, "q and q_out are required");
+  if ((k == nullptr) != (v == nullptr))
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "k and v must both be given or both be NULL (packed input)");
+  if (!aligned16(q) || !aligned16(q_out) || (k && (!aligned16(k) || !aligned16(v))))
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "q, k, v and q_out must be 16-byte aligned");
+  const size_t q_row = (size_t)(k ? s.num_q_heads : s.num_q_heads + 2 * s.num_kv_heads);
+  const size_t q_bytes = (size_t)s.num_tokens * q_row * s.head_dim * 2;
+  const size_t out_bytes = (size_t)s.num_tokens * s.num_q_heads * s.head_dim * 2;
+  const uintptr_t qa = reinterpret_cast<uintptr_t>(q), oa = reinterpret_cast<uintptr_t>(q_out);
+  if (qa < oa + out_bytes && oa < qa + q_bytes)
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "q_out must not overlap q");
+  RotaryLaunch r;
+  r.cos = r.sin = nullptr;
+  r.max_pos = 0;
+  r.rotary_dim = 0;
+  r.interleaved = 0;
+  if (rotary) {
+    const rpa_rotary& ro = *rotary;
+    if (ro.reserved != 0) RPA_FAIL(RPA_ERR_INVALID_ARG, "rotary.reserved != 0");
+    if (!ro.cos_cache || !ro.sin_cache)
+      RPA_FAIL(RPA_ERR_INVALID_ARG, "rotation needs cos_cache and sin_cache");
+    if (!aligned16(ro.cos_cache) || !aligned16(ro.sin_cache))
+      RPA_FAIL(RPA_ERR_INVALID_ARG, "cos_cache / sin_cache must be 16-byte aligned");
+    if (ro.rotary_dim < 16 || ro.rotary_dim % 16 != 0 || ro.rotary_dim > s.head_dim)
+      RPA_FAIL(RPA_ERR_UNSUPPORTED, "rotary_dim %d must be a multiple of 16 in [16, %d]",
+               ro.rotary_dim, s.head_dim);
+    if (ro.max_position <= 0)
+      RPA_FAIL(RPA_ERR_INVALID_ARG, "max_position %d must be positive", ro.max_position);
+    if (ro.interleaved != 0 && ro.interleaved != 1)
+      RPA_FAIL(RPA_ERR_INVALID_ARG, "interleaved must be 0 or 1");
+    r.cos = static_cast<const uint16_t*>(ro.cos_cache);
+    r.sin = static_cast<const uint16_t*>(ro.sin_cache);
+    r.max_pos = ro.max_position;
+    r.rotary_dim = ro.rotary_dim;
+    r.interleaved = ro.interleaved;
+  }
+  int* err = nullptr;
+  st = check_cuda(device_error_word(&err), "device error word");
+  if (st != RPA_OK) return st;
+  r.q = static_cast<const uint16_t*>(q);
+  r.k = static_cast<const uint16_t*>(k);
+  r.v = static_cast<const uint16_t*>(v);
+  r.q_out = static_cast<uint16_t*>(q_out);
+  r.k_pool = static_cast<uint16_t*>(k_pool);
+  r.v_pool = static_cast<uint16_t*>(v_pool);
+  r.block_table = block_table;
+  r.cu_seqlens_q = cu_seqlens_q;
+  r.seq_lens_k = seq_lens_k;
+  r.num_seqs = s.num_seqs;
+  r.num_tokens = s.num_tokens;
+  r.num_q_heads = s.num_q_heads;
+  r.num_kv_heads = s.num_kv_heads;
+  r.head_dim = s.head_dim;
+  r.page_size = s.page_size;
+  r.max_blocks = s.max_blocks_per_seq;
+  r.layout = s.layout;
+  r.num_pages = s.num_pages;
+  r.err = err;
+  return check_cuda(launch_rotary_write(r, static_cast<cudaStream_t>(stream)),
+                    "rotary write launch");
+}
+
 rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const void* v_new,
                        void* k_pool, void* v_pool, const int32_t* block_table,
                        const int32_t* cu_seqlens_q, const int32_t* seq_lens_k,

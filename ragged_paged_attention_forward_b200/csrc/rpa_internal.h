@@ -27,6 +27,7 @@ enum DeviceErrorCode : int {
   kErrDecodeWait = 1 << 0,
   kErrPrefillWait = 1 << 1,
   kErrBadIndex = 1 << 2,
+  kErrBadPosition = 1 << 3,
 };
 
 // One (sequence, key range) item of the split-KV decode kernel; one CTA per (item, KV head).
@@ -158,8 +159,36 @@ struct WriteLaunch {
   int* err;
 };
 
+struct RotaryLaunch {
+  const uint16_t* q;      // [T, Hq, D] or packed [T, (Hq + 2 Hkv) D]
+  const uint16_t* k;      // [T, Hkv, D] or null (packed)
+  const uint16_t* v;
+  const uint16_t* cos;    // [max_pos, rd/2] or null (no rotation)
+  const uint16_t* sin;
+  int32_t max_pos;
+  int32_t rotary_dim;
+  int32_t interleaved;
+  uint16_t* q_out;        // [T, Hq, D]
+  uint16_t* k_pool;
+  uint16_t* v_pool;
+  const int32_t* block_table;
+  const int32_t* cu_seqlens_q;
+  const int32_t* seq_lens_k;
+  int32_t num_seqs;
+  int32_t num_tokens;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t page_size;
+  int32_t max_blocks;
+  int32_t layout;
+  int32_t num_pages;
+  int* err;
+};
+
 // Launchers (return the cudaError_t of the launch).
 cudaError_t launch_write_kv(const WriteLaunch& p, cudaStream_t stream);
+cudaError_t launch_rotary_write(const RotaryLaunch& p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeLaunch& p, const DecodeItemsInline* inl, int nt,
                           cudaStream_t stream);
 cudaError_t launch_merge(const MergeLaunch& p, const MergeRowsInline* inl, cudaStream_t stream);

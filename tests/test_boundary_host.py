@@ -151,3 +151,48 @@ def test_group_table_builder_rejects():
 def test_status_strings():
     for code in range(-6, 1):
         assert api.status_string(code).startswith("RPA_")
+
+
+def _rotary_status(plan, rotary=None, **over):
+    fake = 1 << 20
+    args = dict(q=fake, k=3 << 20, v=5 << 20, q_out=7 << 24, k_pool=fake, v_pool=fake,
+                bt=fake, cu=fake, kv=fake)
+    args.update(over)
+    P = lambda v: None if v is None else ctypes.c_void_p(v)
+    rot = None
+    if rotary is not None:
+        r = dict(cos=9 << 20, sin=11 << 20, max_position=4096, rotary_dim=128, interleaved=0,
+                 reserved=0)
+        r.update(rotary)
+        rot = api.Rotary(P(r["cos"]), P(r["sin"]), r["max_position"], r["rotary_dim"],
+                         r["interleaved"], r["reserved"])
+    return api.lib().rpa_rotary_write_kv(
+        plan.handle, P(args["q"]), P(args["k"]), P(args["v"]),
+        ctypes.byref(rot) if rot is not None else None, P(args["q_out"]), P(args["k_pool"]),
+        P(args["v_pool"]), P(args["bt"]), P(args["cu"]), P(args["kv"]), None)
+
+
+@pytest.mark.parametrize("over,rotary,status", [
+    (dict(q=None), None, api.RPA_ERR_INVALID_ARG),
+    (dict(q_out=None), None, api.RPA_ERR_INVALID_ARG),
+    (dict(v=None), None, api.RPA_ERR_INVALID_ARG),                 # k without v
+    (dict(q_out=(1 << 20) + 256), None, api.RPA_ERR_INVALID_ARG),  # q_out overlaps q
+    (dict(q=(1 << 20) + 8), None, api.RPA_ERR_INVALID_ARG),        # misaligned
+    (dict(k_pool=None), None, api.RPA_ERR_INVALID_ARG),
+    ({}, dict(rotary_dim=24), api.RPA_ERR_UNSUPPORTED),
+    ({}, dict(rotary_dim=256), api.RPA_ERR_UNSUPPORTED),
+    ({}, dict(rotary_dim=0), api.RPA_ERR_UNSUPPORTED),
+    ({}, dict(cos=None), api.RPA_ERR_INVALID_ARG),
+    ({}, dict(sin=(11 << 20) + 4), api.RPA_ERR_INVALID_ARG),       # misaligned cache
+    ({}, dict(max_position=0), api.RPA_ERR_INVALID_ARG),
+    ({}, dict(interleaved=2), api.RPA_ERR_INVALID_ARG),
+    ({}, dict(reserved=1), api.RPA_ERR_INVALID_ARG),
+])
+def test_rotary_write_rejects_on_host(over, rotary, status):
+    p = api.rpa_plan(**_shape())
+    assert _rotary_status(p, rotary, **over) == status
+
+
+def test_rotary_write_zero_tokens_is_a_no_op():
+    p = api.rpa_plan(**_shape(num_seqs=2, num_tokens=0, cu_seqlens_q=[0, 0, 0]))
+    assert _rotary_status(p, dict()) == api.RPA_OK

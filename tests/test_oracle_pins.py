@@ -379,3 +379,111 @@ def test_tolerance_is_reachable_with_bf16_inputs_and_fp32_accumulation():
             err.append(np.abs(o.to(torch.bfloat16).double().numpy() - out[s, hq]))
     err = np.concatenate(err)
     assert err.max() < 2e-2 / 4 and err.mean() < 2e-3 / 4
+
+
+# ------------------------------------------------------------------------------------
+# Rotary position embedding, packed QKV, bf16 rounding (the input pass)
+# ------------------------------------------------------------------------------------
+
+def _bf16_bits_from_f32(v):
+    return torch.tensor(v, dtype=torch.float32).to(torch.bfloat16).view(torch.int16).numpy() \
+        .view(np.uint16)
+
+
+def test_round_bf16_matches_torch_on_fp32_values_and_ties():
+    # fp32-representable values round the same through torch's fp32 -> bf16 conversion
+    g = np.random.default_rng(3)
+    x = g.standard_normal(4000).astype(np.float32) * np.float32(10.0) ** g.integers(-30, 30, 4000)
+    assert np.array_equal(orc.round_bf16(x.astype(np.float64)), _bf16_bits_from_f32(x))
+    # exact ties go to the even significand: 1 + 2^-8 -> 1, 1 + 3*2^-8 -> 1 + 2^-6
+    assert orc.round_bf16(np.array([1 + 2 ** -8]))[0] == 0x3F80
+    assert orc.round_bf16(np.array([1 + 3 * 2 ** -8]))[0] == 0x3F82
+    # a value just above a tie rounds up although its fp32 rounding would be the tie itself
+    assert orc.round_bf16(np.array([1 + 2 ** -8 + 2 ** -40]))[0] == 0x3F81
+
+
+def _unit_angles(n, half, seed):
+    g = np.random.default_rng(seed)
+    theta = g.uniform(-math.pi, math.pi, (n, half))
+    return np.cos(theta), np.sin(theta), theta
+
+
+def test_rotate_split_is_complex_multiplication():
+    D, rd = 16, 12
+    cos, sin, theta = _unit_angles(5, rd // 2, 1)
+    x = np.random.default_rng(2).standard_normal((7, D))
+    pos = np.array([0, 4, 2, 2, 3, 1, 0])
+    out = orc.rotate(x, pos, cos, sin, rd, interleaved=False)
+    z = (x[:, :rd // 2] + 1j * x[:, rd // 2:rd]) * np.exp(1j * theta[pos])
+    assert np.allclose(out[:, :rd // 2], z.real, rtol=0, atol=1e-12)
+    assert np.allclose(out[:, rd // 2:rd], z.imag, rtol=0, atol=1e-12)
+    assert np.array_equal(out[:, rd:], x[:, rd:])  # dims past rotary_dim unchanged
+
+
+def test_rotate_interleaved_is_split_on_permuted_dims():
+    D, rd = 16, 16
+    cos, sin, _ = _unit_angles(3, rd // 2, 4)
+    x = np.random.default_rng(5).standard_normal((6, D))
+    pos = np.array([0, 1, 2, 0, 1, 2])
+    # interleaved pair j = (2j, 2j+1); split pair j = (j, j + rd/2)
+    perm = np.concatenate([np.arange(0, rd, 2), np.arange(1, rd, 2)])
+    a = orc.rotate(x, pos, cos, sin, rd, interleaved=True)
+    b = orc.rotate(x[:, perm], pos, cos, sin, rd, interleaved=False)
+    assert np.allclose(a[:, perm], b, rtol=0, atol=1e-12)
+
+
+def test_rotate_invariants():
+    D, rd = 8, 8
+    # a Pythagorean angle: cos = 3/5, sin = 4/5 exactly; zero angle is the identity
+    cos = np.array([[1.0] * 4, [0.6] * 4])
+    sin = np.array([[0.0] * 4, [0.8] * 4])
+    x = np.random.default_rng(6).standard_normal((2, D))
+    pos = np.array([0, 1])
+    for inter in (False, True):
+        out = orc.rotate(x, pos, cos, sin, rd, interleaved=inter)
+        assert np.array_equal(out[0], x[0])
+        pairs_in = (x[1, 0::2], x[1, 1::2]) if inter else (x[1, :4], x[1, 4:])
+        pairs_out = (out[1, 0::2], out[1, 1::2]) if inter else (out[1, :4], out[1, 4:])
+        assert np.allclose(pairs_in[0] ** 2 + pairs_in[1] ** 2,
+                           pairs_out[0] ** 2 + pairs_out[1] ** 2, rtol=1e-14, atol=0)
+        back = orc.rotate(out, pos, cos, -sin, rd, interleaved=inter)
+        assert np.allclose(back, x, rtol=0, atol=1e-14)
+
+
+def test_rotary_write_uses_past_plus_index_and_packed_columns():
+    # two sequences with different pasts; each position p rotates by the angle p * 0.1
+    Hq, Hkv, D, P = 2, 1, 16, 16
+    b = wl.ragged_batch([20, 9], [3, 9], Hq, Hkv, D, P, seed=64, poison=False)
+    maxp = 32
+    ang = 0.1 * np.arange(maxp)[:, None] * np.ones((1, D // 2))
+    cos_b = _bf16_bits_from_f32(np.cos(ang).astype(np.float32))
+    sin_b = _bf16_bits_from_f32(np.sin(ang).astype(np.float32))
+    packed = torch.cat([b.q.reshape(b.num_tokens, -1), b.k_new.reshape(b.num_tokens, -1),
+                        b.v_new.reshape(b.num_tokens, -1)], dim=1).contiguous()
+    qo, kp, vp = orc.rotary_write_kv(packed, None, None, b.k_pool, b.v_pool, b.block_table,
+                                     b.cu_seqlens_q, b.seq_lens_k, P, b.layout,
+                                     num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D,
+                                     cos=cos_b, sin=sin_b, rotary_dim=D, interleaved=False)
+    qo2, kp2, vp2 = orc.rotary_write_kv(b.q, b.k_new, b.v_new, b.k_pool, b.v_pool,
+                                        b.block_table, b.cu_seqlens_q, b.seq_lens_k, P,
+                                        b.layout, num_q_heads=Hq, num_kv_heads=Hkv,
+                                        head_dim=D, cos=cos_b, sin=sin_b, rotary_dim=D)
+    assert np.array_equal(qo, qo2) and np.array_equal(kp, kp2) and np.array_equal(vp, vp2)
+    # token 1 of sequence 0 sits at position 17 + 1 = 18, token 0 of sequence 1 at 0
+    cw, sw = orc.widen(cos_b), orc.widen(sin_b)
+    for t, p in ((1, 18), (3, 0), (11, 8)):
+        x = orc.widen(orc.bits16(b.q[t, 0]))
+        z = (x[:D // 2] + 1j * x[D // 2:]) * (cw[p] + 1j * sw[p])
+        want = orc.round_bf16(np.concatenate([z.real, z.imag]))
+        assert np.array_equal(qo[t, 0], want)
+    # V is scattered unchanged (the plain KV write of the same tokens)
+    _, vref = orc.write_kv(b.k_pool, b.v_pool, b.k_new, b.v_new, b.block_table,
+                           b.cu_seqlens_q, b.seq_lens_k, P, b.layout)
+    assert np.array_equal(vp, vref)
+    # without caches the pass is the plain split + scatter
+    q3, kp3, _ = orc.rotary_write_kv(packed, None, None, b.k_pool, b.v_pool, b.block_table,
+                                     b.cu_seqlens_q, b.seq_lens_k, P, b.layout,
+                                     num_q_heads=Hq, num_kv_heads=Hkv, head_dim=D)
+    kref, _ = orc.write_kv(b.k_pool, b.v_pool, b.k_new, b.v_new, b.block_table,
+                           b.cu_seqlens_q, b.seq_lens_k, P, b.layout)
+    assert np.array_equal(q3, orc.bits16(b.q)) and np.array_equal(kp3, kref)
