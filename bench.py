@@ -503,6 +503,47 @@ def measure(name, runner, steps, warmup, peaks):
     return res
 
 
+def measure_input_pass(steps, warmup, peaks):
+    """The input pass with rotary embedding (rpa_rotary_write_kv) on the prefill workload's
+    16384 new tokens: packed QKV in, RoPE over all 128 dims (split pairs), Q out, K/V
+    scattered into the pool.  HBM-bound: algorithmic bytes = the packed input read + Q, K, V
+    written + one cos/sin row pair per token.  Timed back to back over rotating copies of
+    the input and the pool (together larger than L2)."""
+    import numpy as np
+    from ragged_paged_attention_forward_b200 import api
+    b, _ = make_workload("prefill")
+    T, Hq, D = b.q.shape
+    Hkv = b.num_kv_heads
+    rd = D
+    runner = Runner("prefill", b, None)
+    d = runner.d
+    packed = torch.cat([d["q"].reshape(T, -1), d["k_new"].reshape(T, -1),
+                        d["v_new"].reshape(T, -1)], dim=1).contiguous()
+    copies = max(3, -(-2 * L2_BYTES // (2 * packed.numel() * 2)) + 1)
+    ins = [packed] + [packed.clone() for _ in range(copies - 1)]
+    q_outs = [torch.empty_like(d["q"]) for _ in range(copies)]
+    max_pos = int(b.seq_lens_k.max()) + 1
+    j = np.arange(rd // 2)
+    ang = np.arange(max_pos)[:, None] / 10000.0 ** (2.0 * j / rd)[None, :]
+    cos = torch.tensor(np.cos(ang), dtype=torch.float32).to(torch.bfloat16).cuda()
+    sin = torch.tensor(np.sin(ang), dtype=torch.float32).to(torch.bfloat16).cuda()
+
+    def call(i):
+        k = i % copies
+        kp, vp = runner.pools[i % len(runner.pools)]
+        api.rpa_rotary_write_kv(runner.plan, ins[k], None, None, q_outs[k], kp, vp,
+                                d["block_table"], d["cu_seqlens_q"], d["seq_lens_k"],
+                                cos, sin, rd, False)
+
+    ms = timed_loop(call, steps, warmup)
+    nbytes = 2.0 * T * (Hq + 2 * Hkv) * D * 2 + T * rd * 2
+    gbps = nbytes / (ms * 1e-3) / 1e9
+    return {"workload": "input pass: 16384 tokens of packed QKV (Hq=32, Hkv=8, D=128), RoPE "
+                        "over 128 dims, Q written, K/V scattered into pages of 64",
+            "ms": ms, "algorithmic_bytes": nbytes, "GBps": gbps,
+            "frac_of_hbm": gbps / peaks["hbm_gbs"], "launches": 1}
+
+
 def cpu_oracle_baseline(name, batch, target_s=12.0, table=None, count=None):
     """Time the fp64 oracle, as it stands, on a bounded sample of the workload: whole
     sequences (all query heads) until about target_s of CPU work."""
@@ -702,6 +743,7 @@ def run_gpu(args):
             secondary[other] = res
             del r2, b2
             torch.cuda.empty_cache()
+        secondary["input_pass"] = measure_input_pass(args.steps, args.warmup, peaks)
         line["secondary"] = secondary
         if "prefill" in secondary:
             line["prefill_TFLOPs"] = secondary["prefill"]["attn_TFLOPs"]
