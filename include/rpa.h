@@ -126,6 +126,32 @@ RPA_API rpa_status rpa_plan(const rpa_shape* shape, const int32_t* cu_seqlens_q,
                     const int32_t* seq_lens_k, const rpa_plan_options* opts,
                     rpa_plan_t* out_plan, size_t* workspace_bytes);
 
+/*
+ * rpa_plan_device -- a plan whose work lists are built on the device at every rpa_forward
+ * call, from the device cu_seqlens_q / seq_lens_k of that call, so that a step takes no
+ * host arrays, needs no host synchronisation and can be captured in a CUDA graph and
+ * replayed with new lengths (the same pointers).  No counterpart in the pages; the
+ * "graph-capturable, device-side planner" that follows the host planner above.
+ *
+ *   shape         num_seqs = B, the length of the lengths arrays (sequences may have
+ *                 q_len 0); num_tokens = the largest T any step will have; the other fields
+ *                 as for rpa_plan.
+ *   max_kv_len    the largest seq_lens_k any step will have (<= max_blocks_per_seq * P).
+ *   opts          optional; decode_split_keys as for rpa_plan; sparse and force_class are
+ *                 not supported (RPA_ERR_UNSUPPORTED).
+ *   workspace_bytes  receives the workspace size for these limits.
+ * Each call of rpa_forward with this plan launches a one-CTA planner kernel (a sequence
+ * goes to the split-KV decode kernel when q_len * G <= 16, else to the tensor-core kernel),
+ * then every kernel with its largest grid; CTAs past the step's counts return at once.
+ * A step beyond the limits (T, kv_len, q_len > kv_len) computes nothing and sets bit 16
+ * of the device error word.  rpa_write_kv with this plan writes the step's tokens only.
+ * The q, k_new, v_new, out and lse buffers given to rpa_forward hold num_tokens rows (the
+ * bound): only the step's rows are read and written.
+ */
+RPA_API rpa_status rpa_plan_device(const rpa_shape* shape, int32_t max_kv_len,
+                           const rpa_plan_options* opts, rpa_plan_t* out_plan,
+                           size_t* workspace_bytes);
+
 /* rpa_plan_get_info -- what the planner chose (host only, no device work). */
 RPA_API rpa_status rpa_plan_get_info(rpa_plan_t plan, rpa_plan_info* info);
 
@@ -285,7 +311,7 @@ RPA_API rpa_status rpa_build_group_tables(const uint8_t* mask, int32_t num_seqs,
  * here and the kernel returns early.  Synchronizes the device.  *code = 0 means no error;
  * otherwise an OR of: 1 decode wait ran out, 2 prefill wait ran out, 4 a page id outside
  * [0, num_pages) or a block index outside the table, 8 a position at or past the rotary
- * caches' max_position.
+ * caches' max_position, 16 a device-planned step beyond its plan's limits.
  */
 RPA_API rpa_status rpa_device_error(int32_t* code, int32_t clear);
 

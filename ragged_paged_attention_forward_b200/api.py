@@ -79,6 +79,10 @@ def lib() -> ctypes.CDLL:
         L.rpa_plan.argtypes = [ctypes.POINTER(Shape), _I32P, _I32P, ctypes.POINTER(PlanOptions),
                                ctypes.POINTER(_P), ctypes.POINTER(ctypes.c_size_t)]
         L.rpa_plan.restype = ctypes.c_int
+        L.rpa_plan_device.argtypes = [ctypes.POINTER(Shape), ctypes.c_int32,
+                                      ctypes.POINTER(PlanOptions), ctypes.POINTER(_P),
+                                      ctypes.POINTER(ctypes.c_size_t)]
+        L.rpa_plan_device.restype = ctypes.c_int
         L.rpa_plan_get_info.argtypes = [_P, ctypes.POINTER(PlanInfo)]
         L.rpa_plan_get_info.restype = ctypes.c_int
         L.rpa_plan_destroy.argtypes = [_P]
@@ -201,6 +205,24 @@ def rpa_plan(*, num_seqs: int, num_tokens: int, num_q_heads: int, num_kv_heads: 
     _check("rpa_plan", lib().rpa_plan(ctypes.byref(shape), _host_i32(cu_seqlens_q),
                                       _host_i32(seq_lens_k), ctypes.byref(opts),
                                       ctypes.byref(handle), ctypes.byref(ws)))
+    return Plan(handle, ws.value)
+
+
+def rpa_plan_device(*, num_seqs: int, max_tokens: int, num_q_heads: int, num_kv_heads: int,
+                    head_dim: int, page_size: int, num_pages: int, max_blocks_per_seq: int,
+                    layout: int, causal: bool, max_kv_len: int,
+                    decode_split_keys: int = 0) -> Plan:
+    """A plan whose work lists are built on the device at every call (CUDA-graph friendly):
+    B = num_seqs sequences, at most max_tokens new tokens and max_kv_len keys per step.  The
+    q / k_new / v_new / out / lse buffers of the calls hold max_tokens rows."""
+    shape = Shape(num_seqs, max_tokens, num_q_heads, num_kv_heads, head_dim, page_size,
+                  num_pages, max_blocks_per_seq, layout, 1 if causal else 0)
+    opts = PlanOptions(0, decode_split_keys, 0)
+    handle = ctypes.c_void_p()
+    ws = ctypes.c_size_t(0)
+    _check("rpa_plan_device", lib().rpa_plan_device(ctypes.byref(shape), int(max_kv_len),
+                                                    ctypes.byref(opts), ctypes.byref(handle),
+                                                    ctypes.byref(ws)))
     return Plan(handle, ws.value)
 
 

@@ -78,6 +78,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  if (p.count && (int)blockIdx.x >= __ldg(p.count)) return;  // device-planned: unused CTA
   const DecodeItem it = p.items ? p.items[blockIdx.x] : inl.v[blockIdx.x];
   const int h = blockIdx.y;
   const int Hq = p.num_q_heads;
@@ -391,7 +392,8 @@ __global__ void __launch_bounds__(128) merge_kernel(MergeLaunch p,
   const int gw = blockIdx.x * 4 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   const int Hq = p.num_q_heads;
-  if (gw >= p.num_rows * Hq) return;
+  const int nrows = p.count ? __ldg(p.count) : p.num_rows;
+  if (gw >= nrows * Hq) return;
   const int r = gw / Hq;
   const int hq = gw - r * Hq;
   const int G = Hq / p.num_kv_heads;

@@ -130,6 +130,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int hpc = (G & 1) == 0 ? 2 : 1;            // query heads per CTA
   const int groups = Hq / hpc;
   const int tile_idx = blockIdx.x / groups;
+  if (p.count && tile_idx >= __ldg(p.count)) return;  // device-planned step: unused CTA
   const int hq0 = (blockIdx.x - tile_idx * groups) * hpc;
   const PrefillTile tile = p.tiles ? p.tiles[tile_idx] : inl.v[tile_idx];
   const int h = hq0 / G;                            // KV head (shared by the pair)

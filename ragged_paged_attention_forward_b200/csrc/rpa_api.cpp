@@ -72,6 +72,11 @@ struct rpa_plan_s {
   PrefillTilesInline pf_inline;
   // pure decode plans fold the KV write into the decode kernel
   bool fuse_write = false;
+  // device-planned plans: the lists are built on the device at every call, up to these caps
+  bool device_mode = false;
+  int max_kv_len = 0;
+  int cap_items = 0, cap_rows = 0, cap_tiles = 0;
+  size_t off_counts = 0;
   int launches_forward = 0;
   int launches_write = 0;
   // fork/join events of a mixed batch (created on first use, on the device of that call)
@@ -345,6 +350,69 @@ rpa_status rpa_plan(const rpa_shape* shape, const int32_t* cu_seqlens_q,
   return RPA_OK;
 }
 
+rpa_status rpa_plan_device(const rpa_shape* shape, int32_t max_kv_len,
+                           const rpa_plan_options* opts, rpa_plan_t* out_plan,
+                           size_t* workspace_bytes) {
+  g_last_error.clear();
+  if (!shape || !out_plan) RPA_FAIL(RPA_ERR_INVALID_ARG, "shape and out_plan must not be NULL");
+  *out_plan = nullptr;
+  rpa_status st = validate_shape(*shape);
+  if (st != RPA_OK) return st;
+  const rpa_shape& s = *shape;
+  rpa_plan_options o;
+  memset(&o, 0, sizeof(o));
+  if (opts) o = *opts;
+  for (int i = 0; i < 5; ++i)
+    if (o.reserved[i] != 0) RPA_FAIL(RPA_ERR_INVALID_ARG, "plan option reserved[%d] != 0", i);
+  if (o.sparse) RPA_FAIL(RPA_ERR_UNSUPPORTED, "device-planned steps take no group tables");
+  if (o.force_class != RPA_CLASS_AUTO)
+    RPA_FAIL(RPA_ERR_UNSUPPORTED, "device-planned steps choose their kernels per sequence");
+  if (o.decode_split_keys != 0 &&
+      (o.decode_split_keys % kDecodeStageKeys != 0 || o.decode_split_keys < kDecodeStageKeys ||
+       o.decode_split_keys > kMaxSplitKeys))
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "decode_split_keys %d must be a multiple of %d in [%d, %d]",
+             o.decode_split_keys, kDecodeStageKeys, kDecodeStageKeys, kMaxSplitKeys);
+  if (max_kv_len < 1 || (long)max_kv_len > (long)s.max_blocks_per_seq * s.page_size)
+    RPA_FAIL(RPA_ERR_SHAPE, "max_kv_len %d must be in [1, max_blocks_per_seq * page_size]",
+             max_kv_len);
+  rpa_plan_s* plan = new (std::nothrow) rpa_plan_s();
+  if (!plan) RPA_FAIL(RPA_ERR_INVALID_ARG, "out of host memory");
+  plan->shape = s;
+  plan->opts = o;
+  plan->device_mode = true;
+  plan->max_kv_len = max_kv_len;
+  plan->batch_class = RPA_CLASS_AUTO;
+  // every sequence whose query heads x tokens fit 16 MMA columns goes to the decode kernel
+  plan->decode_nt = 2;
+  plan->split_keys = o.decode_split_keys ? o.decode_split_keys : 512;
+  const int B = s.num_seqs;
+  const long splits = (max_kv_len + plan->split_keys - 1) / plan->split_keys;
+  plan->cap_items = (int)std::min<long>((long)B * splits, 1L << 24);
+  plan->cap_rows = std::max(s.num_tokens, 1);
+  plan->cap_tiles = (s.num_tokens + kPrefillTileRows - 1) / kPrefillTileRows + B;
+  size_t off = 0;
+  plan->off_counts = off;
+  off = align_up(off + 16, 256);
+  plan->off_dec = off;
+  off = align_up(off + (size_t)plan->cap_items * sizeof(DecodeItem), 256);
+  plan->off_merge = off;
+  off = align_up(off + (size_t)plan->cap_rows * sizeof(MergeRow), 256);
+  plan->off_pf = off;
+  off = align_up(off + (size_t)plan->cap_tiles * sizeof(PrefillTile), 256);
+  const size_t rows_per_item = 8 * plan->decode_nt;
+  plan->off_part_o = off;
+  off = align_up(off + (size_t)plan->cap_items * s.num_kv_heads * rows_per_item * s.head_dim * 4,
+                 256);
+  plan->off_part_lse = off;
+  off = align_up(off + (size_t)plan->cap_items * s.num_kv_heads * rows_per_item * 4, 256);
+  plan->ws_bytes = off;
+  plan->launches_write = 1;
+  plan->launches_forward = 5;  // planner, KV write, tensor-core, decode, merge
+  *out_plan = plan;
+  if (workspace_bytes) *workspace_bytes = plan->ws_bytes;
+  return RPA_OK;
+}
+
 rpa_status rpa_plan_get_info(rpa_plan_t plan, rpa_plan_info* info) {
   if (!plan || !info) RPA_FAIL(RPA_ERR_INVALID_ARG, "plan and info must not be NULL");
   memset(info, 0, sizeof(*info));
@@ -356,6 +424,11 @@ rpa_status rpa_plan_get_info(rpa_plan_t plan, rpa_plan_info* info) {
   info->launches_write = plan->launches_write;
   info->decode_split_keys = plan->split_keys;
   info->workspace_bytes = plan->ws_bytes;
+  if (plan->device_mode) {  // the caps the device-built lists may reach
+    info->num_decode_items = plan->cap_items;
+    info->num_prefill_tiles = plan->cap_tiles;
+    info->num_merge_rows = plan->cap_rows;
+  }
   return RPA_OK;
 }
 
@@ -369,7 +442,7 @@ static rpa_status write_kv_impl(rpa_plan_t plan, const void* k_new, const void* 
   int* err = nullptr;
   rpa_status st = check_cuda(device_error_word(&err), "device error word");
   if (st != RPA_OK) return st;
-  WriteLaunch w;
+  WriteLaunch w{};
   w.k_new = static_cast<const uint16_t*>(k_new);
   w.v_new = static_cast<const uint16_t*>(v_new);
   w.k_pool = static_cast<uint16_t*>(k_pool);
@@ -385,6 +458,7 @@ static rpa_status write_kv_impl(rpa_plan_t plan, const void* k_new, const void* 
   w.max_blocks = s.max_blocks_per_seq;
   w.layout = s.layout;
   w.num_pages = s.num_pages;
+  w.tokens_on_device = plan->device_mode ? 1 : 0;
   w.err = err;
   return check_cuda(launch_write_kv(w, stream), "write_kv launch");
 }
@@ -438,7 +512,7 @@ rpa_status rpa_rotary_write_kv(rpa_plan_t plan, const void* q, const void* k, co
   const uintptr_t qa = reinterpret_cast<uintptr_t>(q), oa = reinterpret_cast<uintptr_t>(q_out);
   if (qa < oa + out_bytes && oa < qa + q_bytes)
     RPA_FAIL(RPA_ERR_INVALID_ARG, "q_out must not overlap q");
-  RotaryLaunch r;
+  RotaryLaunch r{};
   r.cos = r.sin = nullptr;
   r.max_pos = 0;
   r.rotary_dim = 0;
@@ -550,6 +624,104 @@ rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const 
   kv.num_pages = s.num_pages;
   const float scale_log2 = scale * 1.4426950408889634f;
 
+  if (plan->device_mode) {
+    // the lists are built from the device lengths first; every kernel then runs its
+    // largest grid, and CTAs past the step's counts return at once
+    int32_t* counts = reinterpret_cast<int32_t*>(ws + plan->off_counts);
+    PlanDeviceLaunch pl{};
+    pl.cu_seqlens_q = cu_seqlens_q;
+    pl.seq_lens_k = seq_lens_k;
+    pl.num_seqs = s.num_seqs;
+    pl.max_tokens = s.num_tokens;
+    pl.max_kv_len = plan->max_kv_len;
+    pl.num_q_heads = s.num_q_heads;
+    pl.num_kv_heads = s.num_kv_heads;
+    pl.causal = s.causal;
+    pl.split_keys = plan->split_keys;
+    pl.decode_rows = 8 * plan->decode_nt;
+    pl.cap_items = plan->cap_items;
+    pl.cap_rows = plan->cap_rows;
+    pl.cap_tiles = plan->cap_tiles;
+    pl.items = reinterpret_cast<DecodeItem*>(ws + plan->off_dec);
+    pl.rows = reinterpret_cast<MergeRow*>(ws + plan->off_merge);
+    pl.tiles = reinterpret_cast<PrefillTile*>(ws + plan->off_pf);
+    pl.counts = counts;
+    pl.err = err;
+    st = check_cuda(launch_plan_device(pl, stream), "device planner launch");
+    if (st != RPA_OK) return st;
+    // both kernel families: the tensor-core kernel on the side stream, forked after the
+    // planner, the decode kernel and the merge on the caller's stream; joined at the end
+    cudaStream_t pf_stream = stream;
+    st = check_cuda(side_stream(&pf_stream), "side stream");
+    if (st != RPA_OK) return st;
+    if (!plan->fork_ev) {
+      st = check_cuda(cudaEventCreateWithFlags(&plan->fork_ev, cudaEventDisableTiming),
+                      "event create");
+      if (st != RPA_OK) return st;
+      st = check_cuda(cudaEventCreateWithFlags(&plan->join_ev, cudaEventDisableTiming),
+                      "event create");
+      if (st != RPA_OK) return st;
+    }
+    st = check_cuda(cudaEventRecord(plan->fork_ev, stream), "fork record");
+    if (st != RPA_OK) return st;
+    st = check_cuda(cudaStreamWaitEvent(pf_stream, plan->fork_ev, 0), "fork wait");
+    if (st != RPA_OK) return st;
+    PrefillLaunch p{};
+    p.tiles = pl.tiles;
+    p.num_tiles = plan->cap_tiles;
+    p.count = counts + 2;
+    p.q = static_cast<const uint16_t*>(q);
+    p.num_tokens = s.num_tokens;
+    p.num_q_heads = s.num_q_heads;
+    p.num_kv_heads = s.num_kv_heads;
+    p.head_dim = s.head_dim;
+    p.causal = s.causal;
+    p.scale_log2 = scale_log2;
+    p.out = static_cast<uint16_t*>(out);
+    p.lse = lse;
+    p.err = err;
+    p.kv = kv;
+    st = check_cuda(launch_prefill(p, &plan->pf_inline, pf_stream), "prefill launch");
+    if (st != RPA_OK) return st;
+    DecodeLaunch d{};
+    d.items = pl.items;
+    d.num_items = plan->cap_items;
+    d.count = counts;
+    d.rows_per_item = 8 * plan->decode_nt;
+    d.q = static_cast<const uint16_t*>(q);
+    d.num_q_heads = s.num_q_heads;
+    d.num_kv_heads = s.num_kv_heads;
+    d.head_dim = s.head_dim;
+    d.causal = s.causal;
+    d.scale_log2 = scale_log2;
+    d.out = static_cast<uint16_t*>(out);
+    d.lse = lse;
+    d.part_o = reinterpret_cast<float*>(ws + plan->off_part_o);
+    d.part_lse = reinterpret_cast<float*>(ws + plan->off_part_lse);
+    d.err = err;
+    d.kv = kv;
+    st = check_cuda(launch_decode(d, &plan->dec_inline, plan->decode_nt, stream),
+                    "decode launch");
+    if (st != RPA_OK) return st;
+    MergeLaunch m{};
+    m.rows = pl.rows;
+    m.num_rows = plan->cap_rows;
+    m.count = counts + 1;
+    m.rows_per_item = d.rows_per_item;
+    m.num_q_heads = s.num_q_heads;
+    m.num_kv_heads = s.num_kv_heads;
+    m.head_dim = s.head_dim;
+    m.part_o = d.part_o;
+    m.part_lse = d.part_lse;
+    m.out = d.out;
+    m.lse = lse;
+    st = check_cuda(launch_merge(m, &plan->merge_inline, stream), "merge launch");
+    if (st != RPA_OK) return st;
+    st = check_cuda(cudaEventRecord(plan->join_ev, pf_stream), "join record");
+    if (st != RPA_OK) return st;
+    return check_cuda(cudaStreamWaitEvent(stream, plan->join_ev, 0), "join wait");
+  }
+
   // A mixed batch runs the tensor-core kernel on the library's side stream, concurrently with
   // the split-KV decode kernel on the caller's stream: the decode CTAs fill the SMs that the
   // long prefill CTAs leave free.  The caller's stream waits for both before it goes on.
@@ -573,7 +745,7 @@ rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const 
   }
 
   if (!plan->pf_tiles.empty()) {
-    PrefillLaunch p;
+    PrefillLaunch p{};
     p.tiles = plan->inline_lists ? nullptr : reinterpret_cast<const PrefillTile*>(ws + plan->off_pf);
     p.num_tiles = (int32_t)plan->pf_tiles.size();
     p.q = static_cast<const uint16_t*>(q);
@@ -593,7 +765,7 @@ rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const 
     if (st != RPA_OK) return st;
   }
   if (!plan->dec_items.empty()) {
-    DecodeLaunch d;
+    DecodeLaunch d{};
     d.items = plan->inline_lists ? nullptr : reinterpret_cast<const DecodeItem*>(ws + plan->off_dec);
     d.num_items = (int32_t)plan->dec_items.size();
     d.rows_per_item = 8 * plan->decode_nt;
@@ -617,7 +789,7 @@ rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const 
     st = check_cuda(launch_decode(d, &plan->dec_inline, plan->decode_nt, stream), "decode launch");
     if (st != RPA_OK) return st;
     if (!plan->merge_rows.empty()) {
-      MergeLaunch m;
+      MergeLaunch m{};
       m.rows = plan->inline_lists ? nullptr : reinterpret_cast<const MergeRow*>(ws + plan->off_merge);
       m.num_rows = (int32_t)plan->merge_rows.size();
       m.rows_per_item = d.rows_per_item;

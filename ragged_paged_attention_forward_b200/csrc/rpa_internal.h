@@ -28,6 +28,7 @@ enum DeviceErrorCode : int {
   kErrPrefillWait = 1 << 1,
   kErrBadIndex = 1 << 2,
   kErrBadPosition = 1 << 3,
+  kErrLimits = 1 << 4,       // a device-planned step exceeded the plan's limits
 };
 
 // One (sequence, key range) item of the split-KV decode kernel; one CTA per (item, KV head).
@@ -88,6 +89,7 @@ struct PagedKV {
 struct DecodeLaunch {
   const DecodeItem* items;   // null: the items are the kernel's inline parameter list
   int32_t num_items;
+  const int32_t* count;      // device-planned steps: number of valid items (null: num_items)
   int32_t rows_per_item;     // 8 * NT: stride of the partial-result rows
   const uint16_t* q;         // bf16 [T, Hq, D]
   int32_t num_q_heads;
@@ -112,6 +114,7 @@ struct DecodeLaunch {
 struct MergeLaunch {
   const MergeRow* rows;      // null: inline parameter list
   int32_t num_rows;
+  const int32_t* count;      // device-planned steps: number of valid rows (null: num_rows)
   int32_t rows_per_item;
   int32_t num_q_heads;
   int32_t num_kv_heads;
@@ -125,6 +128,7 @@ struct MergeLaunch {
 struct PrefillLaunch {
   const PrefillTile* tiles;  // null: inline parameter list
   int32_t num_tiles;
+  const int32_t* count;      // device-planned steps: number of valid tiles (null: num_tiles)
   const uint16_t* q;
   int32_t num_tokens;
   int32_t num_q_heads;
@@ -156,6 +160,7 @@ struct WriteLaunch {
   int32_t max_blocks;
   int32_t layout;
   int32_t num_pages;
+  int32_t tokens_on_device;  // 1: num_tokens is a bound, the step has cu_seqlens_q[num_seqs]
   int* err;
 };
 
@@ -186,8 +191,31 @@ struct RotaryLaunch {
   int* err;
 };
 
+// The device-side planner: reads the step's lengths on the device and writes the work lists
+// (and their sizes) into the workspace, so that a step needs no host arrays and can be
+// captured in a CUDA graph.  Limits are fixed when the plan is made.
+struct PlanDeviceLaunch {
+  const int32_t* cu_seqlens_q;   // [B+1]
+  const int32_t* seq_lens_k;     // [B]
+  int32_t num_seqs;
+  int32_t max_tokens;
+  int32_t max_kv_len;
+  int32_t num_q_heads;
+  int32_t num_kv_heads;
+  int32_t causal;
+  int32_t split_keys;
+  int32_t decode_rows;           // a sequence goes to the decode kernel when q_len * G <= this
+  int32_t cap_items, cap_rows, cap_tiles;
+  DecodeItem* items;
+  MergeRow* rows;
+  PrefillTile* tiles;
+  int32_t* counts;               // [3]: items, merge rows, tiles
+  int* err;
+};
+
 // Launchers (return the cudaError_t of the launch).
 cudaError_t launch_write_kv(const WriteLaunch& p, cudaStream_t stream);
+cudaError_t launch_plan_device(const PlanDeviceLaunch& p, cudaStream_t stream);
 cudaError_t launch_rotary_write(const RotaryLaunch& p, cudaStream_t stream);
 cudaError_t launch_decode(const DecodeLaunch& p, const DecodeItemsInline* inl, int nt,
                           cudaStream_t stream);

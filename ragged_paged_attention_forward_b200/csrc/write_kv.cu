@@ -29,7 +29,10 @@ __global__ void __launch_bounds__(256) write_kv_kernel(WriteLaunch p) {
   const int nwarps = gridDim.x * warps_per_block;
   const int row_chunks = p.head_dim / 8;                 // 16-byte chunks per D-row
   const int tok_chunks = p.num_kv_heads * row_chunks;   // chunks per token per K or V
-  for (int t = warp; t < p.num_tokens; t += nwarps) {
+  // device-planned steps: num_tokens is only a bound, the step's count is cu[num_seqs]
+  const int T = p.tokens_on_device ? min(p.num_tokens, __ldg(p.cu_seqlens_q + p.num_seqs))
+                                   : p.num_tokens;
+  for (int t = warp; t < T; t += nwarps) {
     const int b = seq_of_token(p.cu_seqlens_q, p.num_seqs, t);
     const int t0 = __ldg(p.cu_seqlens_q + b);
     const int q_len = __ldg(p.cu_seqlens_q + b + 1) - t0;

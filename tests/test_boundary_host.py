@@ -196,3 +196,32 @@ def test_rotary_write_rejects_on_host(over, rotary, status):
 def test_rotary_write_zero_tokens_is_a_no_op():
     p = api.rpa_plan(**_shape(num_seqs=2, num_tokens=0, cu_seqlens_q=[0, 0, 0]))
     assert _rotary_status(p, dict()) == api.RPA_OK
+
+
+def _device_plan(**kw):
+    s = dict(num_seqs=4, max_tokens=512, num_q_heads=32, num_kv_heads=8, head_dim=128,
+             page_size=16, num_pages=1000, max_blocks_per_seq=64, layout=0, causal=True,
+             max_kv_len=1024)
+    s.update(kw)
+    return api.rpa_plan_device(**s)
+
+
+def test_device_plan_sizes_its_workspace_for_the_limits():
+    p = _device_plan()
+    info = p.info()
+    assert info.batch_class == api.CLASS_AUTO
+    assert info.num_decode_items == 4 * (1024 // info.decode_split_keys)
+    assert info.num_merge_rows == 512 and info.num_prefill_tiles == 512 // 128 + 4
+    assert p.workspace_bytes >= info.num_decode_items * 32 and p.workspace_bytes % 256 == 0
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(max_kv_len=0), api.RPA_ERR_SHAPE),
+    (dict(max_kv_len=64 * 16 + 1), api.RPA_ERR_SHAPE),
+    (dict(head_dim=96), api.RPA_ERR_UNSUPPORTED),
+    (dict(decode_split_keys=100), api.RPA_ERR_INVALID_ARG),
+])
+def test_device_plan_rejects(kw, status):
+    with pytest.raises(api.RPAError) as e:
+        _device_plan(**kw)
+    assert e.value.status == status
