@@ -503,6 +503,50 @@ def measure(name, runner, steps, warmup, peaks):
     return res
 
 
+def measure_device_planned_decode(steps, warmup, peaks):
+    """The decode step with a device-side plan (rpa_plan_device), captured in CUDA graphs and
+    replayed: the planner kernel builds the work lists from the device lengths, then the
+    KV write, the decode kernel and the merge run (the tensor-core kernel's CTAs all return
+    at once).  One graph per KV-pool copy, replayed in turn, so no step finds K/V in L2."""
+    from ragged_paged_attention_forward_b200 import api
+    b, _ = make_workload("decode")
+    runner = Runner("decode", b, None)
+    d = runner.d
+    plan = api.rpa_plan_device(num_seqs=b.num_seqs, max_tokens=b.num_tokens,
+                               num_q_heads=b.num_q_heads, num_kv_heads=b.num_kv_heads,
+                               head_dim=b.head_dim, page_size=b.page_size,
+                               num_pages=b.num_pages, max_blocks_per_seq=b.max_blocks,
+                               layout=b.layout, causal=b.causal,
+                               max_kv_len=int(b.seq_lens_k.max()))
+    ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(d["q"])
+
+    def step(kp, vp):
+        api.rpa_forward(plan, d["q"], d["k_new"], d["v_new"], kp, vp, d["block_table"],
+                        d["cu_seqlens_q"], d["seq_lens_k"], None, None, b.scale, out, None, ws)
+
+    for kp, vp in runner.pools:  # warm-up outside the capture
+        step(kp, vp)
+    torch.cuda.synchronize()
+    graphs = []
+    for kp, vp in runner.pools:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(kp, vp)
+        graphs.append(g)
+    ms = timed_loop(lambda i: graphs[i % len(graphs)].replay(), steps, warmup)
+    table, count = runner.host_tables()
+    w = work(b, table, count)
+    gbps = w["step_bytes"] / (ms * 1e-3) / 1e9
+    info = plan.info()
+    res = {"workload": WORKLOAD_TEXT["decode"] + "; device-planned, CUDA-graph replay",
+           "ms_per_step": ms, "step_GBps": gbps, "frac_of_hbm": gbps / peaks["hbm_gbs"],
+           "launches_per_step": info.launches_forward, "decode_split_keys":
+           info.decode_split_keys}
+    del graphs
+    return res
+
+
 def measure_input_pass(steps, warmup, peaks):
     """The input pass with rotary embedding (rpa_rotary_write_kv) on the prefill workload's
     16384 new tokens: packed QKV in, RoPE over all 128 dims (split pairs), Q out, K/V
@@ -744,6 +788,8 @@ def run_gpu(args):
             del r2, b2
             torch.cuda.empty_cache()
         secondary["input_pass"] = measure_input_pass(args.steps, args.warmup, peaks)
+        secondary["decode_device_planned"] = measure_device_planned_decode(args.steps,
+                                                                           args.warmup, peaks)
         line["secondary"] = secondary
         if "prefill" in secondary:
             line["prefill_TFLOPs"] = secondary["prefill"]["attn_TFLOPs"]

@@ -141,7 +141,8 @@ RPA_API rpa_status rpa_plan(const rpa_shape* shape, const int32_t* cu_seqlens_q,
  *                 not supported (RPA_ERR_UNSUPPORTED).
  *   workspace_bytes  receives the workspace size for these limits.
  * Each call of rpa_forward with this plan launches a one-CTA planner kernel (a sequence
- * goes to the split-KV decode kernel when q_len * G <= 16, else to the tensor-core kernel),
+ * goes to the split-KV decode kernel when q_len * G fits 8, 16 or 32 rows -- the smallest
+ * of these that holds G -- else to the tensor-core kernel),
  * then every kernel with its largest grid; CTAs past the step's counts return at once.
  * A step beyond the limits (T, kv_len, q_len > kv_len) computes nothing and sets bit 16
  * of the device error word.  rpa_write_kv with this plan writes the step's tokens only.

@@ -382,10 +382,16 @@ rpa_status rpa_plan_device(const rpa_shape* shape, int32_t max_kv_len,
   plan->device_mode = true;
   plan->max_kv_len = max_kv_len;
   plan->batch_class = RPA_CLASS_AUTO;
-  // every sequence whose query heads x tokens fit 16 MMA columns goes to the decode kernel
-  plan->decode_nt = 2;
-  plan->split_keys = o.decode_split_keys ? o.decode_split_keys : 512;
+  // a sequence goes to the decode kernel when its query heads x tokens fit the smallest MMA
+  // column count that holds one token's group (8, 16 or 32)
+  const int G = s.num_q_heads / s.num_kv_heads;
+  plan->decode_nt = G <= 8 ? 1 : (G <= 16 ? 2 : 4);
   const int B = s.num_seqs;
+  // split size for an average context of max_kv_len / 2, as the host planner would pick it
+  plan->split_keys = o.decode_split_keys
+                         ? o.decode_split_keys
+                         : auto_split_keys((long)B * (max_kv_len / 2) * s.num_kv_heads,
+                                           device_sm_count());
   const long splits = (max_kv_len + plan->split_keys - 1) / plan->split_keys;
   plan->cap_items = (int)std::min<long>((long)B * splits, 1L << 24);
   plan->cap_rows = std::max(s.num_tokens, 1);
