@@ -52,7 +52,10 @@ __global__ void __launch_bounds__(256, 4) rotary_write_kernel(RotaryLaunch p) {
   const bool rot_any = p.cos != nullptr;
   const int half_lanes = rd / 16;       // split mode: lanes holding the first rd/2 dims
   const long nwarps = (long)gridDim.x * warps_per_block;
-  for (long t = (long)blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < p.num_tokens;
+  // num_tokens is exact for host plans and a bound for device plans: the step's own count
+  // is cu_seqlens_q[num_seqs]
+  const int T = min(p.num_tokens, __ldg(p.cu_seqlens_q + p.num_seqs));
+  for (long t = (long)blockIdx.x * warps_per_block + (threadIdx.x >> 5); t < T;
        t += nwarps) {
     // ---- per token: sequence, position, pages, the cos/sin entries of this lane's dims.
     // With at most 32 sequences the warp finds the sequence in one round of loads: lane i

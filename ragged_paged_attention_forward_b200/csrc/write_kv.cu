@@ -40,6 +40,10 @@ __global__ void __launch_bounds__(256) write_kv_kernel(WriteLaunch p) {
     const int pos = past + (t - t0);
     const int blk = pos / p.page_size;
     const int slot = pos - blk * p.page_size;
+    if (pos < 0 || blk >= p.max_blocks) {  // a device-planned step past its limits
+      if (lane == 0) atomicOr(p.err, kErrLimits);
+      continue;
+    }
     const uint4* ksrc = reinterpret_cast<const uint4*>(p.k_new + (size_t)t * tok_chunks * 8);
     const uint4* vsrc = reinterpret_cast<const uint4*>(p.v_new + (size_t)t * tok_chunks * 8);
     if (p.layout == 0) {
