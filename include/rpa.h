@@ -260,6 +260,34 @@ RPA_API rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new
                        void* stream);
 
 /*
+ * rpa_forward_kv8 -- rpa_forward over an fp8 (e4m3) KV cache with per-KV-head scales.  Not
+ * in the pages' shipped kernels: the WebGPU page's commit "FlashAttention: optional
+ * seqlens_q input" lists the quantised KV cache under "Not in scope (deferred)"; this is
+ * that extension for the decode path, which is bandwidth-bound, so one byte per element
+ * halves its traffic.
+ *
+ *   k_pool, v_pool    device uint8 pools of e4m3 codes (1 sign, 4 exponent bits with bias
+ *                     7, 3 mantissa bits; no infinities; 0x7F / 0xFF are NaN; largest
+ *                     finite 448), in shape.layout with one byte per element.
+ *   k_scale, v_scale  device fp32 [Hkv]: key j of KV head h is e4m3(k_pool[j, h]) * k_scale[h]
+ *                     (the same for V).  Positive and finite.
+ *   k_new, v_new      device bf16 [T, Hkv, D], or both NULL.  Each new element x is stored as
+ *                     the e4m3 code nearest to fp32(x) / scale (IEEE fp32 division; ties to
+ *                     the even code; magnitudes past 448 saturate to +-448).
+ *   the rest          as for rpa_forward (no group tables).
+ * Supported: head_dim 128 and host plans whose rows all go to the split-KV decode kernel
+ * (rpa_plan_info.batch_class == RPA_CLASS_DECODE, or num_prefill_tiles == 0); anything else
+ * returns RPA_ERR_UNSUPPORTED.  Scores and P.V run on f16 operands (e4m3 -> f16 is exact;
+ * q must stay within f16's range, |q| < 65504) with fp32 accumulation.
+ */
+RPA_API rpa_status rpa_forward_kv8(rpa_plan_t plan, const void* q, const void* k_new,
+                                   const void* v_new, void* k_pool, void* v_pool,
+                                   const float* k_scale, const float* v_scale,
+                                   const int32_t* block_table, const int32_t* cu_seqlens_q,
+                                   const int32_t* seq_lens_k, float scale, void* out, float* lse,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * rpa_forward_no_alloc -- rpa_forward for callers that cannot allocate device memory.
  * No counterpart in the pages: this is a convenience of this library.
  *

@@ -32,6 +32,17 @@ What it computes (plain definitions, written out; no tiling, no fusion, no reord
   commit).  Each rotated value is the exact ``x1 c - x2 s`` / ``x1 s + x2 c`` rounded once to
   bf16 (nearest, ties to even).
 
+* ``e4m3_decode`` / ``e4m3_encode`` / ``write_kv8`` / ``forward_kv8`` -- the fp8 KV cache
+  (the quantised cache that the WebGPU page's commit "FlashAttention: optional seqlens_q
+  input" defers under "Not in scope (deferred)").  A code is the e4m3 format written out:
+  sign, 4 exponent bits with bias 7, 3 mantissa bits; exponent field 0 holds the subnormals
+  ``m/8 * 2^-6``; ``S.1111.111`` is NaN; no infinities; the largest finite value is 448.
+  Pool element = ``decode(code) * scale[kv head]``; a new element ``x`` is stored as the
+  code nearest to ``fp32(x) / fp32(scale)`` (the quotient rounded once to fp32, then ties to
+  the even code, magnitudes past 448 clamped to 448).  Plain reading of a silent page: the
+  format and the rounding are the standard e4m3 ones; the per-KV-head scale is the plainest
+  of the "per-page or per-head" choices.
+
 Inputs are bf16 bit patterns (numpy ``uint16``) or torch bf16 tensors; every bf16 value is
 widened exactly to fp64 before any arithmetic.  Cache writes move the bf16 bit patterns
 unchanged.
@@ -140,8 +151,8 @@ def write_kv(k_pool, v_pool, k_new, v_new, block_table, cu_seqlens_q, seq_lens_k
 def logical_rows(pool, block_table, layout: int, b: int, h: int, n: int,
                  page_size: int) -> np.ndarray:
     """Keys (or values) ``0 .. n-1`` of sequence ``b``, KV head ``h``, gathered through the
-    block table: uint16 ``[n, D]``."""
-    p = bits16(pool)
+    block table: uint16 ``[n, D]`` (bf16 pools) or uint8 ``[n, D]`` (e4m3 code pools)."""
+    p = codes8(pool) if _is_codes8(pool) else bits16(pool)
     bt = ints(block_table)
     pos = np.arange(n, dtype=np.int64)
     pages = page_of(bt, layout, b, h, pos, page_size)
@@ -183,9 +194,11 @@ def attend_row(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float):
 def attention(q, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k, *, scale: float,
               causal: bool, page_size: int, layout: int = SEQ_MAJOR, num_kv_heads: int,
               group_table=None, group_count=None,
-              rows: Optional[Iterable[Tuple[int, int]]] = None):
+              rows: Optional[Iterable[Tuple[int, int]]] = None, kv_scales=None):
     """Attention of every (token, query head) row -- or of ``rows`` only -- against the pools
-    *as given* (call ``write_kv`` first for the fused semantics).
+    *as given* (call ``write_kv`` first for the fused semantics).  With ``kv_scales =
+    (k_scale, v_scale)`` the pools hold e4m3 codes and key ``j`` of KV head ``h`` is
+    ``e4m3_decode(code) * k_scale[h]`` (likewise V).
 
     Returns ``(out [T, Hq, D] fp64, lse [T, Hq] fp64)``; rows not computed are NaN.
     """
@@ -219,8 +232,15 @@ def attention(q, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k, *, scale
             heads = [hk * G + g for g in range(G)]
             if wanted is not None and not any(h in wanted[t] for t in toks for h in heads):
                 continue
-            K = widen(logical_rows(k_pool, block_table, layout, b, hk, kv_len, page_size))
-            V = widen(logical_rows(v_pool, block_table, layout, b, hk, kv_len, page_size))
+            if kv_scales is None:
+                K = widen(logical_rows(k_pool, block_table, layout, b, hk, kv_len, page_size))
+                V = widen(logical_rows(v_pool, block_table, layout, b, hk, kv_len, page_size))
+            else:
+                ks, vs = (np.asarray(x, dtype=np.float32) for x in kv_scales)
+                K = e4m3_decode(logical_rows(k_pool, block_table, layout, b, hk, kv_len,
+                                             page_size)) * float(ks[hk])
+                V = e4m3_decode(logical_rows(v_pool, block_table, layout, b, hk, kv_len,
+                                             page_size)) * float(vs[hk])
             selected = None
             if gt is not None:
                 selected = set(int(x) for x in gt[b, hk, :int(gc[b, hk])])
@@ -395,3 +415,114 @@ def rotary_write_kv(q, k, v, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens
     kp, vp = write_kv(k_pool, v_pool, kb, vb, block_table, cu_seqlens_q, seq_lens_k,
                       page_size, layout)
     return np.ascontiguousarray(qb), kp, vp
+
+
+# --------------------------------------------------------------------------------------
+# fp8 (e4m3) KV cache
+# --------------------------------------------------------------------------------------
+
+def _is_codes8(x) -> bool:
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            return x.dtype == torch.uint8
+    except ImportError:  # pragma: no cover
+        pass
+    return np.asarray(x).dtype == np.uint8
+
+
+def codes8(x) -> np.ndarray:
+    """e4m3 codes as numpy ``uint8``."""
+    try:
+        import torch
+        if isinstance(x, torch.Tensor):
+            assert x.dtype == torch.uint8, x.dtype
+            return x.detach().cpu().contiguous().numpy()
+    except ImportError:  # pragma: no cover
+        pass
+    x = np.asarray(x)
+    assert x.dtype == np.uint8, x.dtype
+    return x
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """e4m3 codes -> fp64, from the format's fields (exact)."""
+    c = codes8(codes).astype(np.int64)
+    sign = np.where(c >> 7, -1.0, 1.0)
+    e = (c >> 3) & 15
+    m = (c & 7).astype(np.float64)
+    mag = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1.0 + m / 8.0) * np.exp2(e - 7.0))
+    mag = np.where((e == 15) & ((c & 7) == 7), np.nan, mag)
+    return sign * mag
+
+
+# the 127 non-negative finite codes in increasing order of value (code i has value
+# _E4M3_VALUES[i]; consecutive codes are consecutive values)
+_E4M3_VALUES = e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+
+
+def e4m3_encode(x) -> np.ndarray:
+    """fp64 values (typically fp32 quotients) -> e4m3 codes: nearest value, ties to the even
+    code (mantissa LSB 0), magnitudes at or past 448 clamped to 448, NaN -> 0x7F | sign."""
+    x = np.asarray(x, dtype=np.float64)
+    a = np.abs(x)
+    sign = np.signbit(x).astype(np.uint8) << np.uint8(7)
+    hi = np.searchsorted(_E4M3_VALUES, np.minimum(a, 448.0), side="left")  # first >= a
+    hi = np.clip(hi, 0, 0x7E)
+    lo = np.clip(hi - 1, 0, 0x7E)
+    d_hi = _E4M3_VALUES[hi] - a
+    d_lo = a - _E4M3_VALUES[lo]
+    pick_lo = (d_lo < d_hi) | ((d_lo == d_hi) & (lo % 2 == 0))
+    code = np.where(pick_lo, lo, hi)
+    code = np.where(a >= 448.0, 0x7E, code)
+    code = np.where(np.isnan(x), 0x7F, code).astype(np.uint8)
+    return code | sign
+
+
+def e4m3_quantize(bits, scale: float) -> np.ndarray:
+    """bf16 bit patterns -> codes of ``fp32(x) / fp32(scale)`` (one fp32 rounding, then the
+    e4m3 rounding of ``e4m3_encode``)."""
+    y = widen(bits).astype(np.float32) / np.float32(scale)
+    return e4m3_encode(y.astype(np.float64))
+
+
+def write_kv8(k_pool, v_pool, k_new, v_new, k_scale, v_scale, block_table, cu_seqlens_q,
+              seq_lens_k, page_size: int, layout: int = SEQ_MAJOR):
+    """``write_kv`` for e4m3 code pools: each new token's K/V row is quantised with its KV
+    head's scale and stored in its slot.  Returns copies of the code pools."""
+    kp = codes8(k_pool).copy()
+    vp = codes8(v_pool).copy()
+    kn = bits16(k_new)
+    vn = bits16(v_new)
+    ks = np.asarray(k_scale, dtype=np.float32)
+    vs = np.asarray(v_scale, dtype=np.float32)
+    bt = ints(block_table)
+    num_kv_heads = kn.shape[1]
+    for b, (t0, q_len, kv_len, past) in enumerate(seq_ranges(cu_seqlens_q, seq_lens_k)):
+        for i in range(q_len):
+            t = t0 + i
+            pos = past + i
+            slot = pos % page_size
+            for h in range(num_kv_heads):
+                page = bt[b, pos // page_size] if layout == SEQ_MAJOR else bt[b, h, pos // page_size]
+                dst = (page, slot, h) if layout == SEQ_MAJOR else (page, slot)
+                kp[dst] = e4m3_quantize(kn[t, h], float(ks[h]))
+                vp[dst] = e4m3_quantize(vn[t, h], float(vs[h]))
+    return kp, vp
+
+
+def forward_kv8(q, k_new, v_new, k_pool, v_pool, k_scale, v_scale, block_table, cu_seqlens_q,
+                seq_lens_k, *, scale: float, causal: bool, page_size: int,
+                layout: int = SEQ_MAJOR, rows=None):
+    """The fused step over e4m3 code pools: quantising write, then attention over the
+    dequantised keys and values.  Returns ``(out, lse, k_pool_after, v_pool_after)``."""
+    num_kv_heads = len(np.atleast_1d(k_scale))
+    if k_new is not None:
+        kp, vp = write_kv8(k_pool, v_pool, k_new, v_new, k_scale, v_scale, block_table,
+                           cu_seqlens_q, seq_lens_k, page_size, layout)
+    else:
+        kp, vp = codes8(k_pool).copy(), codes8(v_pool).copy()
+    out, lse = attention(q, kp, vp, block_table, cu_seqlens_q, seq_lens_k, scale=scale,
+                         causal=causal, page_size=page_size, layout=layout,
+                         num_kv_heads=num_kv_heads, rows=rows, kv_scales=(k_scale, v_scale))
+    return out, lse, kp, vp

@@ -92,6 +92,9 @@ def lib() -> ctypes.CDLL:
         L.rpa_forward.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_float,
                                   _P, _P, _P, ctypes.c_size_t, _P]
         L.rpa_forward.restype = ctypes.c_int
+        L.rpa_forward_kv8.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+                                      ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]
+        L.rpa_forward_kv8.restype = ctypes.c_int
         L.rpa_forward_no_alloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                            ctypes.c_float, _P, _P, _P]
         L.rpa_forward_no_alloc.restype = ctypes.c_int
@@ -243,6 +246,18 @@ def rpa_forward(plan: Plan, q, k_new, v_new, k_pool, v_pool, block_table, cu_seq
         _ptr(block_table), _ptr(cu_seqlens_q), _ptr(seq_lens_k), _ptr(group_table),
         _ptr(group_count), ctypes.c_float(scale), _ptr(out), _ptr(lse), _ptr(workspace), nbytes,
         _stream(stream)))
+
+
+def rpa_forward_kv8(plan: Plan, q, k_new, v_new, k_pool, v_pool, k_scale, v_scale,
+                    block_table, cu_seqlens_q, seq_lens_k, scale: float, out, lse, workspace,
+                    stream=None):
+    """The fused step over e4m3 (uint8) K/V pools with fp32 per-KV-head scales
+    k_scale, v_scale [Hkv] (decode-class plans, head_dim 128; see include/rpa.h)."""
+    nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
+    _check("rpa_forward_kv8", lib().rpa_forward_kv8(
+        plan.handle, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool),
+        _ptr(k_scale), _ptr(v_scale), _ptr(block_table), _ptr(cu_seqlens_q), _ptr(seq_lens_k),
+        ctypes.c_float(scale), _ptr(out), _ptr(lse), _ptr(workspace), nbytes, _stream(stream)))
 
 
 NO_ALLOC_WORKSPACE_BYTES = 8 << 20

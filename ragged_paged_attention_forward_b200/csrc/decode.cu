@@ -35,13 +35,14 @@ constexpr int kConsumerWarps = 4;
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxItemPages = kMaxSplitKeys / 16 + 1;
 
-template <int D>
+template <int D, bool KV8>
 struct DecodeGeom {
-  static constexpr int kHalves = D / 64;
+  // stage rows are stored in 128-byte halves: 64 bf16 elements, or all 128 e4m3 codes
+  static constexpr int kHalves = KV8 ? 1 : D / 64;
   static constexpr int kStageKeys = kDecodeStageKeys;                 // 64
   static constexpr int kHalfBytes = kStageKeys * 128;                 // 8 KB per half-row tile
   static constexpr int kTensorStageBytes = kHalves * kHalfBytes;      // K (or V) per stage
-  static constexpr int kStages = D == 128 ? 3 : 4;
+  static constexpr int kStages = KV8 ? 6 : D == 128 ? 3 : 4;          // ~96 KB in flight
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kStages * kTensorStageBytes;
   static constexpr int kPagesOff = 2 * kStages * kTensorStageBytes;
@@ -53,18 +54,22 @@ struct DecodeGeom {
                 "stage alignment");
   static_assert(kHalfBytes % 1024 == 0, "half-tile alignment");
   static_assert(kBarOff % 8 == 0, "mbarrier alignment");
+  static_assert(!KV8 || D == 128, "e4m3 pools: head_dim 128");
+  // the four warps' states are combined in the stage ring once it is drained
+  static_assert(2 * kConsumerWarps * 32 * 4 + kConsumerWarps * 32 * (D + 4) * 4 <= kPagesOff,
+                "combine area");
 };
 
 struct alignas(16) U4 {
   uint32_t x, y, z, w;
 };
 
-template <int D, int NT>
+template <int D, int NT, bool KV8>
 __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap vmap, DecodeLaunch p,
                         const __grid_constant__ DecodeItemsInline inl) {
-  using Geo = DecodeGeom<D>;
+  using Geo = DecodeGeom<D, KV8>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -120,7 +125,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       // loaded; the proxy fence orders these plain stores before the TMA reads below.
       const int lo = max(past, it.k_begin);
       const int ntok = it.k_end - lo;
-      const int chunks = D / 8;  // 16-byte chunks per row
+      const int chunks = KV8 ? D / 16 : D / 8;  // 16-byte chunks per pool row
       for (int idx = lane; idx < 2 * ntok * chunks; idx += 32) {
         const int which = idx / (ntok * chunks);
         const int rem = idx - which * ntok * chunks;
@@ -136,10 +141,29 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         const size_t row = p.kv.layout == 0
                                ? ((size_t)page * P + (pos & (P - 1))) * p.num_kv_heads + h
                                : (size_t)page * P + (pos & (P - 1));
-        const uint16_t* src = (which == 0 ? p.k_new : p.v_new) +
-                              ((size_t)tok * p.num_kv_heads + h) * D + c * 8;
-        uint16_t* dst = (which == 0 ? p.k_pool_w : p.v_pool_w) + row * D + c * 8;
-        *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
+        if constexpr (KV8) {
+          // 16 elements -> 16 codes: e4m3(fp32(x) / scale), nearest even, saturating
+          const uint16_t* src = (which == 0 ? p.k_new : p.v_new) +
+                                ((size_t)tok * p.num_kv_heads + h) * D + c * 16;
+          const float sc = __ldg((which == 0 ? p.k_scale : p.v_scale) + h);
+          const uint4 a = __ldg(reinterpret_cast<const uint4*>(src));
+          const uint4 b = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+          auto q2 = [sc](uint32_t v) {  // a bf16 pair -> two codes
+            return pack_e4m3x2(__fdiv_rn(__uint_as_float(v << 16), sc),
+                               __fdiv_rn(__uint_as_float(v & 0xffff0000u), sc));
+          };
+          uint8_t* dst = static_cast<uint8_t*>(which == 0 ? p.k_pool_w : p.v_pool_w) + row * D +
+                         c * 16;
+          *reinterpret_cast<uint4*>(dst) =
+              make_uint4(q2(a.x) | (q2(a.y) << 16), q2(a.z) | (q2(a.w) << 16),
+                         q2(b.x) | (q2(b.y) << 16), q2(b.z) | (q2(b.w) << 16));
+        } else {
+          const uint16_t* src = (which == 0 ? p.k_new : p.v_new) +
+                                ((size_t)tok * p.num_kv_heads + h) * D + c * 8;
+          uint16_t* dst = static_cast<uint16_t*>(which == 0 ? p.k_pool_w : p.v_pool_w) +
+                          row * D + c * 8;
+          *reinterpret_cast<uint4*>(dst) = __ldg(reinterpret_cast<const uint4*>(src));
+        }
       }
       asm volatile("fence.proxy.async.global;" ::: "memory");
       __syncwarp();
@@ -200,8 +224,16 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           reinterpret_cast<const uint32_t*>(p.q + ((size_t)tok * Hq + hq) * D);
 #pragma unroll
       for (int kk = 0; kk < KT; ++kk) {
-        bq[nt][kk][0] = ok ? __ldg(qrow + kk * 8 + (lane & 3)) : 0u;
-        bq[nt][kk][1] = ok ? __ldg(qrow + kk * 8 + 4 + (lane & 3)) : 0u;
+        if constexpr (KV8) {
+          // f16 operands; the head dims of a k-step are taken in the order that makes each
+          // lane's K bytes contiguous: fragment columns (2t, 2t+1 | 2t+8, 2t+9) are dims
+          // 16kk + 4t .. 4t+3 (the same order for Q and K leaves Q.K unchanged)
+          bq[nt][kk][0] = ok ? bf16x2_to_f16x2(__ldg(qrow + kk * 8 + 2 * (lane & 3))) : 0u;
+          bq[nt][kk][1] = ok ? bf16x2_to_f16x2(__ldg(qrow + kk * 8 + 2 * (lane & 3) + 1)) : 0u;
+        } else {
+          bq[nt][kk][0] = ok ? __ldg(qrow + kk * 8 + (lane & 3)) : 0u;
+          bq[nt][kk][1] = ok ? __ldg(qrow + kk * 8 + 4 + (lane & 3)) : 0u;
+        }
       }
     }
     float m[NT][2], ls[NT][2];
@@ -225,6 +257,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         lim[nt][j] = p.causal ? min(it.k_end, past + tok_i + 1) : it.k_end;
       }
 
+    // log2-domain score scale; e4m3 keys carry their KV head's scale (element = code * s)
+    const float sl2 = KV8 ? p.scale_log2 * __ldg(p.k_scale + h) : p.scale_log2;
     const int ar = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;  // K ldmatrix row
     const int vr = warp * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;  // V ldmatrix.trans row
     for (int s = 0; s < nstages; ++s) {
@@ -238,16 +272,33 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
         float c[NT][4];
 #pragma unroll
         for (int nt = 0; nt < NT; ++nt) c[nt][0] = c[nt][1] = c[nt][2] = c[nt][3] = 0.f;
+        if constexpr (KV8) {
+          // key rows g and g + 8 of the warp's 16 (same swizzle phase); per k-step each lane
+          // reads the 4 codes of dims 16kk + 4t .. 4t+3 of both rows
+          const int rg = warp * 16 + (lane >> 2);
 #pragma unroll
-        for (int kk = 0; kk < KT; ++kk) {
-          const int chunk = 2 * kk + (lane >> 4);
-          const uint32_t addr = kbase + (chunk >> 3) * Geo::kHalfBytes + ar * 128 +
-                                (((chunk & 7) ^ (ar & 7)) << 4);
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4(addr, a0, a1, a2, a3);
+          for (int kk = 0; kk < KT; ++kk) {
+            const uint32_t off = (uint32_t)(((kk ^ (rg & 7)) << 4) + 4 * (lane & 3));
+            const uint32_t kg = ld_shared_u32(kbase + rg * 128 + off);
+            const uint32_t kh = ld_shared_u32(kbase + (rg + 8) * 128 + off);
+            const uint32_t a0 = e4m3x2_to_f16x2(kg), a2 = e4m3x2_to_f16x2(kg >> 16);
+            const uint32_t a1 = e4m3x2_to_f16x2(kh), a3 = e4m3x2_to_f16x2(kh >> 16);
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-            mma_bf16_16816(c[nt], a0, a1, a2, a3, bq[nt][kk][0], bq[nt][kk][1]);
+            for (int nt = 0; nt < NT; ++nt)
+              mma_f16_16816(c[nt], a0, a1, a2, a3, bq[nt][kk][0], bq[nt][kk][1]);
+          }
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < KT; ++kk) {
+            const int chunk = 2 * kk + (lane >> 4);
+            const uint32_t addr = kbase + (chunk >> 3) * Geo::kHalfBytes + ar * 128 +
+                                  (((chunk & 7) ^ (ar & 7)) << 4);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4(addr, a0, a1, a2, a3);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+              mma_bf16_16816(c[nt], a0, a1, a2, a3, bq[nt][kk][0], bq[nt][kk][1]);
+          }
         }
         const int k_lo = key0 + (lane >> 2);
         const int k_hi = k_lo + 8;
@@ -257,8 +308,8 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           float pl[2], ph[2];
 #pragma unroll
           for (int j = 0; j < 2; ++j) {
-            const float s_lo = k_lo < lim[nt][j] ? c[nt][j] * p.scale_log2 : -CUDART_INF_F;
-            const float s_hi = k_hi < lim[nt][j] ? c[nt][2 + j] * p.scale_log2 : -CUDART_INF_F;
+            const float s_lo = k_lo < lim[nt][j] ? c[nt][j] * sl2 : -CUDART_INF_F;
+            const float s_hi = k_hi < lim[nt][j] ? c[nt][2 + j] * sl2 : -CUDART_INF_F;
             float tmax = fmaxf(s_lo, s_hi);
             tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 4));
             tmax = fmaxf(tmax, __shfl_xor_sync(0xffffffffu, tmax, 8));
@@ -276,8 +327,13 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
               acc[mt][nt][2 + j] *= alpha;
             }
           }
-          bp[nt][0] = movmatrix_trans(pack_bf16(pl[0], pl[1]));
-          bp[nt][1] = movmatrix_trans(pack_bf16(ph[0], ph[1]));
+          if constexpr (KV8) {
+            bp[nt][0] = movmatrix_trans(pack_f16(pl[0], pl[1]));
+            bp[nt][1] = movmatrix_trans(pack_f16(ph[0], ph[1]));
+          } else {
+            bp[nt][0] = movmatrix_trans(pack_bf16(pl[0], pl[1]));
+            bp[nt][1] = movmatrix_trans(pack_bf16(ph[0], ph[1]));
+          }
         }
         uint8_t* vtile = Vs + slot * Geo::kTensorStageBytes;
         const int nvalid = it.k_end - key0;
@@ -293,16 +349,44 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           __syncwarp();
         }
         const uint32_t vbase = smem_u32(vtile);
+        if constexpr (KV8) {
+          // V^T as the A operand from e4m3 rows: a transposing 8x8 load of byte pairs gives
+          // lane (g, t) the codes of dims 2g, 2g+1 of keys 2t, 2t+1; byte permutes split them
+          // into the (keys 2t, 2t+1) pairs of dim 2g (fragment row g) and of dim 2g+1 (row
+          // g + 8), so M-tile mt holds dims 16mt + 2r (rows r < 8) and 16mt + 2(r-8) + 1
+          const int vrow = warp * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
 #pragma unroll
-        for (int mt = 0; mt < KT; ++mt) {
-          const int chunk = 2 * mt + ((lane >> 3) & 1);
-          const uint32_t addr = vbase + (chunk >> 3) * Geo::kHalfBytes + vr * 128 +
-                                (((chunk & 7) ^ (vr & 7)) << 4);
-          uint32_t a0, a1, a2, a3;
-          ldsm_x4_trans(addr, a0, a1, a2, a3);
+          for (int mt = 0; mt < KT; mt += 2) {
+            const int chunk = mt + (lane >> 4);
+            const uint32_t addr = vbase + vrow * 128 + (((chunk & 7) ^ (vrow & 7)) << 4);
+            uint32_t r0, r1, r2, r3;
+            ldsm_x4_trans(addr, r0, r1, r2, r3);
+            const uint32_t x0 = e4m3x2_to_f16x2(__byte_perm(r0, 0, 0x0020));
+            const uint32_t x1 = e4m3x2_to_f16x2(__byte_perm(r0, 0, 0x0031));
+            const uint32_t x2 = e4m3x2_to_f16x2(__byte_perm(r1, 0, 0x0020));
+            const uint32_t x3 = e4m3x2_to_f16x2(__byte_perm(r1, 0, 0x0031));
+            const uint32_t y0 = e4m3x2_to_f16x2(__byte_perm(r2, 0, 0x0020));
+            const uint32_t y1 = e4m3x2_to_f16x2(__byte_perm(r2, 0, 0x0031));
+            const uint32_t y2 = e4m3x2_to_f16x2(__byte_perm(r3, 0, 0x0020));
+            const uint32_t y3 = e4m3x2_to_f16x2(__byte_perm(r3, 0, 0x0031));
 #pragma unroll
-          for (int nt = 0; nt < NT; ++nt)
-            mma_bf16_16816(acc[mt][nt], a0, a1, a2, a3, bp[nt][0], bp[nt][1]);
+            for (int nt = 0; nt < NT; ++nt) {
+              mma_f16_16816(acc[mt][nt], x0, x1, x2, x3, bp[nt][0], bp[nt][1]);
+              mma_f16_16816(acc[mt + 1][nt], y0, y1, y2, y3, bp[nt][0], bp[nt][1]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int mt = 0; mt < KT; ++mt) {
+            const int chunk = 2 * mt + ((lane >> 3) & 1);
+            const uint32_t addr = vbase + (chunk >> 3) * Geo::kHalfBytes + vr * 128 +
+                                  (((chunk & 7) ^ (vr & 7)) << 4);
+            uint32_t a0, a1, a2, a3;
+            ldsm_x4_trans(addr, a0, a1, a2, a3);
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+              mma_bf16_16816(acc[mt][nt], a0, a1, a2, a3, bp[nt][0], bp[nt][1]);
+          }
         }
         if (nvalid < 16) fence_proxy_async_smem();  // generic writes before the next TMA
       }
@@ -342,14 +426,20 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           float* o = red_o + (warp * COLS + col) * OPAD;
 #pragma unroll
           for (int mt = 0; mt < KT; ++mt) {
-            o[mt * 16 + (lane >> 2)] = acc[mt][nt][j];
-            o[mt * 16 + (lane >> 2) + 8] = acc[mt][nt][2 + j];
+            if constexpr (KV8) {  // fragment rows r, r + 8 are dims 16mt + 2r, 16mt + 2r + 1
+              o[mt * 16 + 2 * (lane >> 2)] = acc[mt][nt][j];
+              o[mt * 16 + 2 * (lane >> 2) + 1] = acc[mt][nt][2 + j];
+            } else {
+              o[mt * 16 + (lane >> 2)] = acc[mt][nt][j];
+              o[mt * 16 + (lane >> 2) + 8] = acc[mt][nt][2 + j];
+            }
           }
         }
     }
     asm volatile("bar.sync 1, 128;" ::: "memory");
     if (!*abort_flag) {
       const int Hkv = p.num_kv_heads;
+      const float vsc = KV8 ? __ldg(p.v_scale + h) : 1.f;  // e4m3 V: element = code * scale
       for (int idx = threadIdx.x; idx < rows * D; idx += kConsumerWarps * 32) {
         const int col = idx / D;
         const int d = idx - col * D;
@@ -365,7 +455,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
             O += red_o[(w * COLS + col) * OPAD + d] * f;
           }
         }
-        const float o = L > 0.f ? O / L : 0.f;
+        const float o = L > 0.f ? O / L * vsc : 0.f;
         const float lse2 = L > 0.f ? M + fast_log2(L) : -CUDART_INF_F;
         const int tok = it.t0 + col / G;
         const int hq = h * G + col % G;
@@ -434,17 +524,17 @@ __global__ void __launch_bounds__(128) merge_kernel(MergeLaunch p,
         W > 0.f ? (M + fast_log2(W)) * 0.69314718055994531f : -CUDART_INF_F;
 }
 
-template <int D, int NT>
+template <int D, int NT, bool KV8>
 cudaError_t launch_decode_t(const DecodeLaunch& p, const DecodeItemsInline* inl,
                             cudaStream_t stream) {
-  using Geo = DecodeGeom<D>;
+  using Geo = DecodeGeom<D, KV8>;
   // 4-D box over the pool: (dims, kv head, slot, page); head-major pools use one "head".
   CUtensorMap kmap, vmap;
   cudaError_t e = encode_kv_map(&kmap, p.kv.k_pool, p.kv, D, kDecodeStageKeys);
   if (e != cudaSuccess) return e;
   e = encode_kv_map(&vmap, p.kv.v_pool, p.kv, D, kDecodeStageKeys);
   if (e != cudaSuccess) return e;
-  auto kern = decode_split_kernel<D, NT>;
+  auto kern = decode_split_kernel<D, NT, KV8>;
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), Geo::kAlloc);
   if (e != cudaSuccess) return e;
   dim3 grid(p.num_items, p.num_kv_heads);
@@ -457,14 +547,20 @@ cudaError_t launch_decode_t(const DecodeLaunch& p, const DecodeItemsInline* inl,
 cudaError_t launch_decode(const DecodeLaunch& p, const DecodeItemsInline* inl, int nt,
                           cudaStream_t stream) {
   if (p.num_items <= 0) return cudaSuccess;
-  if (p.head_dim == 128) {
-    if (nt == 1) return launch_decode_t<128, 1>(p, inl, stream);
-    if (nt == 2) return launch_decode_t<128, 2>(p, inl, stream);
-    return launch_decode_t<128, 4>(p, inl, stream);
+  if (p.kv.kv8) {
+    if (p.head_dim != 128) return cudaErrorInvalidValue;
+    if (nt == 1) return launch_decode_t<128, 1, true>(p, inl, stream);
+    if (nt == 2) return launch_decode_t<128, 2, true>(p, inl, stream);
+    return launch_decode_t<128, 4, true>(p, inl, stream);
   }
-  if (nt == 1) return launch_decode_t<64, 1>(p, inl, stream);
-  if (nt == 2) return launch_decode_t<64, 2>(p, inl, stream);
-  return launch_decode_t<64, 4>(p, inl, stream);
+  if (p.head_dim == 128) {
+    if (nt == 1) return launch_decode_t<128, 1, false>(p, inl, stream);
+    if (nt == 2) return launch_decode_t<128, 2, false>(p, inl, stream);
+    return launch_decode_t<128, 4, false>(p, inl, stream);
+  }
+  if (nt == 1) return launch_decode_t<64, 1, false>(p, inl, stream);
+  if (nt == 2) return launch_decode_t<64, 2, false>(p, inl, stream);
+  return launch_decode_t<64, 4, false>(p, inl, stream);
 }
 
 cudaError_t launch_merge(const MergeLaunch& p, const MergeRowsInline* inl, cudaStream_t stream) {

@@ -46,14 +46,17 @@ cudaError_t encode_kv_map(CUtensorMap* map, const void* pool, const PagedKV& kv,
     return cudaErrorNotSupported;
   }
   const uint64_t heads = kv.layout == 0 ? (uint64_t)kv.num_kv_heads : 1ull;
+  // bf16 pools: boxes of 64 elements (128 bytes); e4m3 pools: 128 one-byte codes
+  const uint64_t eb = kv.kv8 ? 1 : 2;
   cuuint64_t dims[4] = {(cuuint64_t)head_dim, heads, (cuuint64_t)kv.page_size,
                         (cuuint64_t)kv.num_pages};
-  cuuint64_t strides[3] = {(cuuint64_t)head_dim * 2, (cuuint64_t)heads * head_dim * 2,
-                           (cuuint64_t)kv.page_size * heads * head_dim * 2};
+  cuuint64_t strides[3] = {(cuuint64_t)head_dim * eb, (cuuint64_t)heads * head_dim * eb,
+                           (cuuint64_t)kv.page_size * heads * head_dim * eb};
   const int rows = kv.page_size < box_keys ? kv.page_size : box_keys;
-  cuuint32_t box[4] = {64, 1, (cuuint32_t)rows, 1};
+  cuuint32_t box[4] = {(cuuint32_t)(128 / eb), 1, (cuuint32_t)rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
-  CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(pool), dims,
+  CUresult r = enc(map, kv.kv8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
+                   4, const_cast<void*>(pool), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                    CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);

@@ -569,13 +569,15 @@ rpa_status rpa_rotary_write_kv(rpa_plan_t plan, const void* q, const void* k, co
                     "rotary write launch");
 }
 
-rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const void* v_new,
-                       void* k_pool, void* v_pool, const int32_t* block_table,
-                       const int32_t* cu_seqlens_q, const int32_t* seq_lens_k,
-                       const int32_t* group_table, const int32_t* group_count, float scale,
-                       void* out, float* lse, void* workspace, size_t workspace_bytes,
-                       void* stream_) {
-  g_last_error.clear();
+// The fused step for bf16 pools (rpa_forward) and for e4m3 pools (rpa_forward_kv8, kv8 =
+// true, with per-KV-head scales; decode-class plans only, checked by the caller).
+static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new,
+                               const void* v_new, void* k_pool, void* v_pool,
+                               const int32_t* block_table, const int32_t* cu_seqlens_q,
+                               const int32_t* seq_lens_k, const int32_t* group_table,
+                               const int32_t* group_count, float scale, void* out, float* lse,
+                               void* workspace, size_t workspace_bytes, void* stream_,
+                               bool kv8, const float* k_scale, const float* v_scale) {
   rpa_status st = check_common(plan, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k);
   if (st != RPA_OK) return st;
   const rpa_shape& s = plan->shape;
@@ -602,6 +604,8 @@ rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const 
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     RPA_FAIL(RPA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
 
+  if (kv8 && k_new && !plan->fuse_write)
+    RPA_FAIL(RPA_ERR_UNSUPPORTED, "e4m3 pools: the KV write runs inside the decode kernel");
   if (k_new && !plan->fuse_write) {
     st = write_kv_impl(plan, k_new, v_new, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k,
                        stream);
@@ -628,6 +632,7 @@ rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const 
   kv.max_blocks = s.max_blocks_per_seq;
   kv.num_kv_heads = s.num_kv_heads;
   kv.num_pages = s.num_pages;
+  kv.kv8 = kv8 ? 1 : 0;
   const float scale_log2 = scale * 1.4426950408889634f;
 
   if (plan->device_mode) {
@@ -790,8 +795,10 @@ rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const 
     const bool fused = k_new && plan->fuse_write;
     d.k_new = fused ? static_cast<const uint16_t*>(k_new) : nullptr;
     d.v_new = fused ? static_cast<const uint16_t*>(v_new) : nullptr;
-    d.k_pool_w = fused ? static_cast<uint16_t*>(k_pool) : nullptr;
-    d.v_pool_w = fused ? static_cast<uint16_t*>(v_pool) : nullptr;
+    d.k_pool_w = fused ? k_pool : nullptr;
+    d.v_pool_w = fused ? v_pool : nullptr;
+    d.k_scale = k_scale;
+    d.v_scale = v_scale;
     st = check_cuda(launch_decode(d, &plan->dec_inline, plan->decode_nt, stream), "decode launch");
     if (st != RPA_OK) return st;
     if (!plan->merge_rows.empty()) {
@@ -817,6 +824,43 @@ rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const 
     if (st != RPA_OK) return st;
   }
   return RPA_OK;
+}
+
+rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const void* v_new,
+                       void* k_pool, void* v_pool, const int32_t* block_table,
+                       const int32_t* cu_seqlens_q, const int32_t* seq_lens_k,
+                       const int32_t* group_table, const int32_t* group_count, float scale,
+                       void* out, float* lse, void* workspace, size_t workspace_bytes,
+                       void* stream) {
+  g_last_error.clear();
+  return forward_impl(plan, q, k_new, v_new, k_pool, v_pool, block_table, cu_seqlens_q,
+                      seq_lens_k, group_table, group_count, scale, out, lse, workspace,
+                      workspace_bytes, stream, false, nullptr, nullptr);
+}
+
+rpa_status rpa_forward_kv8(rpa_plan_t plan, const void* q, const void* k_new, const void* v_new,
+                           void* k_pool, void* v_pool, const float* k_scale,
+                           const float* v_scale, const int32_t* block_table,
+                           const int32_t* cu_seqlens_q, const int32_t* seq_lens_k, float scale,
+                           void* out, float* lse, void* workspace, size_t workspace_bytes,
+                           void* stream) {
+  g_last_error.clear();
+  if (!plan) RPA_FAIL(RPA_ERR_INVALID_ARG, "plan is NULL");
+  if (plan->shape.head_dim != 128)
+    RPA_FAIL(RPA_ERR_UNSUPPORTED, "e4m3 pools need head_dim 128 (got %d)",
+             plan->shape.head_dim);
+  if (plan->device_mode)
+    RPA_FAIL(RPA_ERR_UNSUPPORTED, "e4m3 pools: device-planned steps are not supported");
+  if (!plan->pf_tiles.empty())
+    RPA_FAIL(RPA_ERR_UNSUPPORTED,
+             "e4m3 pools: only decode-class batches (every row on the split-KV decode kernel)");
+  if (plan->opts.sparse) RPA_FAIL(RPA_ERR_UNSUPPORTED, "e4m3 pools: no group tables");
+  if (!k_scale || !v_scale) RPA_FAIL(RPA_ERR_INVALID_ARG, "k_scale and v_scale are required");
+  if ((reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u))
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "k_scale / v_scale must be 4-byte aligned");
+  return forward_impl(plan, q, k_new, v_new, k_pool, v_pool, block_table, cu_seqlens_q,
+                      seq_lens_k, nullptr, nullptr, scale, out, lse, workspace, workspace_bytes,
+                      stream, true, k_scale, v_scale);
 }
 
 rpa_status rpa_build_group_tables(const uint8_t* mask, int32_t num_seqs, int32_t num_q_heads,

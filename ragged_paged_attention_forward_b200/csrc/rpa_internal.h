@@ -84,6 +84,7 @@ struct PagedKV {
   int32_t max_blocks;
   int32_t num_kv_heads;
   int32_t num_pages;
+  int32_t kv8;             // 1: the pools hold e4m3 codes (one byte per element)
 };
 
 struct DecodeLaunch {
@@ -107,8 +108,12 @@ struct DecodeLaunch {
   // new tokens whose positions fall in its key range, for its KV head.  Null: no write.
   const uint16_t* k_new;     // bf16 [T, Hkv, D]
   const uint16_t* v_new;
-  uint16_t* k_pool_w;
-  uint16_t* v_pool_w;
+  void* k_pool_w;            // bf16 pools, or e4m3 code pools when kv.kv8
+  void* v_pool_w;
+  // e4m3 pools (kv.kv8): element = code * scale[kv head]; new tokens are stored as
+  // e4m3(fp32(x) / scale), nearest even, saturating
+  const float* k_scale;      // [Hkv]
+  const float* v_scale;      // [Hkv]
 };
 
 struct MergeLaunch {

@@ -18,6 +18,13 @@ Input recipe (the same for every consumer):
   * block-table entries past a sequence's last page point at an unused (NaN) page, so a
     kernel that reads past the end produces NaN instead of plausible numbers.
 
+e4m3 (fp8) pools (``with_kv8_pools``): the same batch with its context rows replaced by
+random finite e4m3 codes (sign uniform, exponent field uniform in 3..11, mantissa uniform:
+magnitudes 2^-4 .. 2^4 * 1.875), every other slot holding the NaN code 0x7F for correctness
+runs (0 for timing runs), and per-KV-head fp32 scales drawn uniform in [0.005, 0.02] for K
+and [0.05, 0.2] for V (so bf16 N(0,1) new tokens land across the code range, the largest
+ones saturating).
+
 Layouts (the two page layouts of the CompactAttention page, Fig. 4):
   * sequence-major: pool ``[num_pages, page_size, Hkv, D]``, block_table ``[B, max_blocks]``;
   * KV-head-major: pool ``[num_pages, page_size, D]``, block_table ``[B, Hkv, max_blocks]``.
@@ -331,3 +338,49 @@ WORKLOADS = {
     "mixed": mixed,
     "sparse": sparse,
 }
+
+
+E4M3_NAN_CODE = 0x7F
+
+
+def with_kv8_pools(batch: Batch, *, seed: int, poison: bool = True):
+    """The batch with uint8 e4m3 code pools instead of bf16 ones, plus scales.
+
+    Returns ``(batch8, k_scale [Hkv] fp32, v_scale [Hkv] fp32)``.  Context positions
+    ``0 .. past-1`` of every sequence get random finite codes; all other slots get the NaN
+    code (or 0).  ``k_new``/``v_new`` stay bf16 (they are quantised by the step itself).
+    """
+    g = torch.Generator().manual_seed(int(seed))
+    fill = E4M3_NAN_CODE if poison else 0
+    kp = torch.full(batch.k_pool.shape, fill, dtype=torch.uint8)
+    vp = torch.full(batch.v_pool.shape, fill, dtype=torch.uint8)
+    Hkv, D, P = batch.num_kv_heads, batch.head_dim, batch.page_size
+
+    def draw(n):
+        sign = torch.randint(0, 2, (n, Hkv, D), generator=g, dtype=torch.int32)
+        expo = torch.randint(3, 12, (n, Hkv, D), generator=g, dtype=torch.int32)
+        mant = torch.randint(0, 8, (n, Hkv, D), generator=g, dtype=torch.int32)
+        return ((sign << 7) | (expo << 3) | mant).to(torch.uint8)
+
+    bt = batch.block_table.to(torch.int64)
+    for b, (kv, ql) in enumerate(zip(batch.kv_lens(), batch.q_lens())):
+        past = kv - ql
+        if past <= 0:
+            continue
+        kc, vc = draw(past), draw(past)
+        pos = torch.arange(past)
+        sl = pos % P
+        if batch.layout == SEQ_MAJOR:
+            pg = bt[b][pos // P]
+            kp[pg, sl] = kc
+            vp[pg, sl] = vc
+        else:
+            for h in range(Hkv):
+                pg = bt[b, h][pos // P]
+                kp[pg, sl] = kc[:, h]
+                vp[pg, sl] = vc[:, h]
+    k_scale = (0.005 + 0.015 * torch.rand(Hkv, generator=g)).to(torch.float32)
+    v_scale = (0.05 + 0.15 * torch.rand(Hkv, generator=g)).to(torch.float32)
+    out = dataclasses.replace(batch, k_pool=kp, v_pool=vp, k_logical=None, v_logical=None,
+                              name=(batch.name + "-kv8") if batch.name else "kv8")
+    return out, k_scale, v_scale

@@ -225,3 +225,21 @@ def test_device_plan_rejects(kw, status):
     with pytest.raises(api.RPAError) as e:
         _device_plan(**kw)
     assert e.value.status == status
+
+
+def test_forward_kv8_rejects_before_any_device_work():
+    # decode-only plan, head_dim 128: missing scales are an argument error
+    plan = api.rpa_plan(**_shape())
+    with pytest.raises(api.RPAError) as ei:
+        api.rpa_forward_kv8(plan, None, None, None, None, None, None, None, None, None, None,
+                            0.1, None, None, None, stream=0)
+    assert ei.value.status == api.RPA_ERR_INVALID_ARG
+    # a plan with a prefill row, a head_dim-64 plan and a sparse plan are unsupported
+    for kw in (dict(cu_seqlens_q=[0, 1, 200], num_tokens=200, seq_lens_k=[40, 200]),
+               dict(head_dim=64),
+               dict(layout=1, sparse=True)):
+        plan = api.rpa_plan(**_shape(**kw))
+        with pytest.raises(api.RPAError) as ei:
+            api.rpa_forward_kv8(plan, None, None, None, None, None, None, None, None, None,
+                                None, 0.1, None, None, None, stream=0)
+        assert ei.value.status == api.RPA_ERR_UNSUPPORTED, kw

@@ -487,3 +487,125 @@ def test_rotary_write_uses_past_plus_index_and_packed_columns():
     kref, _ = orc.write_kv(b.k_pool, b.v_pool, b.k_new, b.v_new, b.block_table,
                            b.cu_seqlens_q, b.seq_lens_k, P, b.layout)
     assert np.array_equal(q3, orc.bits16(b.q)) and np.array_equal(kp3, kref)
+
+
+# --------------------------------------------------------------------------------------
+# fp8 (e4m3) KV cache: the codec is pinned to the library's float8_e4m3fn conversions and to
+# hand-derived values; the dequantised attention is pinned to the (already pinned) bf16
+# oracle on values that both formats represent exactly.
+# --------------------------------------------------------------------------------------
+
+def test_e4m3_decode_matches_library_table():
+    codes = np.arange(256, dtype=np.uint8)
+    got = orc.e4m3_decode(codes)
+    ref = torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    assert np.array_equal(np.isnan(got), np.isnan(ref))
+    ok = ~np.isnan(ref)
+    assert np.array_equal(got[ok], ref[ok])
+    assert np.isnan(got[0x7F]) and np.isnan(got[0xFF]) and np.isnan(got).sum() == 2
+    assert got[0x7E] == 448.0 and got[0x01] == 2.0 ** -9 and got[0x38] == 1.0
+
+
+def test_e4m3_encode_nearest_even_matches_library():
+    rng = np.random.default_rng(71)
+    vals = orc.e4m3_decode(np.arange(0x7F, dtype=np.uint8))
+    mids = (vals[1:] + vals[:-1]) / 2             # exact ties (representable in fp32)
+    x = np.concatenate([rng.uniform(-447.9, 447.9, 50000), rng.normal(0, 0.05, 20000),
+                        vals, -vals, mids, -mids]).astype(np.float32)
+    got = orc.e4m3_encode(x.astype(np.float64))
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("x,code", [
+    (1.0, 0x38), (-1.0, 0xB8), (448.0, 0x7E), (500.0, 0x7E), (1e30, 0x7E), (-1e9, 0xFE),
+    (2.0 ** -9, 0x01), (2.0 ** -10, 0x00), (1.5 * 2.0 ** -10, 0x01), (0.0, 0x00), (-0.0, 0x80),
+    (1.0625, 0x38), (1.1875, 0x3A), (2.0 ** -6, 0x08), (7 * 2.0 ** -9, 0x07),
+    (7.5 * 2.0 ** -9, 0x08), (float("nan"), 0x7F)])
+def test_e4m3_encode_hand_values(x, code):
+    # 1.0625 lies halfway between 1.0 (mantissa 000) and 1.125 (001): ties go to the even
+    # mantissa; 1.1875 between 1.125 (001) and 1.25 (010) goes up; 2^-10 is half the
+    # smallest subnormal and rounds to the even code 0; past 448 the code saturates.
+    assert int(orc.e4m3_encode(np.array([x]))[0]) == code
+
+
+def test_e4m3_round_trip_and_error_bound():
+    codes = np.array([c for c in range(256) if c not in (0x7F, 0xFF)], dtype=np.uint8)
+    v = orc.e4m3_decode(codes)
+    back = orc.e4m3_encode(v)
+    assert np.array_equal(orc.e4m3_decode(back), v)       # -0 and +0 both decode to 0
+    rng = np.random.default_rng(72)
+    x = rng.uniform(-440, 440, 20000)
+    err = np.abs(orc.e4m3_decode(orc.e4m3_encode(x)) - x)
+    # half a unit in the last place: 2^-4 relative for normals, 2^-10 absolute below 2^-6
+    assert np.all(err <= np.maximum(np.abs(x) * 2.0 ** -4, 2.0 ** -10) * (1 + 1e-12))
+
+
+def test_e4m3_quantize_divides_in_fp32_first():
+    # 1.0 / 3.0 in fp32 is 0.3333333432674408; e4m3 neighbours 0.3125 and 0.34375
+    bits = np.array([0x3F80], dtype=np.uint16)              # bf16 1.0
+    code = orc.e4m3_quantize(bits, 3.0)
+    assert orc.e4m3_decode(code)[0] == 0.34375
+    # saturation: 2.0 / 2^-9 = 1024 -> 448
+    assert int(orc.e4m3_quantize(bits * 0 + 0x4000, 2.0 ** -9)[0]) == 0x7E
+
+
+@pytest.mark.parametrize("layout", [orc.SEQ_MAJOR, orc.HEAD_MAJOR])
+def test_kv8_attention_equals_bf16_attention_on_shared_values(layout):
+    b = wl.ragged_batch([70, 33, 129], [1, 3, 2], 8, 2, 128, 16, seed=81)
+    if layout == orc.HEAD_MAJOR:
+        b = wl.to_head_major(b)
+    b8, _, _ = wl.with_kv8_pools(b, seed=82)
+    # power-of-two scales keep code * scale exact in bf16: the e4m3 path must then give the
+    # bf16 oracle's numbers on the same values, bit for bit
+    ks = np.array([2.0 ** -5, 2.0 ** -3], dtype=np.float32)
+    vs = np.array([2.0 ** -2, 2.0 ** 1], dtype=np.float32)
+    kp8, vp8 = orc.codes8(b8.k_pool), orc.codes8(b8.v_pool)
+    Hkv = 2
+
+    def to_bf16(codes, scales):
+        c = codes.copy()
+        head_axis = 2 if layout == orc.SEQ_MAJOR else None
+        v = orc.e4m3_decode(c)
+        if head_axis is not None:
+            v = v * scales.reshape(1, 1, Hkv, 1)
+        else:  # head-major: page p belongs to one head; find it from the block table
+            heads = np.zeros(c.shape[0], dtype=np.int64)
+            bt = orc.ints(b8.block_table)
+            for h in range(Hkv):
+                heads[bt[:, h, :].reshape(-1)] = h
+            v = v * scales[heads].reshape(-1, 1, 1)
+        v = np.where(np.isnan(v), 0.0, v)
+        return orc.round_bf16(v)
+
+    # the step writes the new tokens (quantised) first; both sides then read the same
+    # context and new-token values
+    got_o, got_l, kpa, vpa = orc.forward_kv8(b8.q, b8.k_new, b8.v_new, kp8, vp8, ks, vs,
+                                             b8.block_table, b8.cu_seqlens_q, b8.seq_lens_k,
+                                             scale=b8.scale, causal=True, page_size=16,
+                                             layout=layout)
+    kb, vb = to_bf16(kpa, ks), to_bf16(vpa, vs)
+    ref_o, ref_l = orc.attention(b8.q, kb, vb, b8.block_table, b8.cu_seqlens_q, b8.seq_lens_k,
+                                 scale=b8.scale, causal=True, page_size=16, layout=layout,
+                                 num_kv_heads=Hkv)
+    assert np.all(np.isfinite(got_o))
+    assert np.array_equal(got_o, ref_o) and np.array_equal(got_l, ref_l)
+
+
+def test_write_kv8_places_quantised_codes_in_hand_derived_slots():
+    b = wl.ragged_batch([5, 19], [2, 3], 4, 2, 128, 16, seed=83)
+    b8, ks, vs = wl.with_kv8_pools(b, seed=84)
+    kp, vp = orc.write_kv8(b8.k_pool, b8.v_pool, b8.k_new, b8.v_new, ks.numpy(), vs.numpy(),
+                           b8.block_table, b8.cu_seqlens_q, b8.seq_lens_k, 16)
+    bt = orc.ints(b8.block_table)
+    # sequence 1: kv 19, q 3 -> positions 16, 17, 18 -> block 1, slots 0, 1, 2; tokens 2..4
+    for i, pos in enumerate((16, 17, 18)):
+        for h in range(2):
+            want = orc.e4m3_quantize(orc.bits16(b8.k_new)[2 + i, h], float(ks[h]))
+            assert np.array_equal(kp[bt[1, 1], pos % 16, h], want)
+    # untouched slots keep their codes
+    before = orc.codes8(b8.k_pool)
+    mask = np.ones(before.shape[:2], dtype=bool)
+    for (b_, pos) in [(0, 3), (0, 4), (1, 16), (1, 17), (1, 18)]:
+        mask[bt[b_, pos // 16], pos % 16] = False
+    assert np.array_equal(kp[mask], before[mask])
