@@ -547,6 +547,53 @@ def measure_device_planned_decode(steps, warmup, peaks):
     return res
 
 
+def measure_decode_kv8(steps, warmup, peaks):
+    """The decode step over an e4m3 (fp8) KV cache (rpa_forward_kv8): the same 64 sequences
+    as the headline, the context as random finite e4m3 codes with per-KV-head scales, the
+    new tokens quantised by the step's fused write.  HBM-bound: algorithmic bytes = K and V
+    codes read once (1 byte per element) + Q read and O written (bf16) + the new tokens read
+    (bf16) and written (codes).  Timed back to back over rotating pool copies."""
+    from ragged_paged_attention_forward_b200 import api
+    from ragged_paged_attention_forward_b200 import workloads as wl
+    b, _ = make_workload("decode")
+    b8, ks, vs = wl.with_kv8_pools(b, seed=1234, poison=False)
+    d = {k: getattr(b8, k).cuda().contiguous() for k in (
+        "q", "k_new", "v_new", "k_pool", "v_pool", "block_table", "cu_seqlens_q", "seq_lens_k")}
+    ks, vs = ks.cuda(), vs.cuda()
+    pool_bytes = 2 * d["k_pool"].numel()
+    n = max(3, -(-2 * L2_BYTES // pool_bytes) + 1)
+    pools = [(d["k_pool"], d["v_pool"])] + [(d["k_pool"].clone(), d["v_pool"].clone())
+                                            for _ in range(n - 1)]
+    plan = api.rpa_plan(num_seqs=b8.num_seqs, num_tokens=b8.num_tokens,
+                        num_q_heads=b8.num_q_heads, num_kv_heads=b8.num_kv_heads,
+                        head_dim=b8.head_dim, page_size=b8.page_size, num_pages=b8.num_pages,
+                        max_blocks_per_seq=b8.max_blocks, layout=b8.layout, causal=b8.causal,
+                        cu_seqlens_q=b8.cu_seqlens_q, seq_lens_k=b8.seq_lens_k)
+    ws = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(d["q"])
+
+    def step(i):
+        kp, vp = pools[i % len(pools)]
+        api.rpa_forward_kv8(plan, d["q"], d["k_new"], d["v_new"], kp, vp, ks, vs,
+                            d["block_table"], d["cu_seqlens_q"], d["seq_lens_k"], b8.scale, out,
+                            None, ws)
+
+    ms = timed_loop(step, steps, warmup)
+    T, Hq, D = b8.q.shape
+    Hkv = b8.num_kv_heads
+    kv_read = float(sum(b8.kv_lens())) * Hkv * D * 2
+    q_o = 2.0 * T * Hq * D * 2
+    new_kv = 2.0 * T * Hkv * D * (2 + 1)
+    step_bytes = kv_read + q_o + new_kv
+    gbps = step_bytes / (ms * 1e-3) / 1e9
+    info = plan.info()
+    return {"workload": WORKLOAD_TEXT["decode"] + "; K/V cache as e4m3 codes with per-KV-head "
+            "fp32 scales (random finite codes), new tokens quantised in the fused write",
+            "ms_per_step": ms, "step_GBps": gbps, "frac_of_hbm": gbps / peaks["hbm_gbs"],
+            "step_bytes": step_bytes, "tokens_per_s": T / (ms * 1e-3),
+            "launches_per_step": info.launches_forward, "l2": f"{n} pool copies rotate"}
+
+
 def measure_input_pass(steps, warmup, peaks):
     """The input pass with rotary embedding (rpa_rotary_write_kv) on the prefill workload's
     16384 new tokens: packed QKV in, RoPE over all 128 dims (split pairs), Q out, K/V
@@ -788,6 +835,7 @@ def run_gpu(args):
             del r2, b2
             torch.cuda.empty_cache()
         secondary["input_pass"] = measure_input_pass(args.steps, args.warmup, peaks)
+        secondary["decode_kv8"] = measure_decode_kv8(args.steps, args.warmup, peaks)
         secondary["decode_device_planned"] = measure_device_planned_decode(args.steps,
                                                                            args.warmup, peaks)
         line["secondary"] = secondary

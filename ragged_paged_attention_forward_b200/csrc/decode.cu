@@ -35,14 +35,16 @@ constexpr int kConsumerWarps = 4;
 constexpr int kDecodeThreads = (kConsumerWarps + 1) * 32;
 constexpr int kMaxItemPages = kMaxSplitKeys / 16 + 1;
 
-template <int D, bool KV8>
+template <int D, bool KV8, int NT>
 struct DecodeGeom {
   // stage rows are stored in 128-byte halves: 64 bf16 elements, or all 128 e4m3 codes
   static constexpr int kHalves = KV8 ? 1 : D / 64;
   static constexpr int kStageKeys = kDecodeStageKeys;                 // 64
   static constexpr int kHalfBytes = kStageKeys * 128;                 // 8 KB per half-row tile
   static constexpr int kTensorStageBytes = kHalves * kHalfBytes;      // K (or V) per stage
-  static constexpr int kStages = KV8 ? 6 : D == 128 ? 3 : 4;          // ~96 KB in flight
+  // bf16: ~96 KB in flight per CTA, two CTAs per SM; e4m3: 64 KB, three CTAs per SM (more
+  // warps to hide the in-register conversions), six stages when the combine needs room
+  static constexpr int kStages = KV8 ? (NT == 4 ? 6 : 4) : D == 128 ? 3 : 4;
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kStages * kTensorStageBytes;
   static constexpr int kPagesOff = 2 * kStages * kTensorStageBytes;
@@ -56,7 +58,8 @@ struct DecodeGeom {
   static_assert(kBarOff % 8 == 0, "mbarrier alignment");
   static_assert(!KV8 || D == 128, "e4m3 pools: head_dim 128");
   // the four warps' states are combined in the stage ring once it is drained
-  static_assert(2 * kConsumerWarps * 32 * 4 + kConsumerWarps * 32 * (D + 4) * 4 <= kPagesOff,
+  static_assert(2 * kConsumerWarps * 8 * NT * 4 + kConsumerWarps * 8 * NT * (D + 4) * 4 <=
+                    kPagesOff,
                 "combine area");
 };
 
@@ -69,7 +72,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap kmap,
                         const __grid_constant__ CUtensorMap vmap, DecodeLaunch p,
                         const __grid_constant__ DecodeItemsInline inl) {
-  using Geo = DecodeGeom<D, KV8>;
+  using Geo = DecodeGeom<D, KV8, NT>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -527,7 +530,7 @@ __global__ void __launch_bounds__(128) merge_kernel(MergeLaunch p,
 template <int D, int NT, bool KV8>
 cudaError_t launch_decode_t(const DecodeLaunch& p, const DecodeItemsInline* inl,
                             cudaStream_t stream) {
-  using Geo = DecodeGeom<D, KV8>;
+  using Geo = DecodeGeom<D, KV8, NT>;
   // 4-D box over the pool: (dims, kv head, slot, page); head-major pools use one "head".
   CUtensorMap kmap, vmap;
   cudaError_t e = encode_kv_map(&kmap, p.kv.k_pool, p.kv, D, kDecodeStageKeys);
