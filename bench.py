@@ -594,6 +594,79 @@ def measure_decode_kv8(steps, warmup, peaks):
             "launches_per_step": info.launches_forward, "l2": f"{n} pool copies rotate"}
 
 
+def measure_sparse_ablation(steps, warmup, peaks):
+    """Execution-only ablation on the sparse workload (CompactAttention, Fig. 7c): the same
+    unioned block mask run (A) through per-group tables -- a pair of query heads per CTA
+    sharing every K/V tile -- and (B) block-sparse per query tile and head -- tables built per
+    (128-query tile, query head) from the unioned mask written back per head and query block,
+    one head per CTA.  Both compute the same attention (bit for bit); only the execution
+    differs.  Attention only (tables built once, new tokens already in the pool), back to back
+    over rotating pool copies.  (C), for context: block-sparse on the original per-head mask,
+    which selects fewer blocks per row and is a different attention."""
+    from ragged_paged_attention_forward_b200 import api
+    b, mask = make_workload("sparse")
+    runner = Runner("sparse", b, mask)
+    d = runner.d
+    for i in range(len(runner.pools)):  # new tokens into every pool copy
+        runner.step(True, i=i)
+    runner.tables()
+    torch.cuda.synchronize()
+    B, Hq, nqb, nkb = mask.shape
+    Hkv = b.num_kv_heads
+    G = Hq // Hkv
+    qbr = b.num_tokens // nqb  # query rows per mask block (one sequence)
+    # the unioned mask written back per (head, query block)
+    sel = torch.zeros(B, Hkv, nkb + 1, dtype=torch.uint8, device="cuda")
+    idx = torch.where(runner.table >= 0, runner.table, torch.full_like(runner.table, nkb))
+    sel.scatter_(2, idx.long(), 1)
+    union = sel[:, :, :nkb].repeat_interleave(G, dim=1).unsqueeze(2).expand(
+        B, Hq, nqb, nkb).contiguous()
+    nt = -(-nqb // (128 // qbr))
+
+    def qtiles(m):
+        t = torch.empty(B, Hq, nt, nkb, dtype=torch.int32, device="cuda")
+        c = torch.empty(B, Hq, nt, dtype=torch.int32, device="cuda")
+        api.rpa_build_qtile_tables(m, qbr, t, c)
+        return t, c
+
+    tq_u, cq_u = qtiles(union)
+    tq_m, cq_m = qtiles(runner.mask_d)
+    plan_q = api.rpa_plan(num_seqs=b.num_seqs, num_tokens=b.num_tokens,
+                          num_q_heads=b.num_q_heads, num_kv_heads=Hkv, head_dim=b.head_dim,
+                          page_size=b.page_size, num_pages=b.num_pages,
+                          max_blocks_per_seq=b.max_blocks, layout=b.layout, causal=b.causal,
+                          cu_seqlens_q=b.cu_seqlens_q, seq_lens_k=b.seq_lens_k, sparse=2)
+    ws_q = torch.empty(max(plan_q.workspace_bytes, 256), dtype=torch.uint8, device="cuda")
+
+    def attend(plan, ws, t, c):
+        def f(i):
+            kp, vp = runner.pools[i % len(runner.pools)]
+            api.rpa_forward(plan, d["q"], None, None, kp, vp, d["block_table"],
+                            d["cu_seqlens_q"], d["seq_lens_k"], t, c, b.scale, runner.out,
+                            None, ws)
+        return f
+
+    ms_a = timed_loop(attend(runner.plan, runner.ws, runner.table, runner.count), steps, warmup)
+    ms_b = timed_loop(attend(plan_q, ws_q, tq_u, cq_u), steps, warmup)
+    ms_c = timed_loop(attend(plan_q, ws_q, tq_m, cq_m), steps, warmup)
+    table, count = runner.host_tables()
+    w = work(b, table, count)
+    # K/V bytes the CTAs ask for (from L2 or HBM), before the causal cut: every query tile
+    # reads each group's table once per CTA of the group -- G/2 CTAs in (A), G in (B)
+    kv_tile = float(np.asarray(count).sum()) * b.page_size * b.head_dim * 4
+    tiles = -(-b.num_tokens // 128)
+    res = {"workload": "sparse workload, same unioned mask: (A) per-group tables, 2 query heads "
+                       "per CTA; (B) per-(query tile, query head) tables, 1 head per CTA; (C) "
+                       "per-(query tile, query head) tables of the original per-head mask",
+           "union_ms": ms_a, "blocksparse_ms": ms_b, "blocksparse_own_mask_ms": ms_c,
+           "union_TFLOPs": w["flops"] / (ms_a * 1e-3) / 1e12,
+           "blocksparse_TFLOPs": w["flops"] / (ms_b * 1e-3) / 1e12,
+           "union_speedup_over_blocksparse": ms_b / ms_a,
+           "kv_tile_bytes_union": kv_tile * tiles * (G // 2),
+           "kv_tile_bytes_blocksparse": kv_tile * tiles * G}
+    return res
+
+
 def measure_input_pass(steps, warmup, peaks):
     """The input pass with rotary embedding (rpa_rotary_write_kv) on the prefill workload's
     16384 new tokens: packed QKV in, RoPE over all 128 dims (split pairs), Q out, K/V
@@ -836,6 +909,7 @@ def run_gpu(args):
             torch.cuda.empty_cache()
         secondary["input_pass"] = measure_input_pass(args.steps, args.warmup, peaks)
         secondary["decode_kv8"] = measure_decode_kv8(args.steps, args.warmup, peaks)
+        secondary["sparse_ablation"] = measure_sparse_ablation(args.steps, args.warmup, peaks)
         secondary["decode_device_planned"] = measure_device_planned_decode(args.steps,
                                                                            args.warmup, peaks)
         line["secondary"] = secondary

@@ -85,7 +85,8 @@ typedef struct rpa_shape {
 typedef struct rpa_plan_options {
   int32_t force_class;         /* rpa_batch_class; AUTO lets the planner choose            */
   int32_t decode_split_keys;   /* keys per decode split, multiple of 64; 0 = automatic     */
-  int32_t sparse;              /* 1: rpa_forward will be given group tables                */
+  int32_t sparse;              /* 1: rpa_forward will be given group tables; 2: per-(query  */
+                               /* tile, query head) tables (rpa_build_qtile_tables)         */
   int32_t reserved[5];         /* must be zero                                             */
 } rpa_plan_options;
 
@@ -243,7 +244,9 @@ RPA_API rpa_status rpa_rotary_write_kv(rpa_plan_t plan, const void* q, const voi
  *   block_table, cu_seqlens_q, seq_lens_k   as for rpa_write_kv.
  *   group_table       device int32 [B, Hkv, max_blocks_per_seq] of ascending logical
  *                     block indices (rpa_build_group_tables output), or NULL; requires
- *                     RPA_LAYOUT_HEAD_MAJOR and a plan made with opts.sparse = 1.
+ *                     RPA_LAYOUT_HEAD_MAJOR and a plan made with opts.sparse = 1; or, with
+ *                     opts.sparse = 2, rpa_build_qtile_tables' per-(query tile, query head)
+ *                     tables.
  *   group_count       device int32 [B, Hkv] valid entries per table row, or NULL.
  *   scale             softmax scale (typically 1/sqrt(D)); any finite value.
  *   out               device bf16 [T, Hq, D] (round-to-nearest-even).
@@ -342,6 +345,27 @@ RPA_API rpa_status rpa_build_group_tables(const uint8_t* mask, int32_t num_seqs,
  * [0, num_pages) or a block index outside the table, 8 a position at or past the rotary
  * caches' max_position, 16 a device-planned step beyond its plan's limits.
  */
+/*
+ * rpa_build_qtile_tables -- per-(query tile, query head) KV block tables: row (b, hq, tile)
+ * lists, ascending, the KV blocks kb that head hq selects in any query block of the
+ * 128-query tile (query blocks tile * 128/q_block_rows ...); count[b, hq, tile] entries are
+ * valid, the rest are -1.  This is the execution of a block-sparse kernel that works per
+ * query block and head, for CompactAttention's execution-only ablation (Fig. 7c: the same
+ * unioned mask, run block-sparse per query block vs. through per-group tables).  Pass the
+ * tables to rpa_forward (as group_table / group_count) with a plan made with opts.sparse = 2:
+ * the tensor-core kernel then runs one query head per CTA, each reading its own table.
+ *
+ *   mask          device uint8 [B, Hq, nqb, nkb], nonzero = selected.
+ *   q_block_rows  query rows per mask block; must divide 128.
+ *   table         device int32 [B, Hq, ntiles, nkb], ntiles = ceil(nqb * q_block_rows / 128),
+ *                 which must equal ceil(max q_len / 128) of the plan; nkb = max_blocks_per_seq.
+ *   count         device int32 [B, Hq, ntiles].
+ */
+RPA_API rpa_status rpa_build_qtile_tables(const uint8_t* mask, int32_t num_seqs,
+                                          int32_t num_q_heads, int32_t num_q_blocks,
+                                          int32_t num_kv_blocks, int32_t q_block_rows,
+                                          int32_t* table, int32_t* count, void* stream);
+
 RPA_API rpa_status rpa_device_error(int32_t* code, int32_t clear);
 
 /* rpa_status_string -- static description of a status code. */

@@ -25,6 +25,12 @@ What it computes (plain definitions, written out; no tiling, no fusion, no reord
   WebGPU page, "What's shipped").
 * ``build_group_tables`` -- Q-block union, then intra-group union, then the ascending list
   of selected KV blocks per (sequence, KV group) (CompactAttention, Core claim; Fig. 3).
+* ``build_qtile_tables`` -- the per-(query tile, query head) lists of a block-sparse kernel
+  that works per query block and head (CompactAttention, Fig. 7c: the execution-only
+  ablation with the same unioned mask): row ``(b, hq, tile)`` lists, ascending, the KV blocks
+  head ``hq`` selects in any query block of the 128-row tile.  ``attention`` with
+  ``qtile_table`` lets row ``i`` of sequence ``b`` and head ``hq`` see only the blocks of
+  its tile ``i // 128``.
 * ``rotate`` / ``rotary_write_kv`` -- the input pass with rotary position embedding: Q and
   K rows rotated by their position ``past_b + s``, dims at or past ``rotary_dim`` unchanged,
   pairs interleaved ``(2j, 2j+1)`` or split ``(j, j + rotary_dim/2)``; a packed input holds
@@ -194,7 +200,8 @@ def attend_row(q: np.ndarray, K: np.ndarray, V: np.ndarray, scale: float):
 def attention(q, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k, *, scale: float,
               causal: bool, page_size: int, layout: int = SEQ_MAJOR, num_kv_heads: int,
               group_table=None, group_count=None,
-              rows: Optional[Iterable[Tuple[int, int]]] = None, kv_scales=None):
+              rows: Optional[Iterable[Tuple[int, int]]] = None, kv_scales=None,
+              qtile_table=None, qtile_count=None, tile_rows: int = 128):
     """Attention of every (token, query head) row -- or of ``rows`` only -- against the pools
     *as given* (call ``write_kv`` first for the fused semantics).  With ``kv_scales =
     (k_scale, v_scale)`` the pools hold e4m3 codes and key ``j`` of KV head ``h`` is
@@ -209,6 +216,8 @@ def attention(q, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k, *, scale
     seqs = seq_ranges(cu_seqlens_q, seq_lens_k)
     gt = ints(group_table) if group_table is not None else None
     gc = ints(group_count) if group_count is not None else None
+    qt = ints(qtile_table) if qtile_table is not None else None
+    qc = ints(qtile_count) if qtile_count is not None else None
 
     out = np.full((T, Hq, D), np.nan, dtype=np.float64)
     lse = np.full((T, Hq), np.nan, dtype=np.float64)
@@ -250,6 +259,10 @@ def attention(q, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k, *, scale
                 for hq in heads:
                     if wanted is not None and hq not in wanted[t]:
                         continue
+                    if qt is not None:   # this head's table for the row's query tile
+                        tau = (t - t0) // tile_rows
+                        sel = set(int(x) for x in qt[b, hq, tau, :int(qc[b, hq, tau])])
+                        idx = visible_keys(pos, kv_len, causal, page_size, sel)
                     o, l = attend_row(widen(qb[t, hq]), K[idx], V[idx], scale)
                     out[t, hq] = o
                     lse[t, hq] = l
@@ -258,7 +271,8 @@ def attention(q, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k, *, scale
 
 def forward(q, k_new, v_new, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k, *,
             scale: float, causal: bool, page_size: int, layout: int = SEQ_MAJOR,
-            group_table=None, group_count=None, rows=None):
+            group_table=None, group_count=None, rows=None, qtile_table=None,
+            qtile_count=None):
     """The fused step: write the new tokens' K/V into the pools, then attend.
 
     Returns ``(out, lse, k_pool_after, v_pool_after)``."""
@@ -268,7 +282,8 @@ def forward(q, k_new, v_new, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens
     out, lse = attention(q, kp, vp, block_table, cu_seqlens_q, seq_lens_k, scale=scale,
                          causal=causal, page_size=page_size, layout=layout,
                          num_kv_heads=num_kv_heads, group_table=group_table,
-                         group_count=group_count, rows=rows)
+                         group_count=group_count, rows=rows, qtile_table=qtile_table,
+                         qtile_count=qtile_count)
     return out, lse, kp, vp
 
 
@@ -323,6 +338,26 @@ def build_group_tables(mask, num_kv_heads: int):
             sel = [kb for kb in range(nkb) if group_union[b, g, kb]]
             table[b, g, :len(sel)] = sel
             count[b, g] = len(sel)
+    return table, count
+
+
+def build_qtile_tables(mask, q_block_rows: int, tile_rows: int = 128):
+    """Per (sequence, query head, query tile of ``tile_rows`` rows): the ascending KV blocks
+    selected by any of the tile's query blocks.  Returns ``(table [B, Hq, nt, nkb] int32,
+    -1 past the count; count [B, Hq, nt] int32)``."""
+    m = np.asarray(mask.cpu().numpy() if hasattr(mask, "cpu") else mask) != 0
+    B, Hq, nqb, nkb = m.shape
+    per = tile_rows // q_block_rows
+    nt = -(-nqb // per)
+    table = np.full((B, Hq, nt, nkb), -1, dtype=np.int32)
+    count = np.zeros((B, Hq, nt), dtype=np.int32)
+    for b in range(B):
+        for hq in range(Hq):
+            for tau in range(nt):
+                rows = m[b, hq, tau * per:(tau + 1) * per]
+                sel = [kb for kb in range(nkb) if rows[:, kb].any()]
+                table[b, hq, tau, :len(sel)] = sel
+                count[b, hq, tau] = len(sel)
     return table, count
 
 

@@ -104,6 +104,9 @@ def lib() -> ctypes.CDLL:
         L.rpa_build_group_tables.argtypes = [_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                              ctypes.c_int32, ctypes.c_int32, _P, _P, _P]
         L.rpa_build_group_tables.restype = ctypes.c_int
+        L.rpa_build_qtile_tables.argtypes = [_P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                             ctypes.c_int32, ctypes.c_int32, _P, _P, _P]
+        L.rpa_build_qtile_tables.restype = ctypes.c_int
         L.rpa_device_error.argtypes = [_I32P, ctypes.c_int32]
         L.rpa_device_error.restype = ctypes.c_int
         L.rpa_status_string.argtypes = [ctypes.c_int]
@@ -199,10 +202,11 @@ class Plan:
 def rpa_plan(*, num_seqs: int, num_tokens: int, num_q_heads: int, num_kv_heads: int,
              head_dim: int, page_size: int, num_pages: int, max_blocks_per_seq: int,
              layout: int, causal: bool, cu_seqlens_q, seq_lens_k, force_class: int = 0,
-             decode_split_keys: int = 0, sparse: bool = False) -> Plan:
+             decode_split_keys: int = 0, sparse=False) -> Plan:
     shape = Shape(num_seqs, num_tokens, num_q_heads, num_kv_heads, head_dim, page_size,
                   num_pages, max_blocks_per_seq, layout, 1 if causal else 0)
-    opts = PlanOptions(force_class, decode_split_keys, 1 if sparse else 0)
+    # sparse: False/0 none, True/1 per-group tables, 2 per-(query tile, query head) tables
+    opts = PlanOptions(force_class, decode_split_keys, int(sparse))
     handle = ctypes.c_void_p()
     ws = ctypes.c_size_t(0)
     _check("rpa_plan", lib().rpa_plan(ctypes.byref(shape), _host_i32(cu_seqlens_q),
@@ -294,6 +298,15 @@ def rpa_build_group_tables(mask, num_kv_heads: int, table, count, stream=None):
     B, Hq, nqb, nkb = mask.shape
     _check("rpa_build_group_tables", lib().rpa_build_group_tables(
         _ptr(mask), B, Hq, num_kv_heads, nqb, nkb, _ptr(table), _ptr(count), _stream(stream)))
+
+
+def rpa_build_qtile_tables(mask, q_block_rows: int, table, count, stream=None):
+    """Per-(query tile, query head) tables [B, Hq, ntiles, nkb] from a block mask
+    [B, Hq, nqb, nkb] (block-sparse execution, for plans made with sparse=2)."""
+    B, Hq, nqb, nkb = mask.shape
+    _check("rpa_build_qtile_tables", lib().rpa_build_qtile_tables(
+        _ptr(mask), B, Hq, nqb, nkb, int(q_block_rows), _ptr(table), _ptr(count),
+        _stream(stream)))
 
 
 def rpa_device_error(clear: bool = True) -> int:

@@ -145,7 +145,63 @@ __global__ void __launch_bounds__(kVecThreads) group_tables_vec_kernel(
   if (threadIdx.x == 0) count[(size_t)b * Hkv + g] = n;
 }
 
+// Per-(query tile, query head) tables: the execution of a block-sparse kernel that works per
+// query block and head (the comparison of CompactAttention's Fig. 7c, execution-only ablation
+// with the same mask).  Row (b, hq, tile) lists, in ascending order, the KV blocks that head hq
+// selects in any query block of the 128-row query tile; the rest of the row is -1.  One CTA
+// per row; the same ballot compaction as group_tables_kernel.
+__global__ void __launch_bounds__(kThreads) qtile_tables_kernel(
+    const uint8_t* __restrict__ mask, int Hq, int nqb, int nkb, int qb_per_tile, int ntiles,
+    int32_t* __restrict__ table, int32_t* __restrict__ count) {
+  __shared__ int warp_tot[kThreads / 32];
+  __shared__ int base_sh;
+  const int tile = blockIdx.x % ntiles;
+  const int hq = (blockIdx.x / ntiles) % Hq;
+  const int b = blockIdx.x / (ntiles * Hq);
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
+  const uint8_t* m0 = mask + ((size_t)b * Hq + hq) * nqb * nkb;
+  const int qb0 = tile * qb_per_tile;
+  const int qb1 = min(nqb, qb0 + qb_per_tile);
+  int32_t* row = table + (((size_t)b * Hq + hq) * ntiles + tile) * nkb;
+  if (threadIdx.x == 0) base_sh = 0;
+  __syncthreads();
+  for (int start = 0; start < nkb; start += kThreads) {
+    const int kb = start + threadIdx.x;
+    int sel = 0;
+    if (kb < nkb)
+      for (int qb = qb0; qb < qb1 && !sel; ++qb) sel = __ldg(m0 + (size_t)qb * nkb + kb) != 0;
+    const unsigned ballot = __ballot_sync(0xffffffffu, sel);
+    const int in_warp = __popc(ballot & ((1u << lane) - 1u));
+    if (lane == 0) warp_tot[warp] = __popc(ballot);
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int w = 0; w < kThreads / 32; ++w) {
+      const int c = warp_tot[w];
+      if (w < warp) before += c;
+      total += c;
+    }
+    const int base = base_sh;
+    if (sel) row[base + before + in_warp] = kb;
+    __syncthreads();
+    if (threadIdx.x == 0) base_sh = base + total;
+    __syncthreads();
+  }
+  const int n = base_sh;
+  for (int i = n + threadIdx.x; i < nkb; i += kThreads) row[i] = -1;
+  if (threadIdx.x == 0) count[((size_t)b * Hq + hq) * ntiles + tile] = n;
+}
+
 }  // namespace
+
+cudaError_t launch_qtile_tables(const uint8_t* mask, int B, int Hq, int nqb, int nkb,
+                                int qb_per_tile, int ntiles, int32_t* table, int32_t* count,
+                                cudaStream_t stream) {
+  if (B <= 0 || ntiles <= 0) return cudaSuccess;
+  qtile_tables_kernel<<<B * Hq * ntiles, kThreads, 0, stream>>>(mask, Hq, nqb, nkb, qb_per_tile,
+                                                                ntiles, table, count);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_group_tables(const uint8_t* mask, int B, int Hq, int Hkv, int nqb, int nkb,
                                 int32_t* table, int32_t* count, cudaStream_t stream) {

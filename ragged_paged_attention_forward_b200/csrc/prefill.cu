@@ -40,6 +40,7 @@ constexpr int kThreads = 384;
 constexpr int kStagesK = 2;  // K tiles in flight
 constexpr int kStagesV = 2;  // V tiles in flight
 constexpr int kRows = kPrefillTileRows;  // 128
+static_assert(kRows == 128, "query-tile table rows are q_start >> 7");
 constexpr int kKeys = kPrefillTileKeys;  // 128
 constexpr uint32_t kTmemCols = 512;
 constexpr float kMaxTileSum = 0x1p64f;  // a tile whose row sum passes this is redone
@@ -127,7 +128,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int Hq = p.num_q_heads;
   const int G = Hq / p.num_kv_heads;
-  const int hpc = (G & 1) == 0 ? 2 : 1;            // query heads per CTA
+  // query heads per CTA: a pair of one KV group (they share every K/V tile); one head with
+  // per-(query tile, head) tables or an odd group size
+  const int hpc = (p.qtile_table == nullptr && (G & 1) == 0) ? 2 : 1;
   const int groups = Hq / hpc;
   const int tile_idx = blockIdx.x / groups;
   if (p.count && tile_idx >= __ldg(p.count)) return;  // device-planned step: unused CTA
@@ -144,10 +147,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int32_t* table = nullptr;
   int n_entries = 0;
   int n_tiles;
-  if (p.group_table) {
-    const size_t row = (size_t)tile.seq * p.num_kv_heads + h;
-    table = p.group_table + row * p.kv.max_blocks;
-    const int cnt = min(__ldg(p.group_count + row), p.kv.max_blocks);
+  if (p.group_table || p.qtile_table) {
+    // the table of the pair's KV group, or of this query tile and head
+    const size_t row =
+        p.qtile_table ? ((size_t)tile.seq * Hq + hq0) * p.qtiles_per_seq + (tile.q_start >> 7)
+                      : (size_t)tile.seq * p.num_kv_heads + h;
+    table = (p.qtile_table ? p.qtile_table : p.group_table) + row * p.kv.max_blocks;
+    const int cnt =
+        min(__ldg((p.qtile_table ? p.qtile_count : p.group_count) + row), p.kv.max_blocks);
     // entries (ascending block ids) whose block starts before kv_hi; every warp of the CTA
     // runs this search with all its lanes
     n_entries = warp_count_below(table, max(cnt, 0), (kv_hi + P - 1) >> log2P);
@@ -609,7 +616,7 @@ cudaError_t launch_prefill(const PrefillLaunch& p, const PrefillTilesInline* inl
   e = encode_kv_map(&vmap, p.kv.v_pool, p.kv, p.head_dim, kKeys);
   if (e != cudaSuccess) return e;
   const int G = p.num_q_heads / p.num_kv_heads;
-  const int hpc = (G & 1) == 0 ? 2 : 1;
+  const int hpc = (p.qtile_table == nullptr && (G & 1) == 0) ? 2 : 1;  // as in the kernel
   const dim3 grid((unsigned)p.num_tiles * (unsigned)(p.num_q_heads / hpc));
   // the register rebalancing inside the kernel needs exactly the launch budget it was
   // written for; refuse to launch otherwise (a short budget would stall setmaxnreg.inc)

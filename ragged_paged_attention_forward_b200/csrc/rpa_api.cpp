@@ -76,6 +76,8 @@ struct rpa_plan_s {
   bool device_mode = false;
   int max_kv_len = 0;
   int cap_items = 0, cap_rows = 0, cap_tiles = 0;
+  // opts.sparse == 2: query tiles per sequence in the per-(query tile, head) tables
+  int qtiles_per_seq = 0;
   size_t off_counts = 0;
   int launches_forward = 0;
   int launches_write = 0;
@@ -183,6 +185,8 @@ rpa_status rpa_plan(const rpa_shape* shape, const int32_t* cu_seqlens_q,
        o.decode_split_keys > kMaxSplitKeys))
     RPA_FAIL(RPA_ERR_INVALID_ARG, "decode_split_keys %d must be a multiple of %d in [%d, %d]",
              o.decode_split_keys, kDecodeStageKeys, kDecodeStageKeys, kMaxSplitKeys);
+  if (o.sparse < 0 || o.sparse > 2)
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "opts.sparse %d must be 0, 1 or 2", o.sparse);
   if (o.sparse && s.layout != RPA_LAYOUT_HEAD_MAJOR)
     RPA_FAIL(RPA_ERR_UNSUPPORTED, "block-union tables need the KV-head-major layout");
   if (o.sparse && s.page_size > kMaxSparsePage)
@@ -279,6 +283,10 @@ rpa_status rpa_plan(const rpa_shape* shape, const int32_t* cu_seqlens_q,
                    });
 
   // ---- prefill tiles (heaviest first: most visible keys)
+  for (int b = 0; b < B; ++b)
+    plan->qtiles_per_seq = std::max(plan->qtiles_per_seq,
+                                    (cu_seqlens_q[b + 1] - cu_seqlens_q[b] + kPrefillTileRows - 1) /
+                                        kPrefillTileRows);
   for (int b = 0; b < B; ++b) {
     const int t0 = cu_seqlens_q[b];
     const int q_len = cu_seqlens_q[b + 1] - t0;
@@ -596,7 +604,7 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     RPA_FAIL(RPA_ERR_INVALID_ARG, "group tables need the KV-head-major layout");
   if ((group_table != nullptr) != (plan->opts.sparse != 0))
     RPA_FAIL(RPA_ERR_INVALID_ARG,
-             "group tables must be given exactly when the plan was made with opts.sparse = 1");
+             "tables must be given exactly when the plan was made with opts.sparse = 1 or 2");
   if (!std::isfinite(scale)) RPA_FAIL(RPA_ERR_INVALID_ARG, "scale must be finite");
   if (!workspace || workspace_bytes < plan->ws_bytes)
     RPA_FAIL(RPA_ERR_WORKSPACE_TOO_SMALL, "workspace of %zu bytes needed, %zu given",
@@ -768,8 +776,14 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     p.scale_log2 = scale_log2;
     p.out = static_cast<uint16_t*>(out);
     p.lse = lse;
-    p.group_table = group_table;
-    p.group_count = group_count;
+    if (plan->opts.sparse == 2) {
+      p.qtile_table = group_table;
+      p.qtile_count = group_count;
+      p.qtiles_per_seq = plan->qtiles_per_seq;
+    } else {
+      p.group_table = group_table;
+      p.group_count = group_count;
+    }
     p.err = err;
     p.kv = kv;
     st = check_cuda(launch_prefill(p, &plan->pf_inline, pf_stream), "prefill launch");
@@ -882,6 +896,29 @@ rpa_status rpa_build_group_tables(const uint8_t* mask, int32_t num_seqs, int32_t
                                         num_kv_blocks, table, count,
                                         static_cast<cudaStream_t>(stream)),
                     "group-table launch");
+}
+
+rpa_status rpa_build_qtile_tables(const uint8_t* mask, int32_t num_seqs, int32_t num_q_heads,
+                                  int32_t num_q_blocks, int32_t num_kv_blocks,
+                                  int32_t q_block_rows, int32_t* table, int32_t* count,
+                                  void* stream) {
+  g_last_error.clear();
+  if (num_seqs < 0 || num_q_heads <= 0 || num_q_blocks < 0 || num_kv_blocks < 0)
+    RPA_FAIL(RPA_ERR_SHAPE, "invalid table-builder sizes");
+  if (q_block_rows <= 0 || q_block_rows > kPrefillTileRows ||
+      kPrefillTileRows % q_block_rows != 0)
+    RPA_FAIL(RPA_ERR_UNSUPPORTED, "q_block_rows %d must divide %d", q_block_rows,
+             kPrefillTileRows);
+  if (num_kv_blocks > 65536) RPA_FAIL(RPA_ERR_UNSUPPORTED, "num_kv_blocks > 65536");
+  const int qb_per_tile = kPrefillTileRows / q_block_rows;
+  const int ntiles = (num_q_blocks + qb_per_tile - 1) / qb_per_tile;
+  if (num_seqs == 0 || ntiles == 0) return RPA_OK;
+  if (!table || !count || (!mask && num_kv_blocks > 0))
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "mask, table and count are required");
+  return check_cuda(launch_qtile_tables(mask, num_seqs, num_q_heads, num_q_blocks, num_kv_blocks,
+                                        qb_per_tile, ntiles, table, count,
+                                        static_cast<cudaStream_t>(stream)),
+                    "query-tile table launch");
 }
 
 rpa_status rpa_device_error(int32_t* code, int32_t clear) {

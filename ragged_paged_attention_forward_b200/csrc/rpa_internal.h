@@ -145,6 +145,11 @@ struct PrefillLaunch {
   float* lse;
   const int32_t* group_table;  // [B, Hkv, max_blocks] or null
   const int32_t* group_count;  // [B, Hkv] or null
+  // per-(query tile, query head) tables instead (block-sparse execution, one head per CTA):
+  // [B, Hq, qtiles_per_seq, max_blocks] and [B, Hq, qtiles_per_seq], or null
+  const int32_t* qtile_table;
+  const int32_t* qtile_count;
+  int32_t qtiles_per_seq;
   int* err;
   PagedKV kv;
 };
@@ -227,6 +232,9 @@ cudaError_t launch_decode(const DecodeLaunch& p, const DecodeItemsInline* inl, i
 cudaError_t launch_merge(const MergeLaunch& p, const MergeRowsInline* inl, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillLaunch& p, const PrefillTilesInline* inl,
                            cudaStream_t stream);
+cudaError_t launch_qtile_tables(const uint8_t* mask, int B, int Hq, int nqb, int nkb,
+                                int qb_per_tile, int ntiles, int32_t* table, int32_t* count,
+                                cudaStream_t stream);
 cudaError_t launch_group_tables(const uint8_t* mask, int B, int Hq, int Hkv, int nqb, int nkb,
                                 int32_t* table, int32_t* count, cudaStream_t stream);
 

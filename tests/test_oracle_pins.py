@@ -609,3 +609,86 @@ def test_write_kv8_places_quantised_codes_in_hand_derived_slots():
     for (b_, pos) in [(0, 3), (0, 4), (1, 16), (1, 17), (1, 18)]:
         mask[bt[b_, pos // 16], pos % 16] = False
     assert np.array_equal(kp[mask], before[mask])
+
+
+# --------------------------------------------------------------------------------------
+# Per-(query tile, query head) tables: the block-sparse execution of the ablation
+# --------------------------------------------------------------------------------------
+
+def test_qtile_tables_hand_fixture():
+    # B=1, Hq=2, 4 query blocks of 64 rows (two 128-row tiles), 6 KV blocks
+    m = np.zeros((1, 2, 4, 6), dtype=np.uint8)
+    m[0, 0, 0, [0, 3]] = 1      # head 0, tile 0 = q-blocks 0, 1
+    m[0, 0, 1, [3, 5]] = 1
+    m[0, 0, 3, [1]] = 1         # head 0, tile 1 = q-blocks 2, 3
+    m[0, 1, 2, [2, 4]] = 1      # head 1: nothing in tile 0
+    table, count = orc.build_qtile_tables(m, 64)
+    assert table.shape == (1, 2, 2, 6)
+    assert count.tolist() == [[[3, 1], [0, 2]]]
+    assert table[0, 0, 0].tolist() == [0, 3, 5, -1, -1, -1]
+    assert table[0, 0, 1].tolist() == [1, -1, -1, -1, -1, -1]
+    assert table[0, 1, 0].tolist() == [-1] * 6
+    assert table[0, 1, 1].tolist() == [2, 4, -1, -1, -1, -1]
+    # q_block_rows 128: one query block per tile; 32: four per tile
+    t1, c1 = orc.build_qtile_tables(m, 128)
+    assert t1.shape == (1, 2, 4, 6) and c1[0, 0].tolist() == [2, 2, 0, 1]
+    t4, c4 = orc.build_qtile_tables(m, 32)
+    assert t4.shape == (1, 2, 1, 6) and c4[0].tolist() == [[4], [2]]
+
+
+def _expand_union(table, count, Hq, nqb, nkb):
+    """The unioned mask written back per (head, query block): every row of group g holds g's
+    union (so block-sparse execution and per-group tables see the same blocks)."""
+    B, Hkv = count.shape
+    G = Hq // Hkv
+    m = np.zeros((B, Hq, nqb, nkb), dtype=np.uint8)
+    for b in range(B):
+        for g in range(Hkv):
+            sel = table[b, g, :count[b, g]]
+            m[b, g * G:(g + 1) * G, :, sel] = 1
+    return m
+
+
+def test_qtile_tables_of_the_unioned_mask_equal_group_tables():
+    rng = np.random.default_rng(61)
+    mask = (rng.random((2, 8, 5, 23)) < 0.15).astype(np.uint8)
+    gt, gc = orc.build_group_tables(mask, 2)
+    u = _expand_union(gt, gc, 8, 5, 23)
+    qt, qc = orc.build_qtile_tables(u, 64)
+    for b in range(2):
+        for hq in range(8):
+            for tau in range(qt.shape[2]):
+                assert qc[b, hq, tau] == gc[b, hq // 4]
+                assert np.array_equal(qt[b, hq, tau], gt[b, hq // 4])
+
+
+def test_qtile_attention_equals_group_attention_on_the_unioned_mask():
+    P = 16
+    b = wl.ragged_batch([300, 190], [260, 70], 8, 2, 32, P, seed=62, layout=wl.HEAD_MAJOR)
+    nkb = b.max_blocks
+    rng = np.random.default_rng(63)
+    nqb = -(-260 // 64)
+    mask = (rng.random((2, 8, nqb, nkb)) < 0.3).astype(np.uint8)
+    gt, gc = orc.build_group_tables(mask, 2)
+    o1, l1, _, _ = _oracle_forward(b, group_table=gt, group_count=gc)
+    qt, qc = orc.build_qtile_tables(_expand_union(gt, gc, 8, nqb, nkb), 64)
+    o2, l2, _, _ = _oracle_forward(b, qtile_table=qt, qtile_count=qc)
+    assert np.array_equal(o1, o2, equal_nan=True) and np.array_equal(l1, l2, equal_nan=True)
+    # a per-tile mask that differs between tiles and heads is not the union: rows of tile 0
+    # of head 0 keep only block 0 -> attention over keys 0..15 of that row's prefix
+    m2 = np.zeros_like(mask)
+    m2[:, :, :, :] = 1
+    m2[0, 0, :2, :] = 0
+    m2[0, 0, :2, 0] = 1
+    qt2, qc2 = orc.build_qtile_tables(m2, 64)
+    o3, _, _, _ = _oracle_forward(b, qtile_table=qt2, qtile_count=qc2)
+    past = 300 - 260
+    for i in (0, 5, 127):
+        n = min(past + i + 1, P)
+        K = _f64(b.k_logical[0][:n, 0])
+        V = _f64(b.v_logical[0][:n, 0])
+        ref = _sdpa_row(_f64(b.q[i, 0]), K, V, b.scale)
+        assert np.max(np.abs(o3[i, 0] - ref)) < 1e-12
+    dense, _, _, _ = _oracle_forward(b)
+    assert np.array_equal(o3[128:260, 0], dense[128:260, 0])   # tile 1: all blocks
+    assert np.array_equal(o3[:, 1:], dense[:, 1:])
