@@ -403,7 +403,12 @@ rpa_status rpa_plan_device(const rpa_shape* shape, int32_t max_kv_len,
   const long splits = (max_kv_len + plan->split_keys - 1) / plan->split_keys;
   plan->cap_items = (int)std::min<long>((long)B * splits, 1L << 24);
   plan->cap_rows = std::max(s.num_tokens, 1);
-  plan->cap_tiles = (s.num_tokens + kPrefillTileRows - 1) / kPrefillTileRows + B;
+  // a sequence reaches the tensor-core kernel only with q_len * G > 8 * decode_nt, i.e. with
+  // at least qmin tokens, so at most T / qmin sequences add a partial tile each: a bound far
+  // below T / 128 + B for decode-heavy steps, which keeps the grid of early-exiting CTAs small
+  const int qmin = 8 * plan->decode_nt / G + 1;
+  plan->cap_tiles = (s.num_tokens + kPrefillTileRows - 1) / kPrefillTileRows +
+                    std::min(B, s.num_tokens / qmin);
   size_t off = 0;
   plan->off_counts = off;
   off = align_up(off + 16, 256);
@@ -451,7 +456,7 @@ void rpa_plan_destroy(rpa_plan_t plan) { delete plan; }
 static rpa_status write_kv_impl(rpa_plan_t plan, const void* k_new, const void* v_new,
                                 void* k_pool, void* v_pool, const int32_t* block_table,
                                 const int32_t* cu_seqlens_q, const int32_t* seq_lens_k,
-                                cudaStream_t stream) {
+                                cudaStream_t stream, int skip_rows_upto = 0) {
   const rpa_shape& s = plan->shape;
   int* err = nullptr;
   rpa_status st = check_cuda(device_error_word(&err), "device error word");
@@ -473,6 +478,8 @@ static rpa_status write_kv_impl(rpa_plan_t plan, const void* k_new, const void* 
   w.layout = s.layout;
   w.num_pages = s.num_pages;
   w.tokens_on_device = plan->device_mode ? 1 : 0;
+  w.skip_rows_upto = skip_rows_upto;
+  w.group = s.num_q_heads / s.num_kv_heads;
   w.err = err;
   return check_cuda(launch_write_kv(w, stream), "write_kv launch");
 }
@@ -614,7 +621,7 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
 
   if (kv8 && k_new && !plan->fuse_write)
     RPA_FAIL(RPA_ERR_UNSUPPORTED, "e4m3 pools: the KV write runs inside the decode kernel");
-  if (k_new && !plan->fuse_write) {
+  if (k_new && !plan->fuse_write && !plan->device_mode) {
     st = write_kv_impl(plan, k_new, v_new, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k,
                        stream);
     if (st != RPA_OK) return st;
@@ -685,6 +692,13 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     if (st != RPA_OK) return st;
     st = check_cuda(cudaStreamWaitEvent(pf_stream, plan->fork_ev, 0), "fork wait");
     if (st != RPA_OK) return st;
+    // new tokens: the decode kernel writes those of its own rows (as for host plans); the
+    // scatter kernel, on the side stream ahead of the tensor-core kernel, writes the rest
+    if (k_new) {
+      st = write_kv_impl(plan, k_new, v_new, k_pool, v_pool, block_table, cu_seqlens_q,
+                         seq_lens_k, pf_stream, 8 * plan->decode_nt);
+      if (st != RPA_OK) return st;
+    }
     PrefillLaunch p{};
     p.tiles = pl.tiles;
     p.num_tiles = plan->cap_tiles;
@@ -719,6 +733,10 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     d.part_lse = reinterpret_cast<float*>(ws + plan->off_part_lse);
     d.err = err;
     d.kv = kv;
+    d.k_new = static_cast<const uint16_t*>(k_new);
+    d.v_new = static_cast<const uint16_t*>(v_new);
+    d.k_pool_w = k_new ? k_pool : nullptr;
+    d.v_pool_w = k_new ? v_pool : nullptr;
     st = check_cuda(launch_decode(d, &plan->dec_inline, plan->decode_nt, stream),
                     "decode launch");
     if (st != RPA_OK) return st;

@@ -171,6 +171,10 @@ struct WriteLaunch {
   int32_t layout;
   int32_t num_pages;
   int32_t tokens_on_device;  // 1: num_tokens is a bound, the step has cu_seqlens_q[num_seqs]
+  // > 0: skip the tokens of sequences with q_len * group <= skip_rows_upto (their rows go to
+  // the decode kernel, which writes them itself)
+  int32_t skip_rows_upto;
+  int32_t group;
   int* err;
 };
 

@@ -36,6 +36,7 @@ __global__ void __launch_bounds__(256) write_kv_kernel(WriteLaunch p) {
     const int b = seq_of_token(p.cu_seqlens_q, p.num_seqs, t);
     const int t0 = __ldg(p.cu_seqlens_q + b);
     const int q_len = __ldg(p.cu_seqlens_q + b + 1) - t0;
+    if (p.skip_rows_upto > 0 && q_len * p.group <= p.skip_rows_upto) continue;
     const int past = __ldg(p.seq_lens_k + b) - q_len;
     const int pos = past + (t - t0);
     const int blk = pos / p.page_size;

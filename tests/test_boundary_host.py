@@ -213,6 +213,12 @@ def test_device_plan_sizes_its_workspace_for_the_limits():
     assert info.num_decode_items == 4 * (1024 // info.decode_split_keys)
     assert info.num_merge_rows == 512 and info.num_prefill_tiles == 512 // 128 + 4
     assert p.workspace_bytes >= info.num_decode_items * 32 and p.workspace_bytes % 256 == 0
+    # a decode-heavy bound: 64 tokens over 64 sequences; a sequence reaches the tensor-core
+    # kernel only with q_len * G > 8 (q_len >= 3 for G = 4), so at most 21 partial tiles
+    d = _device_plan(num_seqs=64, max_tokens=64).info()
+    assert d.num_prefill_tiles == 1 + 64 // 3
+    g16 = _device_plan(num_seqs=64, max_tokens=64, num_q_heads=128).info()  # G = 16, NT = 2
+    assert g16.num_prefill_tiles == 1 + 64 // 2
 
 
 @pytest.mark.parametrize("kw,status", [
