@@ -58,7 +58,10 @@ cudaError_t encode_kv_map(CUtensorMap* map, const void* pool, const PagedKV& kv,
   CUresult r = enc(map, kv.kv8 ? CU_TENSOR_MAP_DATA_TYPE_UINT8 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16,
                    4, const_cast<void*>(pool), dims,
                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_SWIZZLE_128B,
+                   // a box row is 128 bytes; bf16 rows come in two halves (256 bytes
+                   // together), e4m3 rows are one 128-byte run at a stride of Hkv*D bytes
+                   kv.kv8 ? CU_TENSOR_MAP_L2_PROMOTION_L2_128B : CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     set_last_error("cuTensorMapEncodeTiled(kv) failed with CUresult %d", (int)r);
