@@ -667,6 +667,47 @@ def measure_sparse_ablation(steps, warmup, peaks):
     return res
 
 
+def measure_mixed_kv8(steps, warmup, peaks):
+    """The mixed workload over e4m3 pools (rpa_forward_kv8 with a kv_e4m3 plan): decode rows
+    on the codes directly, the two prefill chunks on an exact bf16 copy of their context made
+    after the quantising write.  Timed as the fused step, back to back over rotating pool
+    copies; the roofline is the sum of the bf16-equivalent tensor time and the e4m3 byte
+    time, as for the bf16 mixed line."""
+    from ragged_paged_attention_forward_b200 import api
+    from ragged_paged_attention_forward_b200 import workloads as wl
+    b, _ = make_workload("mixed")
+    b8, ks, vs = wl.with_kv8_pools(b, seed=4321, poison=False)
+    d = {k: getattr(b8, k).cuda().contiguous() for k in (
+        "q", "k_new", "v_new", "k_pool", "v_pool", "block_table", "cu_seqlens_q", "seq_lens_k")}
+    ks, vs = ks.cuda(), vs.cuda()
+    pool_bytes = 2 * d["k_pool"].numel()
+    n = max(3, -(-2 * L2_BYTES // pool_bytes) + 1)
+    pools = [(d["k_pool"], d["v_pool"])] + [(d["k_pool"].clone(), d["v_pool"].clone())
+                                            for _ in range(n - 1)]
+    plan = api.rpa_plan(num_seqs=b8.num_seqs, num_tokens=b8.num_tokens,
+                        num_q_heads=b8.num_q_heads, num_kv_heads=b8.num_kv_heads,
+                        head_dim=b8.head_dim, page_size=b8.page_size, num_pages=b8.num_pages,
+                        max_blocks_per_seq=b8.max_blocks, layout=b8.layout, causal=b8.causal,
+                        cu_seqlens_q=b8.cu_seqlens_q, seq_lens_k=b8.seq_lens_k, kv_e4m3=True)
+    ws = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(d["q"])
+
+    def step(i):
+        kp, vp = pools[i % len(pools)]
+        api.rpa_forward_kv8(plan, d["q"], d["k_new"], d["v_new"], kp, vp, ks, vs,
+                            d["block_table"], d["cu_seqlens_q"], d["seq_lens_k"], b8.scale, out,
+                            None, ws)
+
+    ms = timed_loop(step, steps, warmup)
+    w = work(b)
+    info = plan.info()
+    return {"workload": WORKLOAD_TEXT["mixed"] + "; K/V cache as e4m3 codes with per-KV-head "
+            "scales", "ms_per_step": ms, "tokens_per_s": b8.num_tokens / (ms * 1e-3),
+            "bf16_equivalent_TFLOPs": w["flops"] / (ms * 1e-3) / 1e12,
+            "launches_per_step": info.launches_forward + 1,
+            "workspace_MB": plan.workspace_bytes / 1e6}
+
+
 def measure_input_pass(steps, warmup, peaks):
     """The input pass with rotary embedding (rpa_rotary_write_kv) on the prefill workload's
     16384 new tokens: packed QKV in, RoPE over all 128 dims (split pairs), Q out, K/V
@@ -909,6 +950,7 @@ def run_gpu(args):
             torch.cuda.empty_cache()
         secondary["input_pass"] = measure_input_pass(args.steps, args.warmup, peaks)
         secondary["decode_kv8"] = measure_decode_kv8(args.steps, args.warmup, peaks)
+        secondary["mixed_kv8"] = measure_mixed_kv8(args.steps, args.warmup, peaks)
         secondary["sparse_ablation"] = measure_sparse_ablation(args.steps, args.warmup, peaks)
         secondary["decode_device_planned"] = measure_device_planned_decode(args.steps,
                                                                            args.warmup, peaks)

@@ -87,7 +87,10 @@ typedef struct rpa_plan_options {
   int32_t decode_split_keys;   /* keys per decode split, multiple of 64; 0 = automatic     */
   int32_t sparse;              /* 1: rpa_forward will be given group tables; 2: per-(query  */
                                /* tile, query head) tables (rpa_build_qtile_tables)         */
-  int32_t reserved[5];         /* must be zero                                             */
+  int32_t kv_e4m3;             /* 1: the pools will hold e4m3 codes (rpa_forward_kv8): the   */
+                               /* workspace also holds a bf16 copy of the context of rows  */
+                               /* that go to the tensor-core kernel                        */
+  int32_t reserved[4];         /* must be zero                                             */
 } rpa_plan_options;
 
 typedef struct rpa_plan_info {
@@ -278,10 +281,13 @@ RPA_API rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new
  *                     the e4m3 code nearest to fp32(x) / scale (IEEE fp32 division; ties to
  *                     the even code; magnitudes past 448 saturate to +-448).
  *   the rest          as for rpa_forward (no group tables).
- * Supported: head_dim 128 and host plans whose rows all go to the split-KV decode kernel
- * (rpa_plan_info.batch_class == RPA_CLASS_DECODE, or num_prefill_tiles == 0); anything else
- * returns RPA_ERR_UNSUPPORTED.  Scores and P.V run on f16 operands (e4m3 -> f16 is exact;
- * q must stay within f16's range, |q| < 65504) with fp32 accumulation.
+ * Supported: head_dim 128, host plans (no group tables).  Rows for the split-KV decode kernel
+ * read the e4m3 pools directly: scores and P.V on f16 operands (e4m3 -> f16 is exact; q must
+ * stay within f16's range, |q| < 65504), fp32 accumulation.  A plan with rows for the
+ * tensor-core kernel must be made with opts.kv_e4m3 = 1: after the write, those sequences'
+ * context is copied to bf16 in the workspace (exactly: every e4m3 value is a bf16 value) and
+ * the tensor-core kernel reads the copy with k_scale[h] folded into its score scale and
+ * v_scale[h] into its output.  Anything else returns RPA_ERR_UNSUPPORTED.
  */
 RPA_API rpa_status rpa_forward_kv8(rpa_plan_t plan, const void* q, const void* k_new,
                                    const void* v_new, void* k_pool, void* v_pool,

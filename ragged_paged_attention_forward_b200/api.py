@@ -39,7 +39,8 @@ class Shape(ctypes.Structure):
 
 class PlanOptions(ctypes.Structure):
     _fields_ = [("force_class", ctypes.c_int32), ("decode_split_keys", ctypes.c_int32),
-                ("sparse", ctypes.c_int32), ("reserved", ctypes.c_int32 * 5)]
+                ("sparse", ctypes.c_int32), ("kv_e4m3", ctypes.c_int32),
+                ("reserved", ctypes.c_int32 * 4)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -202,11 +203,11 @@ class Plan:
 def rpa_plan(*, num_seqs: int, num_tokens: int, num_q_heads: int, num_kv_heads: int,
              head_dim: int, page_size: int, num_pages: int, max_blocks_per_seq: int,
              layout: int, causal: bool, cu_seqlens_q, seq_lens_k, force_class: int = 0,
-             decode_split_keys: int = 0, sparse=False) -> Plan:
+             decode_split_keys: int = 0, sparse=False, kv_e4m3: bool = False) -> Plan:
     shape = Shape(num_seqs, num_tokens, num_q_heads, num_kv_heads, head_dim, page_size,
                   num_pages, max_blocks_per_seq, layout, 1 if causal else 0)
     # sparse: False/0 none, True/1 per-group tables, 2 per-(query tile, query head) tables
-    opts = PlanOptions(force_class, decode_split_keys, int(sparse))
+    opts = PlanOptions(force_class, decode_split_keys, int(sparse), 1 if kv_e4m3 else 0)
     handle = ctypes.c_void_p()
     ws = ctypes.c_size_t(0)
     _check("rpa_plan", lib().rpa_plan(ctypes.byref(shape), _host_i32(cu_seqlens_q),

@@ -399,7 +399,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q_local = tile.q_start + r;
     const int pos = past + q_local;                 // absolute position of this row
     const int lim = p.causal ? min(tile.kv_len, pos + 1) : tile.kv_len;
-    const float sc = p.scale_log2;
+    const float sc = p.k_scale ? p.scale_log2 * __ldg(p.k_scale + h) : p.scale_log2;
     float m_ref = -CUDART_INF_F, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_tiles; ++j) {
@@ -565,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t = tile.t0 + q_local;
       const bool write = q_local < tile.q_len;
       uint16_t* orow = p.out + ((size_t)t * Hq + hq) * D;
-      const float inv = l > 0.f ? 1.f / l : 0.f;
+      const float inv = l > 0.f ? (p.v_scale ? __ldg(p.v_scale + h) : 1.f) / l : 0.f;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t o[32];

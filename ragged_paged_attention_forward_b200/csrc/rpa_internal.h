@@ -150,6 +150,10 @@ struct PrefillLaunch {
   const int32_t* qtile_table;
   const int32_t* qtile_count;
   int32_t qtiles_per_seq;
+  // per-KV-head factors on the scores and the output (the e4m3 path reads exact bf16 copies
+  // of the codes: K = code * k_scale[h], V = code * v_scale[h]); null: 1
+  const float* k_scale;
+  const float* v_scale;
   int* err;
   PagedKV kv;
 };
@@ -157,8 +161,11 @@ struct PrefillLaunch {
 struct WriteLaunch {
   const uint16_t* k_new;
   const uint16_t* v_new;
-  uint16_t* k_pool;
-  uint16_t* v_pool;
+  void* k_pool;              // bf16 pools, or e4m3 code pools when kv8
+  void* v_pool;
+  int32_t kv8;               // 1: store e4m3(fp32(x) / scale[kv head]) codes
+  const float* k_scale;      // [Hkv] (kv8)
+  const float* v_scale;
   const int32_t* block_table;
   const int32_t* cu_seqlens_q;
   const int32_t* seq_lens_k;
@@ -175,6 +182,31 @@ struct WriteLaunch {
   // the decode kernel, which writes them itself)
   int32_t skip_rows_upto;
   int32_t group;
+  int* err;
+};
+
+// e4m3 -> bf16 copy of the context of the sequences that the tensor-core kernel reads: row r
+// of the work list is key position pos of sequence seqs[i] (row_off[i] <= r < row_off[i+1],
+// pos = r - row_off[i]); every KV head's K and V row of that position is converted exactly
+// (every e4m3 value is a bf16 value; the scale is not applied) from the code pools, through
+// block_table, into the bf16 scratch pools, through out_table (same layout).
+struct DequantLaunch {
+  const uint8_t* k_pool;
+  const uint8_t* v_pool;
+  const int32_t* block_table;
+  uint16_t* k_out;
+  uint16_t* v_out;
+  const int32_t* out_table;
+  const int32_t* seqs;
+  const int32_t* row_off;
+  int32_t num_list;          // entries of seqs
+  int32_t num_rows;          // row_off[num_list]
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t page_size;
+  int32_t max_blocks;
+  int32_t layout;
+  int32_t num_pages;
   int* err;
 };
 
@@ -236,6 +268,7 @@ cudaError_t launch_decode(const DecodeLaunch& p, const DecodeItemsInline* inl, i
 cudaError_t launch_merge(const MergeLaunch& p, const MergeRowsInline* inl, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillLaunch& p, const PrefillTilesInline* inl,
                            cudaStream_t stream);
+cudaError_t launch_dequant_kv8(const DequantLaunch& p, cudaStream_t stream);
 cudaError_t launch_qtile_tables(const uint8_t* mask, int B, int Hq, int nqb, int nkb,
                                 int qb_per_tile, int ntiles, int32_t* table, int32_t* count,
                                 cudaStream_t stream);

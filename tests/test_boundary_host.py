@@ -249,3 +249,22 @@ def test_forward_kv8_rejects_before_any_device_work():
             api.rpa_forward_kv8(plan, None, None, None, None, None, None, None, None, None,
                                 None, 0.1, None, None, None, stream=0)
         assert ei.value.status == api.RPA_ERR_UNSUPPORTED, kw
+
+
+def test_kv_e4m3_plan_option():
+    # a plan with a tensor-core row: the e4m3 option adds the bf16 copy of that sequence's
+    # context (scratch table, lists, K and V copies) to the workspace
+    kw = dict(cu_seqlens_q=[0, 1, 200], num_tokens=200, seq_lens_k=[40, 200])
+    plain = api.rpa_plan(**_shape(**kw))
+    e4 = api.rpa_plan(**_shape(**kw), kv_e4m3=True)
+    copy = 2 * 13 * 16 * 8 * 128 * 2            # ceil(200 / 16) pages of K and of V, bf16
+    assert e4.workspace_bytes >= plain.workspace_bytes + copy
+    # decode-only plans need no copy
+    d_plain = api.rpa_plan(**_shape())
+    d_e4 = api.rpa_plan(**_shape(), kv_e4m3=True)
+    assert d_e4.workspace_bytes == d_plain.workspace_bytes
+    for bad, status in ((dict(head_dim=64), api.RPA_ERR_UNSUPPORTED),
+                        (dict(layout=1, sparse=True), api.RPA_ERR_UNSUPPORTED)):
+        with pytest.raises(api.RPAError) as ei:
+            api.rpa_plan(**_shape(**bad), kv_e4m3=True)
+        assert ei.value.status == status

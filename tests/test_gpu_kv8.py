@@ -109,6 +109,39 @@ def test_kv8_without_new_tokens_reads_cache_only():
     assert_lse_close(lse, ref_lse)
 
 
+@pytest.mark.parametrize("layout", [wl.SEQ_MAJOR, wl.HEAD_MAJOR])
+@pytest.mark.parametrize("page", [16, 64])
+def test_kv8_mixed_batch_through_both_kernels(layout, page):
+    # decode rows on the e4m3 pools directly; prefill chunks (with past) on the exact bf16
+    # copy of their context; the new tokens of both quantised by the scatter kernel
+    b = wl.ragged_batch([300, 40, 1500, 9, 700], [300, 1, 213, 1, 77], 32, 8, 128, page,
+                        seed=960 + page)
+    if layout == wl.HEAD_MAJOR:
+        b = wl.to_head_major(b)
+    b8, ks, vs = wl.with_kv8_pools(b, seed=961)
+    out, lse, kp, vp, plan = run_kv8(b8, ks, vs, plan_opts=dict(kv_e4m3=True))
+    info = plan.info()
+    assert info.num_prefill_tiles > 0 and info.num_decode_items > 0
+    ref, ref_lse, kp_ref, vp_ref = oracle_kv8(b8, ks, vs)
+    assert np.array_equal(kp.numpy(), kp_ref) and np.array_equal(vp.numpy(), vp_ref)
+    check_out(out, ref, vs, b8)
+    assert_lse_close(lse, ref_lse)
+
+
+def test_kv8_prefill_only_and_non_causal():
+    import dataclasses
+    b = wl.ragged_batch([640, 200], [512, 200], 16, 4, 128, 32, seed=970)
+    for causal in (True, False):
+        bc = dataclasses.replace(b, causal=causal)
+        b8, ks, vs = wl.with_kv8_pools(bc, seed=971)
+        out, lse, kp, vp, plan = run_kv8(b8, ks, vs, plan_opts=dict(kv_e4m3=True))
+        assert plan.info().num_decode_items == 0
+        ref, ref_lse, kp_ref, _ = oracle_kv8(b8, ks, vs)
+        assert np.array_equal(kp.numpy(), kp_ref)
+        check_out(out, ref, vs, b8)
+        assert_lse_close(lse, ref_lse)
+
+
 def test_kv8_rejects_unsupported_plans():
     b = wl.ragged_batch([300, 40], [300, 1], 8, 2, 128, 16, seed=940)   # has a prefill row
     b8, ks, vs = wl.with_kv8_pools(b, seed=941)
