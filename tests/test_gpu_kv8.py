@@ -152,3 +152,53 @@ def test_kv8_rejects_unsupported_plans():
     b64_8, ks, vs = wl.with_kv8_pools(b64, seed=943)
     with pytest.raises(api.RPAError):
         run_kv8(b64_8, ks, vs)
+
+
+def _sample_rows(batch, n, seed):
+    g = np.random.default_rng(seed)
+    T, Hq = batch.num_tokens, batch.num_q_heads
+    rows = {(int(t), int(h)) for t, h in zip(g.integers(0, T, n), g.integers(0, Hq, n))}
+    cu = batch.cu_seqlens_q.tolist()
+    for b in range(batch.num_seqs):
+        if cu[b + 1] > cu[b]:
+            rows.add((cu[b], int(g.integers(0, Hq))))
+            rows.add((cu[b + 1] - 1, int(g.integers(0, Hq))))
+    return sorted(rows)
+
+
+def _check_rows(out, lse, ref, ref_lse, rows, vs):
+    got = out.double().numpy()
+    vmax = 448.0 * float(vs.max())
+    for t, h in rows:
+        err = np.abs(got[t, h] - ref[t, h])
+        assert np.all(err <= 2.0 ** -8 * vmax + 2.0 ** -8 * np.abs(ref[t, h])), (t, h, err.max())
+        assert abs(float(lse[t, h]) - ref_lse[t, h]) <= 2e-3, (t, h)
+
+
+def test_kv8_decode_workload_full_size_sampled():
+    # the benchmark's decode batch (64 sequences, kv 512-8192) over e4m3 pools, in the launch
+    # configuration the benchmark times; the oracle computes sampled rows one by one
+    b8, ks, vs = wl.with_kv8_pools(wl.decode(), seed=1234)
+    out, lse, kp, vp, plan = run_kv8(b8, ks, vs)
+    assert plan.info().batch_class == api.CLASS_DECODE
+    rows = _sample_rows(b8, 48, seed=5)
+    ref, ref_lse, kp_ref, vp_ref = orc.forward_kv8(
+        b8.q, b8.k_new, b8.v_new, b8.k_pool, b8.v_pool, ks.numpy(), vs.numpy(), b8.block_table,
+        b8.cu_seqlens_q, b8.seq_lens_k, scale=b8.scale, causal=True, page_size=b8.page_size,
+        layout=b8.layout, rows=rows)
+    assert np.array_equal(kp.numpy(), kp_ref) and np.array_equal(vp.numpy(), vp_ref)
+    _check_rows(out, lse, ref, ref_lse, rows, vs)
+
+
+def test_kv8_mixed_workload_full_size_sampled():
+    b8, ks, vs = wl.with_kv8_pools(wl.mixed(), seed=4321)
+    out, lse, kp, vp, plan = run_kv8(b8, ks, vs, plan_opts=dict(kv_e4m3=True))
+    info = plan.info()
+    assert info.num_prefill_tiles > 0 and info.num_decode_items > 0
+    rows = _sample_rows(b8, 48, seed=6)
+    ref, ref_lse, kp_ref, _ = orc.forward_kv8(
+        b8.q, b8.k_new, b8.v_new, b8.k_pool, b8.v_pool, ks.numpy(), vs.numpy(), b8.block_table,
+        b8.cu_seqlens_q, b8.seq_lens_k, scale=b8.scale, causal=True, page_size=b8.page_size,
+        layout=b8.layout, rows=rows)
+    assert np.array_equal(kp.numpy(), kp_ref)
+    _check_rows(out, lse, ref, ref_lse, rows, vs)

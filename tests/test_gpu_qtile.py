@@ -74,3 +74,23 @@ def test_qtile_on_the_unioned_mask_equals_group_tables_bit_for_bit():
     # the same tiles, keys and arithmetic per row: one head per CTA changes no row's result
     assert torch.equal(out_g.view(torch.int16), out_q.view(torch.int16))
     assert torch.equal(lse_g, lse_q)
+
+
+def test_qtile_sparse_workload_full_size_sampled():
+    # the benchmark's sparse configuration (2048 queries at 128K context) run block-sparse per
+    # (query tile, head) on the original per-head mask; sampled rows against the oracle
+    b, mask = wl.sparse()
+    m = mask.numpy()
+    table, count = _gpu_qtile_tables(m, b.num_tokens // m.shape[2])
+    out, lse, _, _, _ = run_forward(b, group_table=table, group_count=count,
+                                    plan_opts=dict(sparse=2))
+    g = np.random.default_rng(7)
+    rows = sorted({(int(t), int(h)) for t, h in zip(g.integers(0, b.num_tokens, 24),
+                                                    g.integers(0, b.num_q_heads, 24))})
+    ref, ref_lse, _, _ = orc.forward(b.q, b.k_new, b.v_new, b.k_pool, b.v_pool, b.block_table,
+                                     b.cu_seqlens_q, b.seq_lens_k, scale=b.scale, causal=True,
+                                     page_size=b.page_size, layout=b.layout,
+                                     qtile_table=table.cpu().numpy(),
+                                     qtile_count=count.cpu().numpy(), rows=rows)
+    assert_close(out, ref, rows=rows)
+    assert_lse_close(lse, ref_lse, rows=rows)
