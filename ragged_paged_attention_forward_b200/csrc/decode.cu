@@ -149,17 +149,11 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
           const uint16_t* src = (which == 0 ? p.k_new : p.v_new) +
                                 ((size_t)tok * p.num_kv_heads + h) * D + c * 16;
           const float sc = __ldg((which == 0 ? p.k_scale : p.v_scale) + h);
-          const uint4 a = __ldg(reinterpret_cast<const uint4*>(src));
-          const uint4 b = __ldg(reinterpret_cast<const uint4*>(src) + 1);
-          auto q2 = [sc](uint32_t v) {  // a bf16 pair -> two codes
-            return pack_e4m3x2(__fdiv_rn(__uint_as_float(v << 16), sc),
-                               __fdiv_rn(__uint_as_float(v & 0xffff0000u), sc));
-          };
           uint8_t* dst = static_cast<uint8_t*>(which == 0 ? p.k_pool_w : p.v_pool_w) + row * D +
                          c * 16;
           *reinterpret_cast<uint4*>(dst) =
-              make_uint4(q2(a.x) | (q2(a.y) << 16), q2(a.z) | (q2(a.w) << 16),
-                         q2(b.x) | (q2(b.y) << 16), q2(b.z) | (q2(b.w) << 16));
+              e4m3_quantize16(__ldg(reinterpret_cast<const uint4*>(src)),
+                              __ldg(reinterpret_cast<const uint4*>(src) + 1), sc);
         } else {
           const uint16_t* src = (which == 0 ? p.k_new : p.v_new) +
                                 ((size_t)tok * p.num_kv_heads + h) * D + c * 8;

@@ -244,6 +244,17 @@ __device__ __forceinline__ uint32_t pack_e4m3x2(float lo, float hi) {
   return d;
 }
 
+// 16 bf16 values (two 16-byte words) -> 16 e4m3 codes of fp32(x) / sc: an IEEE fp32 divide,
+// then nearest-even e4m3 with saturation; code i lands in byte i.
+__device__ __forceinline__ uint4 e4m3_quantize16(const uint4 a, const uint4 b, float sc) {
+  auto q2 = [sc](uint32_t v) {  // a bf16 pair -> two codes
+    return pack_e4m3x2(__fdiv_rn(__uint_as_float(v << 16), sc),
+                       __fdiv_rn(__uint_as_float(v & 0xffff0000u), sc));
+  };
+  return make_uint4(q2(a.x) | (q2(a.y) << 16), q2(a.z) | (q2(a.w) << 16),
+                    q2(b.x) | (q2(b.y) << 16), q2(b.z) | (q2(b.w) << 16));
+}
+
 // Two fp32 -> packed f16x2 (round to nearest even); `lo` lands in bits 0..15.
 __device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
   uint32_t d;

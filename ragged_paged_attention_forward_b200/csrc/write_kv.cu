@@ -25,16 +25,6 @@ __device__ __forceinline__ int seq_of_token(const int32_t* __restrict__ cu, int 
   return lo;
 }
 
-// 16 bf16 values -> 16 e4m3 codes of fp32(x) / sc (IEEE divide, nearest even, saturating)
-__device__ __forceinline__ uint4 quantize16(const uint4 a, const uint4 b, float sc) {
-  auto q2 = [sc](uint32_t v) {
-    return pack_e4m3x2(__fdiv_rn(__uint_as_float(v << 16), sc),
-                       __fdiv_rn(__uint_as_float(v & 0xffff0000u), sc));
-  };
-  return make_uint4(q2(a.x) | (q2(a.y) << 16), q2(a.z) | (q2(a.w) << 16),
-                    q2(b.x) | (q2(b.y) << 16), q2(b.z) | (q2(b.w) << 16));
-}
-
 // e4m3 pools: one warp per token, one 16-byte output chunk (16 codes) per lane and step
 __device__ void write_token_kv8(const WriteLaunch& p, int t, int b, int blk, int slot,
                                 int lane) {
@@ -58,8 +48,10 @@ __device__ void write_token_kv8(const WriteLaunch& p, int t, int b, int blk, int
     const uint4* vs = reinterpret_cast<const uint4*>(p.v_new + src);
     uint8_t* kd = static_cast<uint8_t*>(p.k_pool) + row * p.head_dim + cc * 16;
     uint8_t* vd = static_cast<uint8_t*>(p.v_pool) + row * p.head_dim + cc * 16;
-    *reinterpret_cast<uint4*>(kd) = quantize16(__ldg(ks), __ldg(ks + 1), __ldg(p.k_scale + h));
-    *reinterpret_cast<uint4*>(vd) = quantize16(__ldg(vs), __ldg(vs + 1), __ldg(p.v_scale + h));
+    *reinterpret_cast<uint4*>(kd) =
+        e4m3_quantize16(__ldg(ks), __ldg(ks + 1), __ldg(p.k_scale + h));
+    *reinterpret_cast<uint4*>(vd) =
+        e4m3_quantize16(__ldg(vs), __ldg(vs + 1), __ldg(p.v_scale + h));
   }
 }
 
