@@ -184,6 +184,19 @@ RPA_API rpa_status rpa_write_kv(rpa_plan_t plan, const void* k_new, const void* 
                         void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * rpa_write_kv8 -- rpa_write_kv for e4m3 code pools (see rpa_forward_kv8): every new element
+ * x of KV head h is stored as the e4m3 code nearest to fp32(x) / scale[h] (IEEE fp32 division,
+ * ties to the even code, magnitudes past 448 saturate).  k_pool / v_pool are uint8 pools in
+ * shape.layout; k_scale / v_scale device fp32 [Hkv].  head_dim must be a multiple of 16.
+ * T == 0 returns RPA_OK and launches nothing.
+ */
+RPA_API rpa_status rpa_write_kv8(rpa_plan_t plan, const void* k_new, const void* v_new,
+                                 void* k_pool, void* v_pool, const float* k_scale,
+                                 const float* v_scale, const int32_t* block_table,
+                                 const int32_t* cu_seqlens_q, const int32_t* seq_lens_k,
+                                 void* stream);
+
+/*
  * Rotary position embedding applied by rpa_rotary_write_kv ("[WebGPU] Optimized
  * PagedAttention implementation (2/n)", commit "Phase 1b.2": the rotary program rotates Q and
  * K before the K/V scatter, with position_id = past_b + s and dims >= rotary_dim copied

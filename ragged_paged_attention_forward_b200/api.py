@@ -93,6 +93,8 @@ def lib() -> ctypes.CDLL:
         L.rpa_forward.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, ctypes.c_float,
                                   _P, _P, _P, ctypes.c_size_t, _P]
         L.rpa_forward.restype = ctypes.c_int
+        L.rpa_write_kv8.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
+        L.rpa_write_kv8.restype = ctypes.c_int
         L.rpa_forward_kv8.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                       ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]
         L.rpa_forward_kv8.restype = ctypes.c_int
@@ -250,6 +252,16 @@ def rpa_forward(plan: Plan, q, k_new, v_new, k_pool, v_pool, block_table, cu_seq
         plan.handle, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool),
         _ptr(block_table), _ptr(cu_seqlens_q), _ptr(seq_lens_k), _ptr(group_table),
         _ptr(group_count), ctypes.c_float(scale), _ptr(out), _ptr(lse), _ptr(workspace), nbytes,
+        _stream(stream)))
+
+
+def rpa_write_kv8(plan: Plan, k_new, v_new, k_pool, v_pool, k_scale, v_scale, block_table,
+                  cu_seqlens_q, seq_lens_k, stream=None):
+    """Quantise and scatter the new tokens into e4m3 (uint8) pools with per-KV-head
+    scales."""
+    _check("rpa_write_kv8", lib().rpa_write_kv8(
+        plan.handle, _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool), _ptr(k_scale),
+        _ptr(v_scale), _ptr(block_table), _ptr(cu_seqlens_q), _ptr(seq_lens_k),
         _stream(stream)))
 
 

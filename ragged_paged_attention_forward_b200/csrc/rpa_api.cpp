@@ -567,6 +567,26 @@ rpa_status rpa_write_kv(rpa_plan_t plan, const void* k_new, const void* v_new, v
                        seq_lens_k, static_cast<cudaStream_t>(stream));
 }
 
+rpa_status rpa_write_kv8(rpa_plan_t plan, const void* k_new, const void* v_new, void* k_pool,
+                         void* v_pool, const float* k_scale, const float* v_scale,
+                         const int32_t* block_table, const int32_t* cu_seqlens_q,
+                         const int32_t* seq_lens_k, void* stream) {
+  g_last_error.clear();
+  rpa_status st = check_common(plan, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k);
+  if (st != RPA_OK) return st;
+  if (plan->shape.head_dim % 16 != 0)
+    RPA_FAIL(RPA_ERR_UNSUPPORTED, "e4m3 pools need head_dim a multiple of 16");
+  if (plan->shape.num_tokens == 0) return RPA_OK;
+  if (!k_new || !v_new) RPA_FAIL(RPA_ERR_INVALID_ARG, "k_new and v_new are required");
+  if (!aligned16(k_new) || !aligned16(v_new))
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "k_new / v_new must be 16-byte aligned");
+  if (!k_scale || !v_scale) RPA_FAIL(RPA_ERR_INVALID_ARG, "k_scale and v_scale are required");
+  if ((reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u))
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "k_scale / v_scale must be 4-byte aligned");
+  return write_kv_impl(plan, k_new, v_new, k_pool, v_pool, block_table, cu_seqlens_q,
+                       seq_lens_k, static_cast<cudaStream_t>(stream), 0, k_scale, v_scale);
+}
+
 rpa_status rpa_rotary_write_kv(rpa_plan_t plan, const void* q, const void* k, const void* v,
                                const rpa_rotary* rotary, void* q_out, void* k_pool,
                                void* v_pool, const int32_t* block_table,

@@ -202,3 +202,22 @@ def test_kv8_mixed_workload_full_size_sampled():
         layout=b8.layout, rows=rows)
     assert np.array_equal(kp.numpy(), kp_ref)
     _check_rows(out, lse, ref, ref_lse, rows, vs)
+
+
+@pytest.mark.parametrize("layout", [wl.SEQ_MAJOR, wl.HEAD_MAJOR])
+def test_kv8_standalone_write_bit_exact(layout):
+    b = wl.ragged_batch([70, 300, 9], [70, 5, 9], 16, 4, 128, 32, seed=980)
+    if layout == wl.HEAD_MAJOR:
+        b = wl.to_head_major(b)
+    b8, ks, vs = wl.with_kv8_pools(b, seed=981)
+    plan = plan_for(b8)
+    d = {k: getattr(b8, k).cuda().contiguous() for k in (
+        "k_new", "v_new", "k_pool", "v_pool", "block_table", "cu_seqlens_q", "seq_lens_k")}
+    api.rpa_write_kv8(plan, d["k_new"], d["v_new"], d["k_pool"], d["v_pool"], ks.cuda(),
+                      vs.cuda(), d["block_table"], d["cu_seqlens_q"], d["seq_lens_k"])
+    torch.cuda.synchronize()
+    assert api.rpa_device_error(clear=True) == 0
+    kp, vp = orc.write_kv8(b8.k_pool, b8.v_pool, b8.k_new, b8.v_new, ks.numpy(), vs.numpy(),
+                           b8.block_table, b8.cu_seqlens_q, b8.seq_lens_k, 32, layout)
+    assert np.array_equal(d["k_pool"].cpu().numpy(), kp)
+    assert np.array_equal(d["v_pool"].cpu().numpy(), vp)
