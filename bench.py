@@ -708,6 +708,55 @@ def measure_mixed_kv8(steps, warmup, peaks):
             "workspace_MB": plan.workspace_bytes / 1e6}
 
 
+def measure_device_planned_decode_kv8(steps, warmup, peaks):
+    """The e4m3 decode step with a device plan (kv_e4m3), captured in CUDA graphs and
+    replayed (three launches: planner, decode with the quantising write, merge); one graph
+    per pool copy, replayed in turn."""
+    from ragged_paged_attention_forward_b200 import api
+    from ragged_paged_attention_forward_b200 import workloads as wl
+    b, _ = make_workload("decode")
+    b8, ks, vs = wl.with_kv8_pools(b, seed=1234, poison=False)
+    d = {k: getattr(b8, k).cuda().contiguous() for k in (
+        "q", "k_new", "v_new", "k_pool", "v_pool", "block_table", "cu_seqlens_q", "seq_lens_k")}
+    ks, vs = ks.cuda(), vs.cuda()
+    n = max(3, -(-2 * L2_BYTES // (2 * d["k_pool"].numel())) + 1)
+    pools = [(d["k_pool"], d["v_pool"])] + [(d["k_pool"].clone(), d["v_pool"].clone())
+                                            for _ in range(n - 1)]
+    plan = api.rpa_plan_device(num_seqs=b8.num_seqs, max_tokens=b8.num_tokens,
+                               num_q_heads=b8.num_q_heads, num_kv_heads=b8.num_kv_heads,
+                               head_dim=b8.head_dim, page_size=b8.page_size,
+                               num_pages=b8.num_pages, max_blocks_per_seq=b8.max_blocks,
+                               layout=b8.layout, causal=b8.causal,
+                               max_kv_len=int(b8.seq_lens_k.max()), kv_e4m3=True)
+    ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device="cuda")
+    out = torch.empty_like(d["q"])
+
+    def step(kp, vp):
+        api.rpa_forward_kv8(plan, d["q"], d["k_new"], d["v_new"], kp, vp, ks, vs,
+                            d["block_table"], d["cu_seqlens_q"], d["seq_lens_k"], b8.scale, out,
+                            None, ws)
+
+    for kp, vp in pools:
+        step(kp, vp)
+    torch.cuda.synchronize()
+    graphs = []
+    for kp, vp in pools:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            step(kp, vp)
+        graphs.append(g)
+    ms = timed_loop(lambda i: graphs[i % len(graphs)].replay(), steps, warmup)
+    T, Hq, D = b8.q.shape
+    step_bytes = float(sum(b8.kv_lens())) * b8.num_kv_heads * D * 2 + 2.0 * T * Hq * D * 2 + \
+        2.0 * T * b8.num_kv_heads * D * 3
+    res = {"workload": WORKLOAD_TEXT["decode"] + "; e4m3 pools, device-planned, CUDA-graph "
+           "replay", "ms_per_step": ms, "step_GBps": step_bytes / (ms * 1e-3) / 1e9,
+           "frac_of_hbm": step_bytes / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+           "launches_per_step": plan.info().launches_forward}
+    del graphs
+    return res
+
+
 def measure_input_pass(steps, warmup, peaks):
     """The input pass with rotary embedding (rpa_rotary_write_kv) on the prefill workload's
     16384 new tokens: packed QKV in, RoPE over all 128 dims (split pairs), Q out, K/V
@@ -954,6 +1003,8 @@ def run_gpu(args):
         secondary["sparse_ablation"] = measure_sparse_ablation(args.steps, args.warmup, peaks)
         secondary["decode_device_planned"] = measure_device_planned_decode(args.steps,
                                                                            args.warmup, peaks)
+        secondary["decode_kv8_device_planned"] = measure_device_planned_decode_kv8(
+            args.steps, args.warmup, peaks)
         line["secondary"] = secondary
         if "prefill" in secondary:
             line["prefill_TFLOPs"] = secondary["prefill"]["attn_TFLOPs"]

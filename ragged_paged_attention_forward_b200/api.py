@@ -221,13 +221,14 @@ def rpa_plan(*, num_seqs: int, num_tokens: int, num_q_heads: int, num_kv_heads: 
 def rpa_plan_device(*, num_seqs: int, max_tokens: int, num_q_heads: int, num_kv_heads: int,
                     head_dim: int, page_size: int, num_pages: int, max_blocks_per_seq: int,
                     layout: int, causal: bool, max_kv_len: int,
-                    decode_split_keys: int = 0) -> Plan:
+                    decode_split_keys: int = 0, kv_e4m3: bool = False) -> Plan:
     """A plan whose work lists are built on the device at every call (CUDA-graph friendly):
     B = num_seqs sequences, at most max_tokens new tokens and max_kv_len keys per step.  The
-    q / k_new / v_new / out / lse buffers of the calls hold max_tokens rows."""
+    q / k_new / v_new / out / lse buffers of the calls hold max_tokens rows.  kv_e4m3: for
+    rpa_forward_kv8; every row must fit the decode kernel."""
     shape = Shape(num_seqs, max_tokens, num_q_heads, num_kv_heads, head_dim, page_size,
                   num_pages, max_blocks_per_seq, layout, 1 if causal else 0)
-    opts = PlanOptions(0, decode_split_keys, 0)
+    opts = PlanOptions(0, decode_split_keys, 0, 1 if kv_e4m3 else 0)
     handle = ctypes.c_void_p()
     ws = ctypes.c_size_t(0)
     _check("rpa_plan_device", lib().rpa_plan_device(ctypes.byref(shape), int(max_kv_len),

@@ -422,7 +422,8 @@ rpa_status rpa_plan_device(const rpa_shape* shape, int32_t max_kv_len,
   for (int i = 0; i < 4; ++i)
     if (o.reserved[i] != 0) RPA_FAIL(RPA_ERR_INVALID_ARG, "plan option reserved[%d] != 0", i);
   if (o.sparse) RPA_FAIL(RPA_ERR_UNSUPPORTED, "device-planned steps take no group tables");
-  if (o.kv_e4m3) RPA_FAIL(RPA_ERR_UNSUPPORTED, "device-planned steps: no e4m3 pools");
+  if (o.kv_e4m3 && s.head_dim != 128)
+    RPA_FAIL(RPA_ERR_UNSUPPORTED, "e4m3 pools need head_dim 128 (got %d)", s.head_dim);
   if (o.force_class != RPA_CLASS_AUTO)
     RPA_FAIL(RPA_ERR_UNSUPPORTED, "device-planned steps choose their kernels per sequence");
   if (o.decode_split_keys != 0 &&
@@ -476,7 +477,8 @@ rpa_status rpa_plan_device(const rpa_shape* shape, int32_t max_kv_len,
   off = align_up(off + (size_t)plan->cap_items * s.num_kv_heads * rows_per_item * 4, 256);
   plan->ws_bytes = off;
   plan->launches_write = 1;
-  plan->launches_forward = 5;  // planner, KV write, tensor-core, decode, merge
+  // planner, KV write, tensor-core, decode, merge; e4m3 plans: planner, decode, merge
+  plan->launches_forward = o.kv_e4m3 ? 3 : 5;
   *out_plan = plan;
   if (workspace_bytes) *workspace_bytes = plan->ws_bytes;
   return RPA_OK;
@@ -770,6 +772,7 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     pl.causal = s.causal;
     pl.split_keys = plan->split_keys;
     pl.decode_rows = 8 * plan->decode_nt;
+    pl.no_prefill = kv8 ? 1 : 0;
     pl.cap_items = plan->cap_items;
     pl.cap_rows = plan->cap_rows;
     pl.cap_tiles = plan->cap_tiles;
@@ -781,8 +784,10 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     st = check_cuda(launch_plan_device(pl, stream), "device planner launch");
     if (st != RPA_OK) return st;
     // both kernel families: the tensor-core kernel on the side stream, forked after the
-    // planner, the decode kernel and the merge on the caller's stream; joined at the end
+    // planner, the decode kernel and the merge on the caller's stream; joined at the end.
+    // e4m3 device plans run decode rows only (the planner refused the others): no fork.
     cudaStream_t pf_stream = stream;
+    if (!kv8) {
     st = check_cuda(side_stream(&pf_stream), "side stream");
     if (st != RPA_OK) return st;
     if (!plan->fork_ev) {
@@ -821,6 +826,7 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     p.kv = kv;
     st = check_cuda(launch_prefill(p, &plan->pf_inline, pf_stream), "prefill launch");
     if (st != RPA_OK) return st;
+    }
     DecodeLaunch d{};
     d.items = pl.items;
     d.num_items = plan->cap_items;
@@ -842,6 +848,8 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     d.v_new = static_cast<const uint16_t*>(v_new);
     d.k_pool_w = k_new ? k_pool : nullptr;
     d.v_pool_w = k_new ? v_pool : nullptr;
+    d.k_scale = k_scale;
+    d.v_scale = v_scale;
     st = check_cuda(launch_decode(d, &plan->dec_inline, plan->decode_nt, stream),
                     "decode launch");
     if (st != RPA_OK) return st;
@@ -859,6 +867,7 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     m.lse = lse;
     st = check_cuda(launch_merge(m, &plan->merge_inline, stream), "merge launch");
     if (st != RPA_OK) return st;
+    if (kv8) return RPA_OK;
     st = check_cuda(cudaEventRecord(plan->join_ev, pf_stream), "join record");
     if (st != RPA_OK) return st;
     return check_cuda(cudaStreamWaitEvent(stream, plan->join_ev, 0), "join wait");
@@ -996,9 +1005,10 @@ rpa_status rpa_forward_kv8(rpa_plan_t plan, const void* q, const void* k_new, co
   if (plan->shape.head_dim != 128)
     RPA_FAIL(RPA_ERR_UNSUPPORTED, "e4m3 pools need head_dim 128 (got %d)",
              plan->shape.head_dim);
-  if (plan->device_mode)
-    RPA_FAIL(RPA_ERR_UNSUPPORTED, "e4m3 pools: device-planned steps are not supported");
-  if (!plan->pf_tiles.empty() && !plan->opts.kv_e4m3)
+  if (plan->device_mode && !plan->opts.kv_e4m3)
+    RPA_FAIL(RPA_ERR_UNSUPPORTED,
+             "e4m3 pools with a device plan need a plan made with opts.kv_e4m3 = 1");
+  if (!plan->device_mode && !plan->pf_tiles.empty() && !plan->opts.kv_e4m3)
     RPA_FAIL(RPA_ERR_UNSUPPORTED,
              "e4m3 pools with rows for the tensor-core kernel need a plan made with "
              "opts.kv_e4m3 = 1");

@@ -251,6 +251,7 @@ struct PlanDeviceLaunch {
   int32_t causal;
   int32_t split_keys;
   int32_t decode_rows;           // a sequence goes to the decode kernel when q_len * G <= this
+  int32_t no_prefill;            // 1: a sequence past decode_rows raises kErrLimits, is skipped
   int32_t cap_items, cap_rows, cap_tiles;
   DecodeItem* items;
   MergeRow* rows;

@@ -115,3 +115,72 @@ def test_step_beyond_the_limits_is_reported():
     st.run(b.scale)
     torch.cuda.synchronize()
     assert api.rpa_device_error(clear=True) & 16
+
+
+def test_e4m3_device_plan_graph_replays_decode_batches():
+    # a CUDA graph of rpa_forward_kv8 with a device plan made with kv_e4m3: the decode kernel
+    # quantises its rows' new tokens and reads the codes; replayed over two batches
+    plan = api.rpa_plan_device(num_seqs=B, max_tokens=MAX_T, num_q_heads=HQ, num_kv_heads=HKV,
+                               head_dim=D, page_size=P, num_pages=NUM_PAGES,
+                               max_blocks_per_seq=MAX_BLOCKS, layout=wl.SEQ_MAJOR, causal=True,
+                               max_kv_len=MAX_KV, kv_e4m3=True)
+    assert plan.info().launches_forward == 3
+    z = lambda *s, dt=torch.bfloat16: torch.zeros(*s, dtype=dt, device="cuda")
+    q, out = z(MAX_T, HQ, D), z(MAX_T, HQ, D)
+    k_new, v_new = z(MAX_T, HKV, D), z(MAX_T, HKV, D)
+    lse = z(MAX_T, HQ, dt=torch.float32)
+    kp = z(NUM_PAGES, P, HKV, D, dt=torch.uint8)
+    vp = z(NUM_PAGES, P, HKV, D, dt=torch.uint8)
+    bt, cu, kv = z(B, MAX_BLOCKS, dt=torch.int32), z(B + 1, dt=torch.int32), z(B, dt=torch.int32)
+    ks, vs = z(HKV, dt=torch.float32), z(HKV, dt=torch.float32)
+    ws = torch.empty(plan.workspace_bytes, dtype=torch.uint8, device="cuda")
+
+    def load(b8, k_scale, v_scale):
+        T = b8.num_tokens
+        q.zero_(); k_new.zero_(); v_new.zero_()
+        q[:T].copy_(b8.q); k_new[:T].copy_(b8.k_new); v_new[:T].copy_(b8.v_new)
+        kp.copy_(b8.k_pool); vp.copy_(b8.v_pool)
+        bt.zero_(); bt[:, :b8.max_blocks].copy_(b8.block_table)
+        cu.copy_(b8.cu_seqlens_q); kv.copy_(b8.seq_lens_k)
+        ks.copy_(k_scale); vs.copy_(v_scale)
+
+    def step():
+        api.rpa_forward_kv8(plan, q, k_new, v_new, kp, vp, ks, vs, bt, cu, kv, 1.0 / D ** 0.5,
+                            out, lse, ws)
+
+    batches = [([40, 700, 1, 3000, 129, 64], [1] * 6, 301), ([2, 90, 1500, 33, 4000, 10],
+                                                             [2, 1, 2, 1, 2, 1], 302)]
+    first = True
+    graph = None
+    for kv_lens, q_lens, seed in batches:
+        b = _batch(kv_lens, q_lens, seed)
+        b8, k_scale, v_scale = wl.with_kv8_pools(b, seed=seed + 1)
+        load(b8, k_scale, v_scale)
+        if first:
+            step(); torch.cuda.synchronize()
+            load(b8, k_scale, v_scale)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                step()
+            first = False
+        graph.replay()
+        torch.cuda.synchronize()
+        assert api.rpa_device_error(clear=True) == 0
+        T = b8.num_tokens
+        ref, ref_lse, kp_ref, vp_ref = orc.forward_kv8(
+            b8.q, b8.k_new, b8.v_new, b8.k_pool, b8.v_pool, k_scale.numpy(), v_scale.numpy(),
+            b8.block_table, b8.cu_seqlens_q, b8.seq_lens_k, scale=1.0 / D ** 0.5, causal=True,
+            page_size=P, layout=wl.SEQ_MAJOR)
+        assert np.array_equal(kp.cpu().numpy(), kp_ref) and np.array_equal(vp.cpu().numpy(), vp_ref)
+        got = out[:T].cpu().double().numpy()
+        bound = 2.0 ** -8 * 448.0 * float(v_scale.max()) + 2.0 ** -8 * np.abs(ref)
+        assert np.all(np.abs(got - ref) <= bound)
+        assert_lse_close(lse[:T].cpu(), ref_lse)
+    # a row too long for the decode kernel is refused (limits bit) instead of computed
+    b = _batch([300, 40, 1, 1, 1, 1], [300, 1, 1, 1, 1, 1], 303)
+    b8, k_scale, v_scale = wl.with_kv8_pools(b, seed=304)
+    load(b8, k_scale, v_scale)
+    graph.replay()
+    torch.cuda.synchronize()
+    assert api.rpa_device_error(clear=True) & 16
+    del graph
