@@ -1054,6 +1054,16 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+CASES = {
+    "input_pass": measure_input_pass,
+    "decode_kv8": measure_decode_kv8,
+    "mixed_kv8": measure_mixed_kv8,
+    "sparse_ablation": measure_sparse_ablation,
+    "decode_device_planned": measure_device_planned_decode,
+    "decode_kv8_device_planned": measure_device_planned_decode_kv8,
+}
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -1064,9 +1074,18 @@ def main():
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--case", default=None, choices=list(CASES),
+                    help="time one secondary measurement alone and print its result as one "
+                         "JSON line (for launch lists and profiler captures of that case)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
+    if args.case is not None:
+        if not torch.cuda.is_available():
+            raise SystemExit("--case needs a CUDA device")
+        res = CASES[args.case](args.steps, args.warmup, load_peaks())
+        print(json.dumps({"case": args.case, **res}))
+        return
     if args.impl == "reference":
         run_reference(args)
     else:
