@@ -11,10 +11,13 @@
 // block-table lookup per K/V tile) and the prefill specialisation of "Ragged Paged Attention:
 // A High-Performance and Flexible LLM Inference Kernel for TPU" (Key ideas).
 //
-// B200 design.  One CTA per (128-query tile, pair of query heads of one KV group) -- the two
-// heads share every K/V tile and the same causal mask -- with 384 threads:
-//   warp 0      TMA producer: both Q tiles once, then K and V tiles of 128 keys, page by page
-//               (boxes of [min(P,128) slots x 64 dims], 128-byte swizzle), 2-stage ring;
+// B200 design.  The work comes in units of (128-query tile, pair of query heads of one KV
+// group) -- the two heads share every K/V tile and the same causal mask.  A persistent CTA
+// holds one SM (all 512 TMEM columns) and walks its share of the units, so the next unit's Q,
+// K and V stream in, and its first S is computed, while the current unit's O is written out.
+// 384 threads:
+//   warp 0      TMA producer: both Q tiles of a unit, then K and V tiles of 128 keys, page by
+//               page (boxes of [min(P,128) slots x 64 dims], 128-byte swizzle), 2-stage ring;
 //   warp 1      allocates TMEM; one thread issues the MMAs, interleaving the two heads so the
 //               tensor pipe works on one head while the other head's softmax runs:
 //                 S_h = Q_h K_j^T   (M=128 queries, N=128 keys, K=D; SMEM descriptors)
@@ -61,8 +64,8 @@ struct PfGeom {
   static constexpr int kVOff = kKOff + kStagesK * kTileBytes;
   static constexpr int kBarOff = kVOff + kStagesV * kTileBytes;
   // q_full, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], p_ready[2], o_done[2],
-  // mma_done
-  static constexpr int kNumBars = 1 + 2 * kStagesK + 2 * kStagesV + 6 + 1;
+  // q_empty, mma_done
+  static constexpr int kNumBars = 1 + 2 * kStagesK + 2 * kStagesV + 6 + 2;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 64;
   // at least 120 KB so that a second CTA never shares the SM (and its 512 TMEM columns)
@@ -97,6 +100,17 @@ __device__ __forceinline__ int warp_count_below(const int32_t* t, int n, int lim
   return lo + __popc(__ballot_sync(0xffffffffu, below));
 }
 
+// One unit of work: a 128-query tile of one sequence and the pair (or single head) of query
+// heads it serves, with the key tiles those rows see.
+struct Unit {
+  PrefillTile tile;
+  int hq0, h;            // first query head, KV head
+  int past, kv_hi;       // context before the chunk; keys [0, kv_hi) are visible to the tile
+  const int32_t* table;  // sparse modes: the table row, else null
+  int n_entries;         // sparse modes: table entries before kv_hi
+  int n_tiles;           // 128-key tiles
+};
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap,
@@ -119,7 +133,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* s_full = v_empty + kStagesV;   // [2] per head
   uint64_t* p_ready = s_full + 2;           // [2]
   uint64_t* o_done = p_ready + 2;           // [2]
-  uint64_t* mma_done = o_done + 2;
+  uint64_t* q_empty = o_done + 2;           // the unit's S MMAs are done with Q
+  uint64_t* mma_done = q_empty + 1;
   uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(smem + Geo::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Geo::kMiscOff + 8);
   volatile int* never = reinterpret_cast<volatile int*>(smem + Geo::kMiscOff + 12);  // stays 0
@@ -128,44 +143,56 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int lane = threadIdx.x & 31;
   const int Hq = p.num_q_heads;
   const int G = Hq / p.num_kv_heads;
-  // query heads per CTA: a pair of one KV group (they share every K/V tile); one head with
+  // query heads per unit: a pair of one KV group (they share every K/V tile); one head with
   // per-(query tile, head) tables or an odd group size
   const int hpc = (p.qtile_table == nullptr && (G & 1) == 0) ? 2 : 1;
   const int groups = Hq / hpc;
-  const int tile_idx = blockIdx.x / groups;
-  if (p.count && tile_idx >= __ldg(p.count)) return;  // device-planned step: unused CTA
-  const int hq0 = (blockIdx.x - tile_idx * groups) * hpc;
-  const PrefillTile tile = p.tiles ? p.tiles[tile_idx] : inl.v[tile_idx];
-  const int h = hq0 / G;                            // KV head (shared by the pair)
+  const int n_list = p.count ? min(__ldg(p.count), p.num_tiles) : p.num_tiles;
+  const int num_units = n_list * groups;
   const int P = p.kv.page_size;
   const int log2P = p.kv.log2_page;
-  const int past = tile.kv_len - tile.q_len;
-  const int q_end = min(tile.q_len, tile.q_start + kRows);  // local, exclusive
-  const int kv_hi = p.causal ? min(tile.kv_len, past + q_end) : tile.kv_len;
 
-  // key tiles: dense -> ceil(kv_hi/128); sparse -> visible table entries, 128/P per tile
-  const int32_t* table = nullptr;
-  int n_entries = 0;
-  int n_tiles;
-  if (p.group_table || p.qtile_table) {
-    // the table of the pair's KV group, or of this query tile and head
-    const size_t row =
-        p.qtile_table ? ((size_t)tile.seq * Hq + hq0) * p.qtiles_per_seq + (tile.q_start >> 7)
-                      : (size_t)tile.seq * p.num_kv_heads + h;
-    table = (p.qtile_table ? p.qtile_table : p.group_table) + row * p.kv.max_blocks;
-    const int cnt =
-        min(__ldg((p.qtile_table ? p.qtile_count : p.group_count) + row), p.kv.max_blocks);
-    // entries (ascending block ids) whose block starts before kv_hi; every warp of the CTA
-    // runs this search with all its lanes
-    n_entries = warp_count_below(table, max(cnt, 0), (kv_hi + P - 1) >> log2P);
-    const int per = kKeys >> log2P;
-    n_tiles = (n_entries + per - 1) / per;
-  } else {
-    n_tiles = (kv_hi + kKeys - 1) / kKeys;
-  }
+  // The CTA walks units in rounds of gridDim.x, left to right in even rounds and right to left
+  // in odd ones: the list is sorted heaviest first, so the alternation evens out the SMs' load.
+  auto unit_index = [&](int k) {
+    const int base = k * (int)gridDim.x;
+    return (k & 1) ? base + (int)gridDim.x - 1 - (int)blockIdx.x : base + (int)blockIdx.x;
+  };
+  // every role walks the same units and counts barrier phases itself; called by whole warps
+  // (the table search is warp-cooperative)
+  auto unit_at = [&](int u) {
+    Unit w;
+    const int tile_idx = u / groups;
+    w.hq0 = (u - tile_idx * groups) * hpc;
+    w.tile = p.tiles ? p.tiles[tile_idx] : inl.v[tile_idx];
+    w.h = w.hq0 / G;
+    w.past = w.tile.kv_len - w.tile.q_len;
+    const int q_end = min(w.tile.q_len, w.tile.q_start + kRows);  // local, exclusive
+    w.kv_hi = p.causal ? min(w.tile.kv_len, w.past + q_end) : w.tile.kv_len;
+    // key tiles: dense -> ceil(kv_hi/128); sparse -> visible table entries, 128/P per tile
+    w.table = nullptr;
+    w.n_entries = 0;
+    if (p.group_table || p.qtile_table) {
+      // the table of the pair's KV group, or of this query tile and head
+      const size_t row = p.qtile_table ? ((size_t)w.tile.seq * Hq + w.hq0) * p.qtiles_per_seq +
+                                             (w.tile.q_start >> 7)
+                                       : (size_t)w.tile.seq * p.num_kv_heads + w.h;
+      w.table = (p.qtile_table ? p.qtile_table : p.group_table) + row * p.kv.max_blocks;
+      const int cnt =
+          min(__ldg((p.qtile_table ? p.qtile_count : p.group_count) + row), p.kv.max_blocks);
+      // entries (ascending block ids) whose block starts before kv_hi
+      w.n_entries = warp_count_below(w.table, max(cnt, 0), (w.kv_hi + P - 1) >> log2P);
+      const int per = kKeys >> log2P;
+      w.n_tiles = (w.n_entries + per - 1) / per;
+    } else {
+      w.n_tiles = (w.kv_hi + kKeys - 1) / kKeys;
+    }
+    return w;
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
+    mbar_init(q_empty, 1);
     for (int s = 0; s < kStagesK; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
@@ -200,141 +227,180 @@ __global__ void __launch_bounds__(kThreads, 1)
     regs_dealloc<kRegsControl>();
   if (warp == 0) {
     // ------------------------------------------------------------------ TMA producer
-    if (lane == 0 && n_tiles > 0) {
+    // the whole warp walks the units; lane 0 issues the copies and keeps the counters
+    if (lane == 0) {
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
-      mbar_arrive_expect_tx(q_full, Geo::kTileBytes * hpc);
-      for (int x = 0; x < hpc; ++x)
-#pragma unroll
-        for (int half = 0; half < Geo::kHalves; ++half)
-          tma_load_3d(Qs + x * Geo::kTileBytes + half * Geo::kHalfBytes, &qmap, half * 64,
-                      hq0 + x, tile.t0 + tile.q_start, q_full);
-      const int32_t* bt_row =
-          p.kv.layout == 0
-              ? p.kv.block_table + (size_t)tile.seq * p.kv.max_blocks
-              : p.kv.block_table + ((size_t)tile.seq * p.kv.num_kv_heads + h) * p.kv.max_blocks;
-      const int hcoord = p.kv.layout == 0 ? h : 0;
-      const int box_rows = P < kKeys ? P : kKeys;
-      const uint32_t box_bytes = (uint32_t)box_rows * 128u * Geo::kHalves;
-      int issued[2] = {0, 0};  // K and V tiles whose copies were started
-      for (int j = 0; j < n_tiles; ++j) {
-        int nbox, first_blk = 0, slot0 = 0;
-        if (table) {
-          nbox = min(kKeys >> log2P, n_entries - j * (kKeys >> log2P));
-        } else if (P >= kKeys) {
-          nbox = 1;
-          first_blk = (j * kKeys) >> log2P;
-          slot0 = (j * kKeys) & (P - 1);
-        } else {
-          first_blk = (j * kKeys) >> log2P;
-          nbox = ((min(j * kKeys + kKeys, kv_hi) - 1) >> log2P) - first_blk + 1;
-        }
-        // K first (S needs it first), then V; each waits for its own slot to be released
-        bool stop = false;
-        for (int kv = 0; kv < 2; ++kv) {
-          const int ns = kv == 0 ? kStagesK : kStagesV;
-          const int slot = j % ns;
-          uint64_t* empty = kv == 0 ? &k_empty[slot] : &v_empty[slot];
-          if (j >= ns && !wait_bounded(empty, ((j / ns) - 1) & 1, abort_flag, p.err,
-                                       kErrPrefillWait)) {
-            stop = true;
-            break;
-          }
-          mbar_arrive_expect_tx(kv == 0 ? &k_full[slot] : &v_full[slot], box_bytes * nbox);
-          uint8_t* dst_base = (kv == 0 ? Ks : Vs) + slot * Geo::kTileBytes;
-          const CUtensorMap* map = kv == 0 ? &kmap : &vmap;
-          uint64_t* bar = kv == 0 ? &k_full[slot] : &v_full[slot];
-          for (int i = 0; i < nbox; ++i) {
-            const int blk = table ? __ldg(table + j * (kKeys >> log2P) + i) : first_blk + i;
-            int page = -1;  // out-of-range coordinates make TMA fill zeros: no stray access
-            if (blk >= 0 && blk < p.kv.max_blocks)
-              page = __ldg(bt_row + blk);
-            else if (kv == 0)
-              atomicOr(p.err, kErrBadIndex);
+    }
+    int kv_iter = 0;         // K/V tiles begun, over all units of this CTA
+    int q_iter = 0;          // Q tiles begun
+    int issued[2] = {0, 0};  // K and V tiles whose copies were started
+    bool stop = false;
+    for (int k = 0; !stop; ++k) {
+      const int u = unit_index(k);
+      if (u >= num_units) break;
+      const Unit w = unit_at(u);
+      if (w.n_tiles == 0) continue;
+      if (lane == 0) {
+        // Q of the previous unit stays until its S MMAs are done
+        if (q_iter > 0 &&
+            !wait_bounded(q_empty, (q_iter - 1) & 1, abort_flag, p.err, kErrPrefillWait))
+          stop = true;
+        if (!stop) {
+          mbar_arrive_expect_tx(q_full, Geo::kTileBytes * hpc);
+          for (int x = 0; x < hpc; ++x)
 #pragma unroll
             for (int half = 0; half < Geo::kHalves; ++half)
-              tma_load_4d(dst_base + half * Geo::kHalfBytes + i * box_rows * 128, map, half * 64,
-                          hcoord, slot0, page, bar);
+              tma_load_3d(Qs + x * Geo::kTileBytes + half * Geo::kHalfBytes, &qmap, half * 64,
+                          w.hq0 + x, w.tile.t0 + w.tile.q_start, q_full);
+          ++q_iter;
+        }
+        const int32_t* bt_row =
+            p.kv.layout == 0
+                ? p.kv.block_table + (size_t)w.tile.seq * p.kv.max_blocks
+                : p.kv.block_table +
+                      ((size_t)w.tile.seq * p.kv.num_kv_heads + w.h) * p.kv.max_blocks;
+        const int hcoord = p.kv.layout == 0 ? w.h : 0;
+        const int box_rows = P < kKeys ? P : kKeys;
+        const uint32_t box_bytes = (uint32_t)box_rows * 128u * Geo::kHalves;
+        for (int j = 0; !stop && j < w.n_tiles; ++j) {
+          const int it = kv_iter++;
+          int nbox, first_blk = 0, slot0 = 0;
+          if (w.table) {
+            nbox = min(kKeys >> log2P, w.n_entries - j * (kKeys >> log2P));
+          } else if (P >= kKeys) {
+            nbox = 1;
+            first_blk = (j * kKeys) >> log2P;
+            slot0 = (j * kKeys) & (P - 1);
+          } else {
+            first_blk = (j * kKeys) >> log2P;
+            nbox = ((min(j * kKeys + kKeys, w.kv_hi) - 1) >> log2P) - first_blk + 1;
           }
-          issued[kv] = j + 1;
+          // K first (S needs it first), then V; each waits for its own slot to be released
+          for (int kv = 0; kv < 2; ++kv) {
+            const int ns = kv == 0 ? kStagesK : kStagesV;
+            const int slot = it % ns;
+            uint64_t* empty = kv == 0 ? &k_empty[slot] : &v_empty[slot];
+            if (it >= ns && !wait_bounded(empty, ((it / ns) - 1) & 1, abort_flag, p.err,
+                                          kErrPrefillWait)) {
+              stop = true;
+              break;
+            }
+            mbar_arrive_expect_tx(kv == 0 ? &k_full[slot] : &v_full[slot], box_bytes * nbox);
+            uint8_t* dst_base = (kv == 0 ? Ks : Vs) + slot * Geo::kTileBytes;
+            const CUtensorMap* map = kv == 0 ? &kmap : &vmap;
+            uint64_t* bar = kv == 0 ? &k_full[slot] : &v_full[slot];
+            for (int i = 0; i < nbox; ++i) {
+              const int blk =
+                  w.table ? __ldg(w.table + j * (kKeys >> log2P) + i) : first_blk + i;
+              int page = -1;  // out-of-range coordinates make TMA fill zeros: no stray access
+              if (blk >= 0 && blk < p.kv.max_blocks)
+                page = __ldg(bt_row + blk);
+              else if (kv == 0)
+                atomicOr(p.err, kErrBadIndex);
+#pragma unroll
+              for (int half = 0; half < Geo::kHalves; ++half)
+                tma_load_4d(dst_base + half * Geo::kHalfBytes + i * box_rows * 128, map,
+                            half * 64, hcoord, slot0, page, bar);
+            }
+            issued[kv] = it + 1;
+          }
         }
-        if (stop) break;
       }
-      if (*abort_flag) {
-        // let copies in flight land before shared memory goes away (time-bounded only: the
-        // raised abort flag must not cut these waits short)
-        wait_bounded(q_full, 0, never, nullptr, 0, kWaitTimeoutNs / 8);
-        for (int kv = 0; kv < 2; ++kv) {
-          const int ns = kv == 0 ? kStagesK : kStagesV;
-          for (int j = max(0, issued[kv] - ns); j < issued[kv]; ++j)
-            wait_bounded(kv == 0 ? &k_full[j % ns] : &v_full[j % ns], (j / ns) & 1, never,
-                         nullptr, 0, kWaitTimeoutNs / 8);
-        }
+      stop = __shfl_sync(0xffffffffu, stop, 0);
+    }
+    if (lane == 0 && *abort_flag) {
+      // let copies in flight land before shared memory goes away (time-bounded only: the
+      // raised abort flag must not cut these waits short)
+      if (q_iter > 0)
+        wait_bounded(q_full, (q_iter - 1) & 1, never, nullptr, 0, kWaitTimeoutNs / 8);
+      for (int kv = 0; kv < 2; ++kv) {
+        const int ns = kv == 0 ? kStagesK : kStagesV;
+        for (int i = max(0, issued[kv] - ns); i < issued[kv]; ++i)
+          wait_bounded(kv == 0 ? &k_full[i % ns] : &v_full[i % ns], (i / ns) & 1, never,
+                       nullptr, 0, kWaitTimeoutNs / 8);
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    if (n_tiles > 0) {
-      constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKeys, false, false);
-      constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
-      // Descriptors are built once; an MMA's operands differ from the base only in the start
-      // address field (bits 0..13, in 16-byte units, no carry for addresses below 256 KB), so
-      // each MMA needs one add per operand instead of rebuilding a 64-bit descriptor.
-      const uint64_t dq0 = smem_desc_sw128(smem_u32(Qs), 16, 1024);
-      const uint64_t dk0 = smem_desc_sw128(smem_u32(Ks), 16, 1024);
-      const uint64_t dv0 = smem_desc_sw128(smem_u32(Vs), Geo::kHalfBytes, 1024);
-      auto issue_s = [&](int x, int j) {  // S_x = Q_x K_j^T into TMEM columns [128x, +128)
-        const uint32_t a_lo = (uint32_t)dq0 + (uint32_t)((x * Geo::kTileBytes) >> 4);
-        const uint32_t b_lo =
-            (uint32_t)dk0 + (uint32_t)(((j % kStagesK) * Geo::kTileBytes) >> 4);
-        const uint32_t a_hi = (uint32_t)(dq0 >> 32), b_hi = (uint32_t)(dk0 >> 32);
-        const uint32_t d = tmem + x * 128;
+    constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKeys, false, false);
+    constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+    // Descriptors are built once; an MMA's operands differ from the base only in the start
+    // address field (bits 0..13, in 16-byte units, no carry for addresses below 256 KB), so
+    // each MMA needs one add per operand instead of rebuilding a 64-bit descriptor.
+    const uint64_t dq0 = smem_desc_sw128(smem_u32(Qs), 16, 1024);
+    const uint64_t dk0 = smem_desc_sw128(smem_u32(Ks), 16, 1024);
+    const uint64_t dv0 = smem_desc_sw128(smem_u32(Vs), Geo::kHalfBytes, 1024);
+    auto issue_s = [&](int x, int it) {  // S_x = Q_x K^T (K tile `it`) into TMEM [128x, +128)
+      const uint32_t a_lo = (uint32_t)dq0 + (uint32_t)((x * Geo::kTileBytes) >> 4);
+      const uint32_t b_lo =
+          (uint32_t)dk0 + (uint32_t)(((it % kStagesK) * Geo::kTileBytes) >> 4);
+      const uint32_t a_hi = (uint32_t)(dq0 >> 32), b_hi = (uint32_t)(dk0 >> 32);
+      const uint32_t d = tmem + x * 128;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (uint32_t)(((kk >> 2) * Geo::kHalfBytes + (kk & 3) * 32) >> 4);
-          if (kk == 0) umma_ss_lh<0>(d, a_lo + off, a_hi, b_lo + off, b_hi, idesc_s);
-          else umma_ss_lh<1>(d, a_lo + off, a_hi, b_lo + off, b_hi, idesc_s);
-        }
-        umma_commit(&s_full[x]);
-      };
-      auto issue_o = [&](int x, int j) {  // O_x += P_x V_j
-        const uint32_t b_lo =
-            (uint32_t)dv0 + (uint32_t)(((j % kStagesV) * Geo::kTileBytes) >> 4);
-        const uint32_t b_hi = (uint32_t)(dv0 >> 32);
-        const uint32_t d = tmem + 256 + x * 128;
-        const uint32_t a = tmem + x * 128;
-        const uint32_t acc0 = j > 0 ? 1u : 0u;
+      for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t off = (uint32_t)(((kk >> 2) * Geo::kHalfBytes + (kk & 3) * 32) >> 4);
+        if (kk == 0) umma_ss_lh<0>(d, a_lo + off, a_hi, b_lo + off, b_hi, idesc_s);
+        else umma_ss_lh<1>(d, a_lo + off, a_hi, b_lo + off, b_hi, idesc_s);
+      }
+      umma_commit(&s_full[x]);
+    };
+    auto issue_o = [&](int x, int it, bool first) {  // O_x (+)= P_x V (V tile `it`)
+      const uint32_t b_lo =
+          (uint32_t)dv0 + (uint32_t)(((it % kStagesV) * Geo::kTileBytes) >> 4);
+      const uint32_t b_hi = (uint32_t)(dv0 >> 32);
+      const uint32_t d = tmem + 256 + x * 128;
+      const uint32_t a = tmem + x * 128;
+      const uint32_t acc0 = first ? 0u : 1u;
 #pragma unroll
-        for (int kk = 0; kk < kKeys / 16; ++kk)
-          umma_ts_lh(d, a + kk * 8, b_lo + (uint32_t)((kk * 2048) >> 4), b_hi, idesc_o,
-                     kk > 0 ? 1u : acc0);
-        umma_commit(&o_done[x]);
-      };
-      bool ok = warp_wait_bounded(q_full, 0, abort_flag, p.err, kErrPrefillWait) &&
-                warp_wait_bounded(&k_full[0], 0, abort_flag, p.err, kErrPrefillWait);
-      if (ok && lane == 0) {
+      for (int kk = 0; kk < kKeys / 16; ++kk)
+        umma_ts_lh(d, a + kk * 8, b_lo + (uint32_t)((kk * 2048) >> 4), b_hi, idesc_o,
+                   kk > 0 ? 1u : acc0);
+      umma_commit(&o_done[x]);
+    };
+    bool ok = true;
+    int kv_iter = 0;  // K/V tiles consumed, over all units of this CTA
+    int q_iter = 0;   // units with key tiles
+    for (int k = 0; ok; ++k) {
+      const int u = unit_index(k);
+      if (u >= num_units) break;
+      const Unit w = unit_at(u);
+      if (w.n_tiles == 0) continue;
+      // The unit's first S goes in as soon as its Q and first K tile are in: the softmax
+      // warps are still writing out the previous unit's O (the first P.V of this unit, which
+      // overwrites O, waits for their P, which they produce only after that).
+      ok = warp_wait_bounded(q_full, q_iter & 1, abort_flag, p.err, kErrPrefillWait) &&
+           warp_wait_bounded(&k_full[kv_iter % kStagesK], (kv_iter / kStagesK) & 1,
+                             abort_flag, p.err, kErrPrefillWait);
+      ++q_iter;
+      if (!ok) break;
+      if (lane == 0) {
         tc_fence_after();
-        for (int x = 0; x < hpc; ++x) issue_s(x, 0);
-        umma_commit(&k_empty[0]);  // K_0 is free once both S MMAs finish
+        for (int x = 0; x < hpc; ++x) issue_s(x, kv_iter);
+        umma_commit(&k_empty[kv_iter % kStagesK]);  // free once both S MMAs finish
+        if (w.n_tiles == 1) umma_commit(q_empty);    // the unit's last S
       }
       __syncwarp();
-      for (int j = 0; ok && j < n_tiles; ++j) {
-        const int slot = j % kStagesV;
-        if (!warp_wait_bounded(&v_full[slot], (j / kStagesV) & 1, abort_flag, p.err,
-                               kErrPrefillWait))
+      for (int j = 0; ok && j < w.n_tiles; ++j) {
+        const int it = kv_iter + j;
+        const int slot = it % kStagesV;
+        if (!warp_wait_bounded(&v_full[slot], (it / kStagesV) & 1, abort_flag, p.err,
+                               kErrPrefillWait)) {
+          ok = false;
           break;
+        }
         // V rows past the last real key may hold anything (NaN tail slots, a stale tile):
         // P = 0 there does not cancel a NaN in the product, so the rows are zeroed.
         int nvalid;
-        if (table) {
+        if (w.table) {
           const int per = kKeys >> log2P;
-          const int ne = min(per, n_entries - j * per);
-          const int last = __ldg(table + j * per + ne - 1);
-          nvalid = (ne - 1) * P + min(P, tile.kv_len - (last << log2P));
+          const int ne = min(per, w.n_entries - j * per);
+          const int last = __ldg(w.table + j * per + ne - 1);
+          nvalid = (ne - 1) * P + min(P, w.tile.kv_len - (last << log2P));
         } else {
-          const int covered = min(tile.kv_len, ((kv_hi + P - 1) >> log2P) << log2P);
+          const int covered = min(w.tile.kv_len, ((w.kv_hi + P - 1) >> log2P) << log2P);
           nvalid = min(kKeys, covered - j * kKeys);
         }
         if (nvalid < kKeys) {
@@ -351,246 +417,264 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         // per head: O_x += P_x V_j as soon as P_x is ready, then S_x for the next tile (it
         // overwrites P_x in TMEM, so it must follow the P.V MMA, which tcgen05 keeps in order)
-        const bool more = j + 1 < n_tiles;
-        const int nslot = (j + 1) % kStagesK;
+        const bool more = j + 1 < w.n_tiles;
+        const int nslot = (it + 1) % kStagesK;
         for (int x = 0; x < hpc; ++x) {
-          if (!warp_wait_bounded(&p_ready[x], j & 1, abort_flag, p.err, kErrPrefillWait)) {
+          if (!warp_wait_bounded(&p_ready[x], it & 1, abort_flag, p.err, kErrPrefillWait)) {
             ok = false;
             break;
           }
           if (lane == 0) {
             tc_fence_after();
-            issue_o(x, j);
+            issue_o(x, it, j == 0);
             if (x == hpc - 1) umma_commit(&v_empty[slot]);
           }
           __syncwarp();
           if (more) {
-            if (!warp_wait_bounded(&k_full[nslot], ((j + 1) / kStagesK) & 1, abort_flag, p.err,
-                                   kErrPrefillWait)) {
+            if (!warp_wait_bounded(&k_full[nslot], ((it + 1) / kStagesK) & 1, abort_flag,
+                                   p.err, kErrPrefillWait)) {
               ok = false;
               break;
             }
             if (lane == 0) {
               tc_fence_after();
-              issue_s(x, j + 1);
-              if (x == hpc - 1) umma_commit(&k_empty[nslot]);
+              issue_s(x, it + 1);
+              if (x == hpc - 1) {
+                umma_commit(&k_empty[nslot]);
+                if (j + 2 == w.n_tiles) umma_commit(q_empty);  // the unit's last S
+              }
             }
             __syncwarp();
           }
         }
-        if (!ok) break;
       }
-      // every MMA issued so far must finish before TMEM is released
-      if (lane == 0) umma_commit(mma_done);
-      __syncwarp();
-      warp_wait_bounded(mma_done, 0, never, nullptr, 0, kWaitTimeoutNs / 8);
+      kv_iter += w.n_tiles;
     }
+    // every MMA issued so far must finish before TMEM is released
+    if (lane == 0) umma_commit(mma_done);
+    __syncwarp();
+    warp_wait_bounded(mma_done, 0, never, nullptr, 0, kWaitTimeoutNs / 8);
   }
   } else if ((warp - 4) / 4 < hpc) {
     // ------------------------------------------------------------------ softmax (head x)
     regs_alloc<kRegsSoftmax>();
     const int x = (warp - 4) / 4;
-    const int hq = hq0 + x;
     const int wq = warp & 3;                        // TMEM lane quarter of this warp
     const int r = wq * 32 + lane;                   // query row == TMEM lane
     const uint32_t lane_off = (uint32_t)(wq * 32) << 16;
     const uint32_t ts = tmem + x * 128 + lane_off;
     const uint32_t to = tmem + 256 + x * 128 + lane_off;
-    const int q_local = tile.q_start + r;
-    const int pos = past + q_local;                 // absolute position of this row
-    const int lim = p.causal ? min(tile.kv_len, pos + 1) : tile.kv_len;
-    const float sc = p.k_scale ? p.scale_log2 * __ldg(p.k_scale + h) : p.scale_log2;
-    float m_ref = -CUDART_INF_F, l = 0.f;
     bool ok = true;
-    for (int j = 0; j < n_tiles; ++j) {
-      if (!warp_wait_bounded(&s_full[x], j & 1, abort_flag, p.err, kErrPrefillWait)) {
-        ok = false;
-        break;
-      }
-      tc_fence_after();
-      uint32_t sr[kKeys];
-#pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(ts + c * 32, sr + c * 32);
-      // first key position of each column group: dense -> j*128; sparse -> lane e holds the
-      // start of the tile's e-th table block (missing entries map past every limit)
-      int ent = j * kKeys;
-      int tile_last;  // last key position the tile may hold
-      bool partial = false;
-      if (table) {
-        const int per = kKeys >> log2P;
-        const int e0 = j * per;
-        const int ne = min(per, n_entries - e0);
-        ent = 0x3fff0000;
-        if (lane < ne) ent = __ldg(table + e0 + lane) << log2P;
-        tile_last = __shfl_sync(0xffffffffu, ent, ne - 1) + P - 1;
-        partial = ne < per;
-      } else {
-        tile_last = j * kKeys + kKeys - 1;
-      }
-      const bool need_mask = partial || tile_last >= tile.kv_len ||
-                             (p.causal && tile_last > past + tile.q_start);
-      tmem_wait_ld();
-      uint32_t vis[kKeys / 32];  // visibility bits (masked tiles only)
-      if (need_mask) {
-#pragma unroll
-        for (int w = 0; w < kKeys / 32; ++w) vis[w] = 0u;
-#pragma unroll
-        for (int c = 0; c < kKeys; ++c) {
-          const int kp = table ? __shfl_sync(0xffffffffu, ent, c >> log2P) + (c & (P - 1))
-                               : ent + c;
-          vis[c >> 5] |= (kp < lim ? 1u : 0u) << (c & 31);
-        }
-      }
-      // The reference max m_ref comes from the first tile in which the row sees a key; later
-      // tiles take P against it with no max pass, so P may exceed 1.  That costs no precision
-      // (fp32 and bf16 are relative formats) until a tile's row sum passes 2^64; such a tile,
-      // rare in practice, is redone once against its own max, with O and l rescaled.
-      bool need_max = m_ref == -CUDART_INF_F;
-      float fac = 1.f;
-      bool rescale = false;
-      float rs;
-#pragma unroll 1
-      for (int attempt = 0;; ++attempt) {
-        if (__any_sync(0xffffffffu, need_max)) {
-          // row max of scale*S over the visible columns: short trees of independent
-          // accumulators, not a 128-long dependency chain
-          float mx;
-          if (need_mask) {
-            float acc[8];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) acc[k] = -CUDART_INF_F;
-#pragma unroll
-            for (int c = 0; c < kKeys; ++c)
-              acc[c & 7] = fmaxf(acc[c & 7], (vis[c >> 5] >> (c & 31)) & 1u
-                                                 ? __uint_as_float(sr[c]) * sc
-                                                 : -CUDART_INF_F);
-            mx = fmaxf(fmaxf(fmaxf(acc[0], acc[1]), fmaxf(acc[2], acc[3])),
-                       fmaxf(fmaxf(acc[4], acc[5]), fmaxf(acc[6], acc[7])));
-          } else {
-            // scale*max(S) for a non-negative scale, scale*min(S) for a negative one;
-            // 3-input max/min: two new values per instruction, four accumulators
-            float acc[4];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) acc[k] = __uint_as_float(sr[k]);
-            if (sc >= 0.f) {
-#pragma unroll
-              for (int c = 4; c < kKeys; c += 2)
-                acc[(c >> 1) & 3] = fmax3(acc[(c >> 1) & 3], __uint_as_float(sr[c]),
-                                          __uint_as_float(sr[c + 1]));
-              mx = fmaxf(fmax3(acc[0], acc[1], acc[2]), acc[3]) * sc;
-            } else {
-#pragma unroll
-              for (int c = 4; c < kKeys; c += 2)
-                acc[(c >> 1) & 3] = fmin3(acc[(c >> 1) & 3], __uint_as_float(sr[c]),
-                                          __uint_as_float(sr[c + 1]));
-              mx = fminf(fmin3(acc[0], acc[1], acc[2]), acc[3]) * sc;
-            }
-          }
-          if (need_max && mx > m_ref) {  // mx = -inf: still no visible key
-            if (m_ref != -CUDART_INF_F) {
-              fac = fast_exp2(m_ref - mx);
-              rescale = true;
-            }
-            m_ref = mx;
-          }
-        }
-        const float neg_m = m_ref == -CUDART_INF_F ? 0.f : -m_ref;
-        // P = exp2(scale*S - m): one packed FFMA per pair of elements and one EX2 per
-        // element; the row sum is kept in four packed partial sums
-        const uint64_t sc2 = f2_pack(sc, sc);
-        const uint64_t nm2 = f2_pack(neg_m, neg_m);
-        uint64_t rsum2[4];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) rsum2[k] = 0ull;
-#pragma unroll
-        for (int c = 0; c < kKeys; c += 2) {
-          float t0, t1;
-          f2_unpack(
-              f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2), t0,
-              t1);
-          float p0 = fast_exp2(t0);
-          float p1 = fast_exp2(t1);
-          if (need_mask) {
-            p0 = (vis[c >> 5] >> (c & 31)) & 1u ? p0 : 0.f;
-            p1 = (vis[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u ? p1 : 0.f;
-          }
-          rsum2[(c >> 1) & 3] = f2_add(rsum2[(c >> 1) & 3], f2_pack(p0, p1));
-          sr[c >> 1] = pack_bf16(p0, p1);  // P as bf16 pairs, over the consumed S values
-        }
-        rs = 0.f;
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          float a, b;
-          f2_unpack(rsum2[k], a, b);
-          rs += a + b;
-        }
-        const bool over = !(rs <= kMaxTileSum);
-        if (attempt > 0 || !__any_sync(0xffffffffu, over)) break;
-        need_max = over;
-#pragma unroll
-        for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(ts + c * 32, sr + c * 32);
-        tmem_wait_ld();
-      }
-      l = l * fac + rs;
-#pragma unroll
-      for (int c = 0; c < kKeys / 64; ++c) tmem_st32(ts + c * 32, sr + c * 32);
-      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-        // O += P V of the previous tile must be complete before O is rescaled
-        if (!warp_wait_bounded(&o_done[x], (j - 1) & 1, abort_flag, p.err, kErrPrefillWait)) {
+    int it0 = 0;  // S tiles of this head before the current unit
+    for (int k = 0; ok; ++k) {
+      const int u = unit_index(k);
+      if (u >= num_units) break;
+      const Unit w = unit_at(u);
+      const PrefillTile& tile = w.tile;
+      const int32_t* table = w.table;
+      const int n_entries = w.n_entries;
+      const int n_tiles = w.n_tiles;
+      const int past = w.past;
+      const int h = w.h;
+      const int hq = w.hq0 + x;
+      const int q_local = tile.q_start + r;
+      const int pos = past + q_local;                 // absolute position of this row
+      const int lim = p.causal ? min(tile.kv_len, pos + 1) : tile.kv_len;
+      const float sc = p.k_scale ? p.scale_log2 * __ldg(p.k_scale + h) : p.scale_log2;
+      float m_ref = -CUDART_INF_F, l = 0.f;
+      for (int j = 0; j < n_tiles; ++j) {
+        if (!warp_wait_bounded(&s_full[x], (it0 + j) & 1, abort_flag, p.err,
+                               kErrPrefillWait)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        uint32_t sr[kKeys];
+#pragma unroll
+        for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(ts + c * 32, sr + c * 32);
+        // first key position of each column group: dense -> j*128; sparse -> lane e holds the
+        // start of the tile's e-th table block (missing entries map past every limit)
+        int ent = j * kKeys;
+        int tile_last;  // last key position the tile may hold
+        bool partial = false;
+        if (table) {
+          const int per = kKeys >> log2P;
+          const int e0 = j * per;
+          const int ne = min(per, n_entries - e0);
+          ent = 0x3fff0000;
+          if (lane < ne) ent = __ldg(table + e0 + lane) << log2P;
+          tile_last = __shfl_sync(0xffffffffu, ent, ne - 1) + P - 1;
+          partial = ne < per;
+        } else {
+          tile_last = j * kKeys + kKeys - 1;
+        }
+        const bool need_mask = partial || tile_last >= tile.kv_len ||
+                               (p.causal && tile_last > past + tile.q_start);
+        tmem_wait_ld();
+        uint32_t vis[kKeys / 32];  // visibility bits (masked tiles only)
+        if (need_mask) {
+#pragma unroll
+          for (int w = 0; w < kKeys / 32; ++w) vis[w] = 0u;
+#pragma unroll
+          for (int c = 0; c < kKeys; ++c) {
+            const int kp = table ? __shfl_sync(0xffffffffu, ent, c >> log2P) + (c & (P - 1))
+                                 : ent + c;
+            vis[c >> 5] |= (kp < lim ? 1u : 0u) << (c & 31);
+          }
+        }
+        // The reference max m_ref comes from the first tile in which the row sees a key; later
+        // tiles take P against it with no max pass, so P may exceed 1.  That costs no precision
+        // (fp32 and bf16 are relative formats) until a tile's row sum passes 2^64; such a tile,
+        // rare in practice, is redone once against its own max, with O and l rescaled.
+        bool need_max = m_ref == -CUDART_INF_F;
+        float fac = 1.f;
+        bool rescale = false;
+        float rs;
+#pragma unroll 1
+        for (int attempt = 0;; ++attempt) {
+          if (__any_sync(0xffffffffu, need_max)) {
+            // row max of scale*S over the visible columns: short trees of independent
+            // accumulators, not a 128-long dependency chain
+            float mx;
+            if (need_mask) {
+              float acc[8];
+#pragma unroll
+              for (int k = 0; k < 8; ++k) acc[k] = -CUDART_INF_F;
+#pragma unroll
+              for (int c = 0; c < kKeys; ++c)
+                acc[c & 7] = fmaxf(acc[c & 7], (vis[c >> 5] >> (c & 31)) & 1u
+                                                   ? __uint_as_float(sr[c]) * sc
+                                                   : -CUDART_INF_F);
+              mx = fmaxf(fmaxf(fmaxf(acc[0], acc[1]), fmaxf(acc[2], acc[3])),
+                         fmaxf(fmaxf(acc[4], acc[5]), fmaxf(acc[6], acc[7])));
+            } else {
+              // scale*max(S) for a non-negative scale, scale*min(S) for a negative one;
+              // 3-input max/min: two new values per instruction, four accumulators
+              float acc[4];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) acc[k] = __uint_as_float(sr[k]);
+              if (sc >= 0.f) {
+#pragma unroll
+                for (int c = 4; c < kKeys; c += 2)
+                  acc[(c >> 1) & 3] = fmax3(acc[(c >> 1) & 3], __uint_as_float(sr[c]),
+                                            __uint_as_float(sr[c + 1]));
+                mx = fmaxf(fmax3(acc[0], acc[1], acc[2]), acc[3]) * sc;
+              } else {
+#pragma unroll
+                for (int c = 4; c < kKeys; c += 2)
+                  acc[(c >> 1) & 3] = fmin3(acc[(c >> 1) & 3], __uint_as_float(sr[c]),
+                                            __uint_as_float(sr[c + 1]));
+                mx = fminf(fmin3(acc[0], acc[1], acc[2]), acc[3]) * sc;
+              }
+            }
+            if (need_max && mx > m_ref) {  // mx = -inf: still no visible key
+              if (m_ref != -CUDART_INF_F) {
+                fac = fast_exp2(m_ref - mx);
+                rescale = true;
+              }
+              m_ref = mx;
+            }
+          }
+          const float neg_m = m_ref == -CUDART_INF_F ? 0.f : -m_ref;
+          // P = exp2(scale*S - m): one packed FFMA per pair of elements and one EX2 per
+          // element; the row sum is kept in four packed partial sums
+          const uint64_t sc2 = f2_pack(sc, sc);
+          const uint64_t nm2 = f2_pack(neg_m, neg_m);
+          uint64_t rsum2[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) rsum2[k] = 0ull;
+#pragma unroll
+          for (int c = 0; c < kKeys; c += 2) {
+            float t0, t1;
+            f2_unpack(
+                f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2), t0,
+                t1);
+            float p0 = fast_exp2(t0);
+            float p1 = fast_exp2(t1);
+            if (need_mask) {
+              p0 = (vis[c >> 5] >> (c & 31)) & 1u ? p0 : 0.f;
+              p1 = (vis[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u ? p1 : 0.f;
+            }
+            rsum2[(c >> 1) & 3] = f2_add(rsum2[(c >> 1) & 3], f2_pack(p0, p1));
+            sr[c >> 1] = pack_bf16(p0, p1);  // P as bf16 pairs, over the consumed S values
+          }
+          rs = 0.f;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            float a, b;
+            f2_unpack(rsum2[k], a, b);
+            rs += a + b;
+          }
+          const bool over = !(rs <= kMaxTileSum);
+          if (attempt > 0 || !__any_sync(0xffffffffu, over)) break;
+          need_max = over;
+#pragma unroll
+          for (int c = 0; c < kKeys / 32; ++c) tmem_ld32(ts + c * 32, sr + c * 32);
+          tmem_wait_ld();
+        }
+        l = l * fac + rs;
+#pragma unroll
+        for (int c = 0; c < kKeys / 64; ++c) tmem_st32(ts + c * 32, sr + c * 32);
+        if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+          // O += P V of the previous tile must be complete before O is rescaled
+          if (!warp_wait_bounded(&o_done[x], (it0 + j - 1) & 1, abort_flag, p.err,
+                                 kErrPrefillWait)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(to + c * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * fac);
+            tmem_st32(to + c * 32, o);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_ready[x]);
+      }
+      // ---- epilogue: O / l -> bf16 (a row that saw no key gets 0 and lse = -inf)
+      if (ok && n_tiles > 0) {
+        ok = warp_wait_bounded(&o_done[x], (it0 + n_tiles - 1) & 1, abort_flag, p.err,
+                               kErrPrefillWait);
+        tc_fence_after();
+      }
+      if (ok) {
+        const int t = tile.t0 + q_local;
+        const bool write = q_local < tile.q_len;
+        uint16_t* orow = p.out + ((size_t)t * Hq + hq) * D;
+        const float inv = l > 0.f ? (p.v_scale ? __ldg(p.v_scale + h) : 1.f) / l : 0.f;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
-          tmem_ld32(to + c * 32, o);
-          tmem_wait_ld();
+          if (n_tiles > 0) {
+            tmem_ld32(to + c * 32, o);
+            tmem_wait_ld();
+          } else {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = __float_as_uint(__uint_as_float(o[i]) * fac);
-          tmem_st32(to + c * 32, o);
-        }
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&p_ready[x]);
-    }
-    // ---- epilogue: O / l -> bf16 (a row that saw no key gets 0 and lse = -inf)
-    if (ok && n_tiles > 0) {
-      ok = warp_wait_bounded(&o_done[x], (n_tiles - 1) & 1, abort_flag, p.err,
-                             kErrPrefillWait);
-      tc_fence_after();
-    }
-    if (ok) {
-      const int t = tile.t0 + q_local;
-      const bool write = q_local < tile.q_len;
-      uint16_t* orow = p.out + ((size_t)t * Hq + hq) * D;
-      const float inv = l > 0.f ? (p.v_scale ? __ldg(p.v_scale + h) : 1.f) / l : 0.f;
+            for (int i = 0; i < 32; ++i) o[i] = 0u;
+          }
+          if (write) {
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t o[32];
-        if (n_tiles > 0) {
-          tmem_ld32(to + c * 32, o);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int i = 0; i < 32; ++i) o[i] = 0u;
-        }
-        if (write) {
-#pragma unroll
-          for (int i = 0; i < 32; i += 8) {
-            U4 v;
-            v.x = pack_bf16(__uint_as_float(o[i + 0]) * inv, __uint_as_float(o[i + 1]) * inv);
-            v.y = pack_bf16(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
-            v.z = pack_bf16(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
-            v.w = pack_bf16(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-            *reinterpret_cast<U4*>(orow + c * 32 + i) = v;
+            for (int i = 0; i < 32; i += 8) {
+              U4 v;
+              v.x = pack_bf16(__uint_as_float(o[i + 0]) * inv, __uint_as_float(o[i + 1]) * inv);
+              v.y = pack_bf16(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
+              v.z = pack_bf16(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
+              v.w = pack_bf16(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
+              *reinterpret_cast<U4*>(orow + c * 32 + i) = v;
+            }
           }
         }
+        if (write && p.lse)
+          p.lse[(size_t)t * Hq + hq] =
+              l > 0.f ? (m_ref + fast_log2(l)) * 0.69314718055994531f : -CUDART_INF_F;
       }
-      if (write && p.lse)
-        p.lse[(size_t)t * Hq + hq] =
-            l > 0.f ? (m_ref + fast_log2(l)) * 0.69314718055994531f : -CUDART_INF_F;
+      it0 += n_tiles;
     }
   } else {
     regs_dealloc<kRegsControl>();  // head B's warpgroup when the group size is odd
@@ -617,7 +701,14 @@ cudaError_t launch_prefill(const PrefillLaunch& p, const PrefillTilesInline* inl
   if (e != cudaSuccess) return e;
   const int G = p.num_q_heads / p.num_kv_heads;
   const int hpc = (p.qtile_table == nullptr && (G & 1) == 0) ? 2 : 1;  // as in the kernel
-  const dim3 grid((unsigned)p.num_tiles * (unsigned)(p.num_q_heads / hpc));
+  // persistent: one CTA per SM at most (each holds all of an SM's TMEM)
+  int dev = 0, sms = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  const long units = (long)p.num_tiles * (p.num_q_heads / hpc);
+  const dim3 grid((unsigned)(units < sms ? units : sms));
   // the register rebalancing inside the kernel needs exactly the launch budget it was
   // written for; refuse to launch otherwise (a short budget would stall setmaxnreg.inc)
   {
