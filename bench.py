@@ -1083,7 +1083,7 @@ def main():
     if args.case is not None:
         if not torch.cuda.is_available():
             raise SystemExit("--case needs a CUDA device")
-        res = CASES[args.case](args.steps, args.warmup, load_peaks())
+        res = CASES[args.case](args.steps, args.warmup, load_peaks()[0])
         print(json.dumps({"case": args.case, **res}))
         return
     if args.impl == "reference":

@@ -15,6 +15,8 @@
 // group) -- the two heads share every K/V tile and the same causal mask.  A persistent CTA
 // holds one SM (all 512 TMEM columns) and walks its share of the units, so the next unit's Q,
 // K and V stream in, and its first S is computed, while the current unit's O is written out.
+// Beside a decode kernel (mixed batches, device-planned steps) the grid has one CTA per unit
+// instead, so that decode CTAs take SMs as units finish.
 // 384 threads:
 //   warp 0      TMA producer: both Q tiles of a unit, then K and V tiles of 128 keys, page by
 //               page (boxes of [min(P,128) slots x 64 dims], 128-byte swizzle), 2-stage ring;
@@ -151,6 +153,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int num_units = n_list * groups;
   const int P = p.kv.page_size;
   const int log2P = p.kv.log2_page;
+  if ((int)blockIdx.x >= num_units) return;  // no unit at all (device-planned step)
 
   // The CTA walks units in rounds of gridDim.x, left to right in even rounds and right to left
   // in odd ones: the list is sorted heaviest first, so the alternation evens out the SMs' load.
@@ -701,14 +704,19 @@ cudaError_t launch_prefill(const PrefillLaunch& p, const PrefillTilesInline* inl
   if (e != cudaSuccess) return e;
   const int G = p.num_q_heads / p.num_kv_heads;
   const int hpc = (p.qtile_table == nullptr && (G & 1) == 0) ? 2 : 1;  // as in the kernel
-  // persistent: one CTA per SM at most (each holds all of an SM's TMEM)
-  int dev = 0, sms = 0;
-  e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
+  // persistent: one CTA per SM at most (each holds all of an SM's TMEM); otherwise one CTA
+  // per unit, which the kernel's unit walk reduces to its first unit
   const long units = (long)p.num_tiles * (p.num_q_heads / hpc);
-  const dim3 grid((unsigned)(units < sms ? units : sms));
+  long ctas = units;
+  if (p.persistent) {
+    int dev = 0, sms = 0;
+    e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    if (ctas > sms) ctas = sms;
+  }
+  const dim3 grid((unsigned)ctas);
   // the register rebalancing inside the kernel needs exactly the launch budget it was
   // written for; refuse to launch otherwise (a short budget would stall setmaxnreg.inc)
   {

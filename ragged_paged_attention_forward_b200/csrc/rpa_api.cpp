@@ -908,6 +908,7 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     p.scale_log2 = scale_log2;
     p.out = static_cast<uint16_t*>(out);
     p.lse = lse;
+    p.persistent = fork ? 0 : 1;  // beside the decode kernel: one CTA per unit
     if (plan->opts.sparse == 2) {
       p.qtile_table = group_table;
       p.qtile_count = group_count;

@@ -154,6 +154,9 @@ struct PrefillLaunch {
   // of the codes: K = code * k_scale[h], V = code * v_scale[h]); null: 1
   const float* k_scale;
   const float* v_scale;
+  // 1: one CTA per SM walks the units (a launch that has the GPU to itself); 0: one CTA per
+  // unit, so that a decode kernel running beside it takes SMs as units finish
+  int32_t persistent;
   int* err;
   PagedKV kv;
 };
