@@ -268,3 +268,19 @@ def test_kv_e4m3_plan_option():
         with pytest.raises(api.RPAError) as ei:
             api.rpa_plan(**_shape(**bad), kv_e4m3=True)
         assert ei.value.status == status
+
+
+def test_e4m3_device_plan_runs_decode_rows_only():
+    # planner, decode (with the quantising write of its rows) and merge: no scatter, no copy,
+    # no tensor-core launch and no side stream
+    p = _device_plan(kv_e4m3=True)
+    assert p.info().launches_forward == 3
+    assert _device_plan().info().launches_forward == 5
+    with pytest.raises(api.RPAError) as e:
+        _device_plan(kv_e4m3=True, head_dim=64)
+    assert e.value.status == api.RPA_ERR_UNSUPPORTED
+    # e4m3 pools with a device plan made without the option are refused before device work
+    with pytest.raises(api.RPAError) as ei:
+        api.rpa_forward_kv8(_device_plan(), None, None, None, None, None, None, None, None,
+                            None, None, 0.1, None, None, None, stream=0)
+    assert ei.value.status == api.RPA_ERR_UNSUPPORTED
