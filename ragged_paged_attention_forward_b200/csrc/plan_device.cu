@@ -55,7 +55,7 @@ __device__ __forceinline__ void block_scan4(int (&v)[4], int (&total)[4],
     total[k] = warp_sums[31][k];
     v[k] = before + incl[k] - v[k];
   }
-  __syncthreads();  // warp_sums is reused by the next round
+  __syncthreads();  // warp_sums is reused by the next 1024 sequences
 }
 
 __global__ void __launch_bounds__(kPlanThreads) plan_device_kernel(PlanDeviceLaunch p) {
