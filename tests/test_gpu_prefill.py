@@ -236,3 +236,26 @@ def test_sparse_config_full_size_sampled():
     ref, ref_lse, _, _ = oracle_forward(b, group_table=rt, group_count=rc, rows=rows)
     assert_close(out, ref, rows=rows)
     assert_lse_close(lse, ref_lse, rows=rows)
+
+
+def test_sparse_persistent_walk_with_empty_units():
+    # 16 query tiles x 16 head pairs = 256 units over at most one CTA per SM, so CTAs walk
+    # several units.  The heads of KV groups 4-7 select only blocks from position 3072 on, so
+    # for them the first 8 tiles (rows before position 3072) have no key tile at all: those
+    # units produce zeros and lse = -inf, and come after units with work in a CTA's walk.
+    b = wl.ragged_batch([4096], [2048], 32, 8, 128, 64, seed=71, layout=wl.HEAD_MAJOR)
+    nqb, nkb = 2048 // 64, b.max_blocks
+    rng = np.random.default_rng(72)
+    mask = (rng.random((1, 32, nqb, nkb)) < 0.3).astype(np.uint8)
+    mask[..., 4096 // 64:] = 0     # no block past the sequence
+    mask[:, 16:, :, :48] = 0       # groups 4-7: blocks 48.. only (keys 3072..)
+    table, count = orc.build_group_tables(mask, 8)
+    out, lse, _, _, _ = run_forward(b, group_table=torch.from_numpy(table),
+                                    group_count=torch.from_numpy(count))
+    assert torch.all(out[:1024, 16:] == 0)
+    assert torch.all(torch.isneginf(lse[:1024, 16:]))
+    rows = sorted(set(_sample_rows(b, 24, seed=73)) |
+                  {(t, h) for t in (0, 1023, 1024, 1500, 2047) for h in (0, 15, 16, 31)})
+    ref, ref_lse, _, _ = oracle_forward(b, group_table=table, group_count=count, rows=rows)
+    assert_close(out, ref, rows=rows)
+    assert_lse_close(lse, ref_lse, rows=rows)
