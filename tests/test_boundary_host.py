@@ -284,3 +284,14 @@ def test_e4m3_device_plan_runs_decode_rows_only():
         api.rpa_forward_kv8(_device_plan(), None, None, None, None, None, None, None, None,
                             None, None, 0.1, None, None, None, stream=0)
     assert ei.value.status == api.RPA_ERR_UNSUPPORTED
+
+
+def test_plan_accepts_odd_group_sizes():
+    # G = 3: three rows per token on the decode kernel; a 40-token row (120 rows) goes to the
+    # tensor-core kernel, one query head per CTA
+    p = api.rpa_plan(**_shape(num_q_heads=12, num_kv_heads=4))
+    info = p.info()
+    assert info.num_prefill_tiles == 0 and info.num_decode_items >= 2
+    m = api.rpa_plan(**_shape(num_q_heads=12, num_kv_heads=4, num_tokens=41,
+                              cu_seqlens_q=[0, 1, 41], seq_lens_k=[40, 200])).info()
+    assert m.num_prefill_tiles == 1 and m.num_decode_items >= 1
