@@ -270,7 +270,8 @@ def rpa_forward_kv8(plan: Plan, q, k_new, v_new, k_pool, v_pool, k_scale, v_scal
                     block_table, cu_seqlens_q, seq_lens_k, scale: float, out, lse, workspace,
                     stream=None):
     """The fused step over e4m3 (uint8) K/V pools with fp32 per-KV-head scales
-    k_scale, v_scale [Hkv] (decode-class plans, head_dim 128; see include/rpa.h)."""
+    k_scale, v_scale [Hkv] (head_dim 128, no group tables).  Plans with rows for the
+    tensor-core kernel, and device plans, must be made with kv_e4m3=True; see include/rpa.h."""
     nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("rpa_forward_kv8", lib().rpa_forward_kv8(
         plan.handle, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool),
