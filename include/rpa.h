@@ -294,16 +294,16 @@ RPA_API rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new
  *                     the e4m3 code nearest to fp32(x) / scale (IEEE fp32 division; ties to
  *                     the even code; magnitudes past 448 saturate to +-448).
  *   the rest          as for rpa_forward (no group tables).
- * Supported: head_dim 128, no group tables; device plans (rpa_plan_device) made with
- * opts.kv_e4m3 = 1 run decode rows only -- a row too long for the decode kernel is refused
- * with bit 16 of the device error word -- so a decode step over e4m3 pools can be captured
- * in a CUDA graph.  Rows for the split-KV decode kernel
- * read the e4m3 pools directly: scores and P.V on f16 operands (e4m3 -> f16 is exact; q must
- * stay within f16's range, |q| < 65504), fp32 accumulation.  A plan with rows for the
+ * Supported: head_dim 128, no group tables.  Rows for the split-KV decode kernel read the
+ * e4m3 pools directly: scores and P.V on f16 operands (e4m3 -> f16 is exact; q must stay
+ * within f16's range, |q| < 65504), fp32 accumulation.  A host plan with rows for the
  * tensor-core kernel must be made with opts.kv_e4m3 = 1: after the write, those sequences'
  * context is copied to bf16 in the workspace (exactly: every e4m3 value is a bf16 value) and
  * the tensor-core kernel reads the copy with k_scale[h] folded into its score scale and
- * v_scale[h] into its output.  Anything else returns RPA_ERR_UNSUPPORTED.
+ * v_scale[h] into its output.  A device plan (rpa_plan_device) must be made with
+ * opts.kv_e4m3 = 1 and runs decode rows only -- a row too long for the decode kernel is
+ * refused with bit 16 of the device error word -- so a decode step over e4m3 pools can be
+ * captured in a CUDA graph.  Anything else returns RPA_ERR_UNSUPPORTED.
  */
 RPA_API rpa_status rpa_forward_kv8(rpa_plan_t plan, const void* q, const void* k_new,
                                    const void* v_new, void* k_pool, void* v_pool,
