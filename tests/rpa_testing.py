@@ -98,3 +98,60 @@ def assert_lse_close(lse_gpu, lse_ref, rows=None, tol=2e-3):
     d = np.abs(np.where(both_inf, 0.0, g) - np.where(both_inf, 0.0, r))
     assert np.all(np.isfinite(d)), "lse mismatch in -inf pattern"
     assert d.max() <= tol, f"lse max err {d.max():.3e}"
+
+
+# ------------------------------------------------------------------ e4m3 (fp8) KV cache
+
+def kv8_vmax(v_pool_codes, v_scale, block_table=None, layout=orc.SEQ_MAJOR) -> float:
+    """The largest |V| an e4m3 V pool holds: per KV head, the largest finite code magnitude
+    times that head's scale, maximised over the heads.  e4m3 magnitudes grow with the low
+    seven bits of the code (0x7F is NaN), so a histogram of those bits finds each head's
+    largest value.  A KV-head-major pool needs the block table to know which pages belong to
+    which head."""
+    codes = orc.codes8(v_pool_codes)
+    vs = np.asarray(v_scale, dtype=np.float64)
+    best = 0.0
+    for h in range(len(vs)):
+        if layout == orc.SEQ_MAJOR:
+            c = codes[:, :, h, :]
+        else:
+            pages = np.unique(orc.ints(block_table)[:, h, :])
+            c = codes[pages[(pages >= 0) & (pages < codes.shape[0])]]
+        hist = np.bincount(c.ravel() & np.uint8(0x7F), minlength=128)
+        hist[0x7F] = 0
+        if hist.any():
+            top = int(np.nonzero(hist)[0].max())
+            best = max(best, float(orc.e4m3_decode(np.array([top], np.uint8))[0]) * vs[h])
+    return best
+
+
+def kv8_output_errors(out, ref, vmax, rows=None):
+    """Check e4m3-cache attention against the fp64 oracle; returns (ok, max_ratio, mean_err).
+
+    Error model.  Scores are exact: e4m3 -> f16 and bf16 -> f16 are exact conversions, f16
+    products are exact in fp32, and the fp32 sums over D = 128 terms add a relative error far
+    below 2^-20.  The probabilities are rounded before P.V -- to f16 on the split-KV kernel
+    (relative 2^-11), to bf16 on the tensor-core kernel (relative 2^-9) -- and the output is
+    rounded to bf16 (relative 2^-9).  So a row's error is at most
+    2^-9 * sum_j w_j |v_j| + 2^-9 |o| <= 2^-9 * max|V| + 2^-9 |o|.  The pointwise bound
+    allowed is twice that, 2^-8 * (max|V| + |o|), with max|V| the largest value the batch's
+    V pool actually holds after the write (``kv8_vmax``).  The P rounding errors are
+    independent from key to key, so they average out: the mean absolute error must also meet
+    the bf16 tolerance's mean-abs criterion, TOL_MEAN."""
+    got = out.double().numpy() if isinstance(out, torch.Tensor) else np.asarray(out, np.float64)
+    if rows is not None:
+        it = np.array([r[0] for r in rows])
+        ih = np.array([r[1] for r in rows])
+        got, ref = got[it, ih], ref[it, ih]
+    if not np.all(np.isfinite(got)):
+        return False, float("inf"), float("inf")
+    err = np.abs(got - ref)
+    bound = 2.0 ** -8 * (vmax + np.abs(ref))
+    ratio = float((err / bound).max())
+    mean = float(err.mean())
+    return ratio <= 1.0 and mean <= TOL_MEAN, ratio, mean
+
+
+def assert_kv8_close(out, ref, vmax, rows=None):
+    ok, ratio, mean = kv8_output_errors(out, ref, vmax, rows)
+    assert ok, f"e4m3 attention: worst err/bound {ratio:.3f}, mean err {mean:.3e}"

@@ -692,3 +692,31 @@ def test_qtile_attention_equals_group_attention_on_the_unioned_mask():
     dense, _, _, _ = _oracle_forward(b)
     assert np.array_equal(o3[128:260, 0], dense[128:260, 0])   # tile 1: all blocks
     assert np.array_equal(o3[:, 1:], dense[:, 1:])
+
+
+def test_kv8_output_check_rejects_a_dropped_decode_split():
+    # The e4m3 attention check of the GPU tests must be able to fail.  Plant the mistake a
+    # broken split-KV merge would make -- the last key split of two sequences lost (keys from
+    # 256 of the 300-key sequence, from 768 of the 1025-key one) -- and require the check to
+    # reject it, while the exact result rounded to bf16 passes.
+    from tests.rpa_testing import kv8_output_errors, kv8_vmax
+    b = wl.ragged_batch([1, 17, 300, 1025, 64], [1] * 5, 32, 8, 128, 16, seed=916)
+    b8, ks, vs = wl.with_kv8_pools(b, seed=901)
+    ref, _, kp, vp = orc.forward_kv8(b8.q, b8.k_new, b8.v_new, b8.k_pool, b8.v_pool,
+                                     ks.numpy(), vs.numpy(), b8.block_table, b8.cu_seqlens_q,
+                                     b8.seq_lens_k, scale=b8.scale, causal=True,
+                                     page_size=16, layout=b8.layout)
+    vmax = kv8_vmax(vp, vs.numpy())
+    assert 1.0 < vmax < 10.0
+    exact = torch.from_numpy(ref).to(torch.bfloat16)
+    assert kv8_output_errors(exact, ref, vmax)[0]
+    # attention of tokens 2 and 3 over their first split only (same pages, shorter context)
+    cut, _ = orc.attention(b8.q, kp, vp, b8.block_table, b8.cu_seqlens_q,
+                           np.array([1, 17, 256, 768, 64], dtype=np.int32), scale=b8.scale,
+                           causal=True, page_size=16, layout=b8.layout, num_kv_heads=8,
+                           rows=[(t, h) for t in (2, 3) for h in range(32)],
+                           kv_scales=(ks.numpy(), vs.numpy()))
+    mutated = ref.copy()
+    mutated[2:4] = cut[2:4]
+    ok, ratio, mean = kv8_output_errors(torch.from_numpy(mutated).to(torch.bfloat16), ref, vmax)
+    assert not ok and ratio > 1.0 and mean > 2e-3, (ratio, mean)
