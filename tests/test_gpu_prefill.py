@@ -26,6 +26,19 @@ def _sample_rows(batch, n, seed):
     return sorted(rows)
 
 
+def _unit_rows(batch, units):
+    """Every row of whole tensor-core work units.  A unit is a 128-query tile of one sequence
+    and a pair of query heads of one KV group: ``(seq, local tile, first head)`` selects the
+    tile's rows (clipped to the sequence) for heads ``h0`` and ``h0 + 1``."""
+    cu = batch.cu_seqlens_q.tolist()
+    rows = set()
+    for b, tile, h0 in units:
+        lo, hi = tile * 128, min(cu[b + 1] - cu[b], tile * 128 + 128)
+        assert lo < hi, (b, tile)
+        rows.update((cu[b] + i, h) for i in range(lo, hi) for h in (h0, h0 + 1))
+    return sorted(rows)
+
+
 def test_prefill_small_no_past():
     b = wl.ragged_batch([200, 64], [200, 64], 8, 2, 128, 64, seed=51)
     ref, ref_lse, kp, vp = oracle_forward(b)
@@ -124,11 +137,21 @@ def test_prefill_page_permutation_gives_identical_output():
     assert torch.equal(o1, o2)
 
 
-def test_prefill_config_full_size_sampled():
+def test_prefill_config_full_size_whole_units():
+    # The prefill workload (4 x 4096 causal) in the launch the benchmark times: a persistent
+    # grid of one CTA per SM walking 2048 units (128-query tile x query-head pair) in rounds
+    # of the grid size, left to right, then right to left.  The planner sorts tiles heaviest
+    # first (stable), so list position p holds sequence p % 4, tile 31 - p // 4, and unit
+    # 16 p + pair.  Whole units are compared: the first, a middle and the last tile of every
+    # sequence, and units of the walk's first round (positions 0, 5) and second round
+    # (positions 9 and 13, pairs 8 and 3: units 152 and 211).
     b = wl.prefill()
     out, lse, gk, gv, plan = run_forward(b)
     assert plan.info().batch_class == api.CLASS_PREFILL
-    rows = _sample_rows(b, 96, seed=1)
+    units = [(s, 0, 2 * s) for s in range(4)] + [(s, 15, 8 + 2 * s) for s in range(4)] + \
+            [(s, 31, 16 + 2 * s) for s in range(4)] + \
+            [(0, 31, 0), (1, 30, 14), (1, 29, 16), (1, 28, 6)]
+    rows = _unit_rows(b, units)
     ref, ref_lse, kp, vp = oracle_forward(b, rows=rows)
     assert_close(out, ref, rows=rows)
     assert_lse_close(lse, ref_lse, rows=rows)
@@ -137,16 +160,26 @@ def test_prefill_config_full_size_sampled():
 
 
 @pytest.mark.parametrize("shuffle", [False, True])
-def test_mixed_config_full_size_sampled(shuffle):
+def test_mixed_config_full_size_whole_units(shuffle):
+    # The mixed workload: 48 decode rows (split-KV kernel) and chunks of 512 and 976 queries
+    # with past 1024 and 8192 (tensor-core kernel, one CTA per unit).  Whole units of both
+    # chunks -- first, middle and last tile, the 976-query chunk's last tile ragged (80 rows)
+    # -- and every query head of each decode row's KV group.
     b = wl.mixed(shuffle=shuffle)
     out, lse, _, _, plan = run_forward(b)
     info = plan.info()
     assert info.num_prefill_tiles > 0 and info.num_decode_items > 0
-    rows = _sample_rows(b, 96, seed=2)
-    # every decode row too (one head each)
     cu = b.cu_seqlens_q.tolist()
-    rows = sorted(set(rows) | {(cu[i], i % 32) for i in range(b.num_seqs)
-                                if cu[i + 1] - cu[i] == 1})
+    q_lens = [cu[i + 1] - cu[i] for i in range(b.num_seqs)]
+    c512, c976 = q_lens.index(512), q_lens.index(976)
+    units = [(c512, 0, 0), (c512, 1, 30), (c512, 3, 12),
+             (c976, 0, 4), (c976, 4, 18), (c976, 7, 0), (c976, 7, 26)]
+    rows = set(_unit_rows(b, units))
+    for i in range(b.num_seqs):
+        if q_lens[i] == 1:
+            g = i % 8
+            rows.update((cu[i], h) for h in range(4 * g, 4 * g + 4))
+    rows = sorted(rows)
     ref, ref_lse, _, _ = oracle_forward(b, rows=rows)
     assert_close(out, ref, rows=rows)
     assert_lse_close(lse, ref_lse, rows=rows)
@@ -221,7 +254,12 @@ def test_sparse_rows_without_visible_blocks():
     assert_lse_close(lse, ref_lse)
 
 
-def test_sparse_config_full_size_sampled():
+def test_sparse_config_full_size_whole_units():
+    # The sparse workload (2048 queries at 128K context, per-group tables) in the persistent
+    # launch: 16 tiles x 16 pairs = 256 units over 148 CTAs.  The list holds tile 15 - p at
+    # position p, unit 16 p + pair.  Whole units: the first of round one (tile 15, pair 0),
+    # a middle one (tile 8, pair 9), and two of round two (tile 6, pair 6 = unit 150; tile 0,
+    # pair 15 = unit 255, the last).
     b, mask = wl.sparse()
     m = mask.cuda()
     nkb = mask.shape[-1]
@@ -232,7 +270,7 @@ def test_sparse_config_full_size_sampled():
     rt, rc = orc.build_group_tables(mask, 8)
     assert np.array_equal(table.cpu().numpy(), rt) and np.array_equal(count.cpu().numpy(), rc)
     out, lse, _, _, _ = run_forward(b, group_table=table, group_count=count)
-    rows = _sample_rows(b, 24, seed=3)
+    rows = _unit_rows(b, [(0, 15, 0), (0, 8, 18), (0, 6, 12), (0, 0, 30)])
     ref, ref_lse, _, _ = oracle_forward(b, group_table=rt, group_count=rc, rows=rows)
     assert_close(out, ref, rows=rows)
     assert_lse_close(lse, ref_lse, rows=rows)
@@ -254,8 +292,54 @@ def test_sparse_persistent_walk_with_empty_units():
                                     group_count=torch.from_numpy(count))
     assert torch.all(out[:1024, 16:] == 0)
     assert torch.all(torch.isneginf(lse[:1024, 16:]))
+    # whole units, in list order (tile 15 - p at position p, unit 16 p + pair): round one
+    # with keys (tile 15, pair 8) and without (tile 7, pair 12 = unit 140); round two
+    # without keys (tile 6, pair 9 = unit 153) and with (tile 5, pair 2; tile 0, pair 0)
     rows = sorted(set(_sample_rows(b, 24, seed=73)) |
-                  {(t, h) for t in (0, 1023, 1024, 1500, 2047) for h in (0, 15, 16, 31)})
+                  set(_unit_rows(b, [(0, 15, 16), (0, 7, 24), (0, 6, 18), (0, 5, 4),
+                                     (0, 0, 0)])))
     ref, ref_lse, _, _ = oracle_forward(b, group_table=table, group_count=count, rows=rows)
     assert_close(out, ref, rows=rows)
     assert_lse_close(lse, ref_lse, rows=rows)
+
+
+# ------------------------------------------------------------------ odd GQA group sizes
+
+@pytest.mark.parametrize("layout", [wl.SEQ_MAJOR, wl.HEAD_MAJOR])
+@pytest.mark.parametrize("Hq,Hkv", [(12, 4), (40, 8)])
+def test_odd_group_size_mixed_batch(Hq, Hkv, layout):
+    # G = 3 and G = 5 (the WebGPU page's test list covers MHA and GQA variants): the
+    # tensor-core kernel then takes one query head per unit (a head pair must share a KV
+    # group), and the split-KV kernel packs G x q_len query rows of a group into its MMA's N.
+    b = wl.ragged_batch([1, 300, 777, 260, 2000], [1, 2, 1, 200, 150], Hq, Hkv, 128, 16,
+                        seed=97 + Hq, layout=layout)
+    ref, ref_lse, _, _ = oracle_forward(b)
+    out, lse, _, _, plan = run_forward(b)
+    info = plan.info()
+    assert info.num_decode_items > 0 and info.num_prefill_tiles > 0
+    assert_close(out, ref)
+    assert_lse_close(lse, ref_lse)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(12, 4), (40, 8)])
+def test_odd_group_size_prefill_persistent(Hq, Hkv):
+    # a prefill-only batch: the persistent grid walks one-head units
+    b = wl.ragged_batch([700, 1300, 129], [700, 600, 129], Hq, Hkv, 128, 64, seed=99 + Hq)
+    ref, ref_lse, kp, vp = oracle_forward(b)
+    out, lse, gk, gv, plan = run_forward(b)
+    assert plan.info().batch_class == api.CLASS_PREFILL
+    assert_close(out, ref)
+    assert_lse_close(lse, ref_lse)
+    assert np.array_equal(orc.bits16(gk), kp) and np.array_equal(orc.bits16(gv), vp)
+
+
+@pytest.mark.parametrize("Hq,Hkv", [(12, 4), (40, 8)])
+def test_odd_group_size_decode(Hq, Hkv):
+    b = wl.ragged_batch([1, 17, 300, 1025, 64], [1] * 5, Hq, Hkv, 128, 16, seed=101 + Hq)
+    ref, ref_lse, kp, vp = oracle_forward(b)
+    out, lse, gk, gv, plan = run_forward(b, plan_opts=dict(decode_split_keys=256))
+    info = plan.info()
+    assert info.batch_class == api.CLASS_DECODE and info.num_merge_rows > 0
+    assert_close(out, ref)
+    assert_lse_close(lse, ref_lse)
+    assert np.array_equal(orc.bits16(gk), kp) and np.array_equal(orc.bits16(gv), vp)
