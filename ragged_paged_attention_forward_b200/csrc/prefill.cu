@@ -33,6 +33,7 @@
 // TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+D) O_B [384,384+D).  Bounded waits.
 // An odd GQA group size runs with head B switched off.
 #include <cuda_bf16.h>
+#include <type_traits>
 #include <math_constants.h>
 
 #include "ptx.cuh"
@@ -580,27 +581,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const float neg_m = m_ref == -CUDART_INF_F ? 0.f : -m_ref;
           // P = exp2(scale*S - m): one packed FFMA per pair of elements and one EX2 per
-          // element; the row sum is kept in four packed partial sums
+          // element; the row sum is kept in four packed partial sums.  The loop exists twice:
+          // most tiles see every key and take the version without the visibility selects.
           const uint64_t sc2 = f2_pack(sc, sc);
           const uint64_t nm2 = f2_pack(neg_m, neg_m);
           uint64_t rsum2[4];
 #pragma unroll
           for (int k = 0; k < 4; ++k) rsum2[k] = 0ull;
+          auto exp_pass = [&](auto masked) {
+            constexpr bool kMasked = decltype(masked)::value;
 #pragma unroll
-          for (int c = 0; c < kKeys; c += 2) {
-            float t0, t1;
-            f2_unpack(
-                f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2, nm2), t0,
-                t1);
-            float p0 = fast_exp2(t0);
-            float p1 = fast_exp2(t1);
-            if (need_mask) {
-              p0 = (vis[c >> 5] >> (c & 31)) & 1u ? p0 : 0.f;
-              p1 = (vis[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u ? p1 : 0.f;
+            for (int c = 0; c < kKeys; c += 2) {
+              float t0, t1;
+              f2_unpack(f2_fma(f2_pack(__uint_as_float(sr[c]), __uint_as_float(sr[c + 1])), sc2,
+                               nm2),
+                        t0, t1);
+              float p0 = fast_exp2(t0);
+              float p1 = fast_exp2(t1);
+              if constexpr (kMasked) {
+                p0 = (vis[c >> 5] >> (c & 31)) & 1u ? p0 : 0.f;
+                p1 = (vis[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u ? p1 : 0.f;
+              }
+              rsum2[(c >> 1) & 3] = f2_add(rsum2[(c >> 1) & 3], f2_pack(p0, p1));
+              sr[c >> 1] = pack_bf16(p0, p1);  // P as bf16 pairs, over the consumed S values
             }
-            rsum2[(c >> 1) & 3] = f2_add(rsum2[(c >> 1) & 3], f2_pack(p0, p1));
-            sr[c >> 1] = pack_bf16(p0, p1);  // P as bf16 pairs, over the consumed S values
-          }
+          };
+          if (need_mask)
+            exp_pass(std::true_type{});
+          else
+            exp_pass(std::false_type{});
           rs = 0.f;
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
