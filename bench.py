@@ -1015,6 +1015,20 @@ def run_gpu(args):
             line["prefill_frac_of_bf16_peak"] = secondary["prefill"]["frac_of_bf16_peak"]
     line["peaks"] = dict(peaks, source=peak_src)
     line["hbm_frac"] = value / world / peaks["hbm_gbs"]
+    # one compact object last, so that the end of the line alone holds every workload's
+    # figures (attention time, throughput, fraction of the roofline)
+    summary = {name: {"attn_ms": round(attn_ms, 5), "roofline_frac": round(roof["frac"], 4)}}
+    for k, v in line.get("secondary", {}).items():
+        if "attn_ms" in v:
+            summary[k] = {"attn_ms": round(v["attn_ms"], 5),
+                          "roofline_frac": round(v.get("roofline_frac", float("nan")), 4),
+                          "TFLOPs": round(v["attn_TFLOPs"], 1), "GBps": round(v["attn_GBps"], 1)}
+        elif "ms_per_step" in v:
+            summary[k] = {"ms_per_step": round(v["ms_per_step"], 5)}
+            for key in ("frac_of_hbm", "union_ms", "blocksparse_ms"):
+                if key in v:
+                    summary[k][key] = round(v[key], 5)
+    line["summary"] = summary
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist:

@@ -90,7 +90,12 @@ typedef struct rpa_plan_options {
   int32_t kv_e4m3;             /* 1: the pools will hold e4m3 codes (rpa_forward_kv8): the   */
                                /* workspace also holds a bf16 copy of the context of rows  */
                                /* that go to the tensor-core kernel                        */
-  int32_t reserved[4];         /* must be zero                                             */
+  int32_t wait_test_us;        /* diagnostics, for tests of the bounded waits only: > 0    */
+                               /* makes the split-KV decode kernel load no K/V and give up */
+                               /* each of its waits after this many microseconds (at most  */
+                               /* 1000000), so rpa_forward computes no attention and sets  */
+                               /* bit 1 of the device error word; 0 for real work          */
+  int32_t reserved[3];         /* must be zero                                             */
 } rpa_plan_options;
 
 typedef struct rpa_plan_info {
@@ -333,6 +338,9 @@ RPA_API rpa_status rpa_forward_kv8(rpa_plan_t plan, const void* q, const void* k
  * or different host threads on one device) race and must be serialised by the caller.  The
  * array keeps the last call's contents; nothing in it needs to start at zero, because every
  * call rewrites its work lists and every partial result before reading them.
+ * The looked-up address is kept for the life of the process: after cudaDeviceReset (or any
+ * other teardown of the device's primary context) it is stale, so do not call this entry
+ * point on a device after resetting it.
  */
 #define RPA_NO_ALLOC_WORKSPACE_BYTES ((size_t)8 << 20)
 
@@ -342,6 +350,10 @@ RPA_API rpa_status rpa_forward_no_alloc(rpa_plan_t plan, const void* q, const vo
                                         const int32_t* seq_lens_k, const int32_t* group_table,
                                         const int32_t* group_count, float scale, void* out,
                                         float* lse, void* stream);
+
+/* The size of rpa_forward_no_alloc's built-in scratch, RPA_NO_ALLOC_WORKSPACE_BYTES, as
+ * compiled into the library (for bindings that do not read this header).  No CUDA call. */
+RPA_API size_t rpa_no_alloc_workspace_bytes(void);
 
 /*
  * rpa_build_group_tables -- block-union KV selection (CompactAttention, Core claim and
@@ -359,14 +371,6 @@ RPA_API rpa_status rpa_build_group_tables(const uint8_t* mask, int32_t num_seqs,
                                   int32_t num_kv_blocks, int32_t* table, int32_t* count,
                                   void* stream);
 
-/*
- * rpa_device_error -- read (and optionally clear) the library's device error word on the
- * current device.  Kernels never spin without bound: a wait that runs out records a code
- * here and the kernel returns early.  Synchronizes the device.  *code = 0 means no error;
- * otherwise an OR of: 1 decode wait ran out, 2 prefill wait ran out, 4 a page id outside
- * [0, num_pages) or a block index outside the table, 8 a position at or past the rotary
- * caches' max_position, 16 a device-planned step beyond its plan's limits.
- */
 /*
  * rpa_build_qtile_tables -- per-(query tile, query head) KV block tables: row (b, hq, tile)
  * lists, ascending, the KV blocks kb that head hq selects in any query block of the
@@ -388,6 +392,14 @@ RPA_API rpa_status rpa_build_qtile_tables(const uint8_t* mask, int32_t num_seqs,
                                           int32_t num_kv_blocks, int32_t q_block_rows,
                                           int32_t* table, int32_t* count, void* stream);
 
+/*
+ * rpa_device_error -- read (and optionally clear) the library's device error word on the
+ * current device.  Kernels never spin without bound: a wait that runs out records a code
+ * here and the kernel returns early.  Synchronizes the device.  *code = 0 means no error;
+ * otherwise an OR of: 1 decode wait ran out, 2 prefill wait ran out, 4 a page id outside
+ * [0, num_pages) or a block index outside the table, 8 a position at or past the rotary
+ * caches' max_position, 16 a device-planned step beyond its plan's limits.
+ */
 RPA_API rpa_status rpa_device_error(int32_t* code, int32_t clear);
 
 /* rpa_status_string -- static description of a status code. */

@@ -40,7 +40,7 @@ class Shape(ctypes.Structure):
 class PlanOptions(ctypes.Structure):
     _fields_ = [("force_class", ctypes.c_int32), ("decode_split_keys", ctypes.c_int32),
                 ("sparse", ctypes.c_int32), ("kv_e4m3", ctypes.c_int32),
-                ("reserved", ctypes.c_int32 * 4)]
+                ("wait_test_us", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3)]
 
 
 class PlanInfo(ctypes.Structure):
@@ -101,6 +101,8 @@ def lib() -> ctypes.CDLL:
         L.rpa_forward_no_alloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                            ctypes.c_float, _P, _P, _P]
         L.rpa_forward_no_alloc.restype = ctypes.c_int
+        L.rpa_no_alloc_workspace_bytes.argtypes = []
+        L.rpa_no_alloc_workspace_bytes.restype = ctypes.c_size_t
         L.rpa_rotary_write_kv.argtypes = [_P, _P, _P, _P, ctypes.POINTER(Rotary), _P, _P, _P,
                                           _P, _P, _P, _P]
         L.rpa_rotary_write_kv.restype = ctypes.c_int
@@ -205,11 +207,15 @@ class Plan:
 def rpa_plan(*, num_seqs: int, num_tokens: int, num_q_heads: int, num_kv_heads: int,
              head_dim: int, page_size: int, num_pages: int, max_blocks_per_seq: int,
              layout: int, causal: bool, cu_seqlens_q, seq_lens_k, force_class: int = 0,
-             decode_split_keys: int = 0, sparse=False, kv_e4m3: bool = False) -> Plan:
+             decode_split_keys: int = 0, sparse=False, kv_e4m3: bool = False,
+             wait_test_us: int = 0) -> Plan:
+    """wait_test_us > 0 is for tests of the bounded device waits only (see include/rpa.h):
+    the decode kernel then loads nothing and reports its waits running out."""
     shape = Shape(num_seqs, num_tokens, num_q_heads, num_kv_heads, head_dim, page_size,
                   num_pages, max_blocks_per_seq, layout, 1 if causal else 0)
     # sparse: False/0 none, True/1 per-group tables, 2 per-(query tile, query head) tables
-    opts = PlanOptions(force_class, decode_split_keys, int(sparse), 1 if kv_e4m3 else 0)
+    opts = PlanOptions(force_class, decode_split_keys, int(sparse), 1 if kv_e4m3 else 0,
+                       int(wait_test_us))
     handle = ctypes.c_void_p()
     ws = ctypes.c_size_t(0)
     _check("rpa_plan", lib().rpa_plan(ctypes.byref(shape), _host_i32(cu_seqlens_q),
@@ -279,7 +285,9 @@ def rpa_forward_kv8(plan: Plan, q, k_new, v_new, k_pool, v_pool, k_scale, v_scal
         ctypes.c_float(scale), _ptr(out), _ptr(lse), _ptr(workspace), nbytes, _stream(stream)))
 
 
-NO_ALLOC_WORKSPACE_BYTES = 8 << 20
+def no_alloc_workspace_bytes() -> int:
+    """Size of rpa_forward_no_alloc's built-in scratch, as compiled into the library."""
+    return int(lib().rpa_no_alloc_workspace_bytes())
 
 
 def rpa_forward_no_alloc(plan: Plan, q, k_new, v_new, k_pool, v_pool, block_table,

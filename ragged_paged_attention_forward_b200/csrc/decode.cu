@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
       asm volatile("fence.proxy.async.global;" ::: "memory");
       __syncwarp();
     }
-    if (lane == 0) {
+    if (lane == 0 && p.test_wait_ns == 0) {
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
       const int hcoord = p.kv.layout == 0 ? h : 0;
@@ -261,7 +261,7 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
     for (int s = 0; s < nstages; ++s) {
       const int slot = s % Geo::kStages;
       if (!warp_wait_bounded(&full[slot], (s / Geo::kStages) & 1, abort_flag, p.err,
-                             kErrDecodeWait))
+                             kErrDecodeWait, p.test_wait_ns ? p.test_wait_ns : kWaitTimeoutNs))
         break;
       const int key0 = it.k_begin + s * Geo::kStageKeys + warp * 16;
       if (key0 < it.k_end) {

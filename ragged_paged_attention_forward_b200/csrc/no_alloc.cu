@@ -82,3 +82,5 @@ extern "C" rpa_status rpa_forward_no_alloc(rpa_plan_t plan, const void* q, const
                      seq_lens_k, group_table, group_count, scale, out, lse, ws,
                      kStaticWorkspaceBytes, stream);
 }
+
+extern "C" size_t rpa_no_alloc_workspace_bytes(void) { return kStaticWorkspaceBytes; }

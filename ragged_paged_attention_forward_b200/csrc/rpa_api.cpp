@@ -180,8 +180,10 @@ rpa_status rpa_plan(const rpa_shape* shape, const int32_t* cu_seqlens_q,
   rpa_plan_options o;
   memset(&o, 0, sizeof(o));
   if (opts) o = *opts;
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 3; ++i)
     if (o.reserved[i] != 0) RPA_FAIL(RPA_ERR_INVALID_ARG, "plan option reserved[%d] != 0", i);
+  if (o.wait_test_us < 0 || o.wait_test_us > 1000000)
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "opts.wait_test_us %d must be in [0, 1000000]", o.wait_test_us);
   if (o.kv_e4m3 < 0 || o.kv_e4m3 > 1)
     RPA_FAIL(RPA_ERR_INVALID_ARG, "opts.kv_e4m3 %d must be 0 or 1", o.kv_e4m3);
   if (o.kv_e4m3 && s.head_dim != 128)
@@ -419,9 +421,12 @@ rpa_status rpa_plan_device(const rpa_shape* shape, int32_t max_kv_len,
   rpa_plan_options o;
   memset(&o, 0, sizeof(o));
   if (opts) o = *opts;
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 3; ++i)
     if (o.reserved[i] != 0) RPA_FAIL(RPA_ERR_INVALID_ARG, "plan option reserved[%d] != 0", i);
+  if (o.wait_test_us < 0 || o.wait_test_us > 1000000)
+    RPA_FAIL(RPA_ERR_INVALID_ARG, "opts.wait_test_us %d must be in [0, 1000000]", o.wait_test_us);
   if (o.sparse) RPA_FAIL(RPA_ERR_UNSUPPORTED, "device-planned steps take no group tables");
+  if (o.wait_test_us) RPA_FAIL(RPA_ERR_UNSUPPORTED, "opts.wait_test_us: host plans only");
   if (o.kv_e4m3 && s.head_dim != 128)
     RPA_FAIL(RPA_ERR_UNSUPPORTED, "e4m3 pools need head_dim 128 (got %d)", s.head_dim);
   if (o.force_class != RPA_CLASS_AUTO)
@@ -956,6 +961,7 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     d.v_pool_w = fused ? v_pool : nullptr;
     d.k_scale = k_scale;
     d.v_scale = v_scale;
+    d.test_wait_ns = (uint32_t)plan->opts.wait_test_us * 1000u;
     st = check_cuda(launch_decode(d, &plan->dec_inline, plan->decode_nt, stream), "decode launch");
     if (st != RPA_OK) return st;
     if (!plan->merge_rows.empty()) {

@@ -114,6 +114,9 @@ struct DecodeLaunch {
   // e4m3(fp32(x) / scale), nearest even, saturating
   const float* k_scale;      // [Hkv]
   const float* v_scale;      // [Hkv]
+  // diagnostics (tests of the bounded waits): nonzero = load no K/V and give up every wait
+  // after this many nanoseconds, so the waits run out and the kernel reports it
+  uint32_t test_wait_ns;
 };
 
 struct MergeLaunch {

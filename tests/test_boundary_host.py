@@ -27,6 +27,14 @@ def test_library_exports_every_declared_entry_point():
         assert hasattr(L, n), n
 
 
+def test_no_alloc_scratch_size_matches_the_header():
+    # the binding reads the size from the library; it must be the header's macro
+    text = open(os.path.join(ROOT, "include", "rpa.h")).read()
+    m = re.search(r"#define RPA_NO_ALLOC_WORKSPACE_BYTES \(\(size_t\)(\d+) << (\d+)\)", text)
+    assert m, "macro not found"
+    assert api.no_alloc_workspace_bytes() == int(m.group(1)) << int(m.group(2))
+
+
 def _shape(**kw):
     s = dict(num_seqs=2, num_tokens=2, num_q_heads=32, num_kv_heads=8, head_dim=128,
              page_size=16, num_pages=100, max_blocks_per_seq=16, layout=0, causal=True,
@@ -51,6 +59,8 @@ def _shape(**kw):
     (dict(sparse=True), api.RPA_ERR_UNSUPPORTED),                      # sparse needs head-major
     (dict(decode_split_keys=100), api.RPA_ERR_INVALID_ARG),
     (dict(force_class=7), api.RPA_ERR_INVALID_ARG),
+    (dict(wait_test_us=-1), api.RPA_ERR_INVALID_ARG),
+    (dict(wait_test_us=1000001), api.RPA_ERR_INVALID_ARG),
 ])
 def test_plan_rejects(kw, status):
     with pytest.raises(api.RPAError) as ei:

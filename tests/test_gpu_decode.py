@@ -149,3 +149,33 @@ def test_group_tables_bit_exact_vector_path(nkb, nqb, density):
     t, c = _tables_on_gpu(mask, 4)
     rt, rc = orc.build_group_tables(mask, 4)
     assert np.array_equal(t, rt) and np.array_equal(c, rc)
+
+
+def test_bounded_wait_runs_out_reports_and_leaves_the_context_usable():
+    # Failure detection without a GPU fault: with the diagnostic plan option the decode
+    # kernel issues no K/V copy, so its consumers' waits on the copies can only run out.  They
+    # give up after 2 ms (not the normal 2 s), record bit 1 in the device error word and the
+    # kernel returns; nothing is left in flight.  The next normal step on the same context
+    # must be correct.
+    import time
+    b = wl.ragged_batch([300, 1025, 64], [1, 1, 1], 32, 8, 128, 16, seed=111)
+    assert api.rpa_device_error(clear=True) == 0
+    plan = plan_for(b, wait_test_us=2000)
+    assert plan.info().batch_class == api.CLASS_DECODE
+    d = to_device(b)
+    out = torch.zeros_like(d["q"])
+    ws = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    t0 = time.perf_counter()
+    api.rpa_forward(plan, d["q"], d["k_new"], d["v_new"], d["k_pool"], d["v_pool"],
+                    d["block_table"], d["cu_seqlens_q"], d["seq_lens_k"], None, None, b.scale,
+                    out, None, ws)
+    torch.cuda.synchronize()
+    elapsed = time.perf_counter() - t0
+    assert api.rpa_device_error(clear=True) == 1     # decode wait ran out, nothing else
+    assert elapsed < 1.0, elapsed                     # well before the normal 2 s limit
+    ref, ref_lse, kp, vp = oracle_forward(b)
+    out, lse, gk, gv, _ = run_forward(b)
+    assert_close(out, ref)
+    assert_lse_close(lse, ref_lse)
+    assert np.array_equal(orc.bits16(gk), kp) and np.array_equal(orc.bits16(gv), vp)
