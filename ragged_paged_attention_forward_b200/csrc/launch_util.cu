@@ -3,6 +3,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <vector>
 
 #include "rpa_internal.h"
 
@@ -113,17 +114,35 @@ cudaError_t ensure_smem_attr(const void* kernel, int bytes) {
   return cudaSuccess;
 }
 
-cudaError_t side_stream(cudaStream_t* stream) {
-  static cudaStream_t streams[kMaxDevices] = {nullptr};
+cudaError_t side_stream(cudaStream_t caller, cudaStream_t* stream) {
+  // one side stream per (device, caller stream), so that callers on different streams do
+  // not serialise their tensor-core work on a shared one; past kMaxSideStreams caller streams
+  // on a device, later callers share the existing side streams (correct, less concurrent)
+  constexpr size_t kMaxSideStreams = 64;
+  struct Entry {
+    cudaStream_t caller;
+    cudaStream_t side;
+  };
+  static std::vector<Entry> table[kMaxDevices];
   static std::mutex mu;
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lock(mu);
-  if (!streams[dev]) {
-    cudaError_t e = cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking);
-    if (e != cudaSuccess) return e;
+  std::vector<Entry>& t = table[dev];
+  for (const Entry& e : t)
+    if (e.caller == caller) {
+      *stream = e.side;
+      return cudaSuccess;
+    }
+  if (t.size() >= kMaxSideStreams) {
+    *stream = t[(reinterpret_cast<uintptr_t>(caller) >> 4) % t.size()].side;
+    return cudaSuccess;
   }
-  *stream = streams[dev];
+  cudaStream_t side = nullptr;
+  cudaError_t e = cudaStreamCreateWithFlags(&side, cudaStreamNonBlocking);
+  if (e != cudaSuccess) return e;
+  t.push_back(Entry{caller, side});
+  *stream = side;
   return cudaSuccess;
 }
 

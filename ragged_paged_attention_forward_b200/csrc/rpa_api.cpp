@@ -793,7 +793,7 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     // e4m3 device plans run decode rows only (the planner refused the others): no fork.
     cudaStream_t pf_stream = stream;
     if (!kv8) {
-    st = check_cuda(side_stream(&pf_stream), "side stream");
+    st = check_cuda(side_stream(stream, &pf_stream), "side stream");
     if (st != RPA_OK) return st;
     if (!plan->fork_ev) {
       st = check_cuda(cudaEventCreateWithFlags(&plan->fork_ev, cudaEventDisableTiming),
@@ -884,7 +884,7 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
   const bool fork = !plan->pf_tiles.empty() && !plan->dec_items.empty();
   cudaStream_t pf_stream = stream;
   if (fork) {
-    st = check_cuda(side_stream(&pf_stream), "side stream");
+    st = check_cuda(side_stream(stream, &pf_stream), "side stream");
     if (st != RPA_OK) return st;
     if (!plan->fork_ev) {
       st = check_cuda(cudaEventCreateWithFlags(&plan->fork_ev, cudaEventDisableTiming),

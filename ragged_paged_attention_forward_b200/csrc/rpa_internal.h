@@ -298,7 +298,7 @@ cudaError_t encode_q_map(CUtensorMap* map, const void* q, int num_tokens, int nu
 cudaError_t ensure_smem_attr(const void* kernel, int bytes);
 // A non-blocking stream of the current device owned by the library (created once), on which
 // the tensor-core kernel of a mixed batch runs next to the split-KV decode kernel.
-cudaError_t side_stream(cudaStream_t* stream);
+cudaError_t side_stream(cudaStream_t caller, cudaStream_t* stream);
 int device_sm_count();
 
 // Sets the thread-local error text returned by rpa_last_error().

@@ -206,6 +206,36 @@ def test_mixed_output_is_stream_ordered():
     assert_close(out.cpu(), ref)
 
 
+def test_mixed_steps_from_two_caller_streams():
+    # Two callers on two streams of one device: each mixed step forks its tensor-core kernel
+    # onto a side stream that belongs to its own caller stream and joins it back, so work
+    # queued on each caller's stream right after its call sees every output row.
+    b1 = wl.ragged_batch([700, 3000, 1500, 40], [300, 1, 1, 40], 8, 2, 128, 16, seed=62)
+    b2 = wl.ragged_batch([900, 2000, 64], [200, 1, 64], 8, 2, 128, 16, seed=63)
+    runs = []
+    for b in (b1, b2):
+        plan = plan_for(b)
+        assert plan.info().batch_class == api.CLASS_MIXED
+        d = to_device(b)
+        out = torch.full_like(d["q"], float("nan"))
+        ws = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device="cuda")
+        runs.append((b, plan, d, out, ws, torch.cuda.Stream(), torch.empty_like(out)))
+    torch.cuda.synchronize()
+    for b, plan, d, out, ws, s, snap in runs:
+        api.rpa_forward(plan, d["q"], d["k_new"], d["v_new"], d["k_pool"], d["v_pool"],
+                        d["block_table"], d["cu_seqlens_q"], d["seq_lens_k"], None, None,
+                        b.scale, out, None, ws, stream=s)
+        with torch.cuda.stream(s):
+            snap.copy_(out)  # queued on the caller's stream, no synchronisation in between
+    torch.cuda.synchronize()
+    assert api.rpa_device_error(clear=True) == 0
+    for b, plan, d, out, ws, s, snap in runs:
+        assert torch.equal(snap, out)
+        ref, _, kp, vp = oracle_forward(b)
+        assert_close(out.cpu(), ref)
+        assert np.array_equal(orc.bits16(d["k_pool"].cpu()), kp)
+
+
 # ------------------------------------------------------------------ sparse block-union mode
 
 def _sparse_case(kv_len, chunk, page, seed, density=None, Hq=8, Hkv=2, D=128):
