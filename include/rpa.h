@@ -259,7 +259,12 @@ RPA_API rpa_status rpa_rotary_write_kv(rpa_plan_t plan, const void* q, const voi
  *
  *   q                 device bf16 [T, Hq, D].
  *   k_new, v_new      device bf16 [T, Hkv, D], or both NULL when the cache already holds
- *                     the new tokens (e.g. after rpa_write_kv).
+ *                     the new tokens (e.g. after rpa_write_kv).  Given, a batch of short rows
+ *                     and a mixed batch have the attention kernels write them into the pools
+ *                     themselves (the cache write fused with attention, "Ragged Paged
+ *                     Attention ..." Key ideas); a batch of only long rows, e4m3 pools and
+ *                     device plans run a scatter kernel first.  Either way the pools hold
+ *                     every new row when the call's work completes.
  *   k_pool, v_pool    device bf16 pools (written in place, then read: the alias rule
  *                     of the WebGPU page -- input and output cache are one buffer).
  *   block_table, cu_seqlens_q, seq_lens_k   as for rpa_write_kv.

@@ -114,11 +114,13 @@ struct Unit {
   int n_tiles;           // 128-key tiles
 };
 
-template <int D>
+template <int D, bool kFuse>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap,
                    const __grid_constant__ CUtensorMap kmap,
-                   const __grid_constant__ CUtensorMap vmap, PrefillLaunch p,
+                   const __grid_constant__ CUtensorMap vmap,
+                   const __grid_constant__ CUtensorMap knmap,
+                   const __grid_constant__ CUtensorMap vnmap, PrefillLaunch p,
                    const __grid_constant__ PrefillTilesInline inl) {
   using Geo = PfGeom<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -236,6 +238,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&qmap);
       tma_prefetch_desc(&kmap);
       tma_prefetch_desc(&vmap);
+      if (kFuse && p.fuse_rows > 0) {
+        tma_prefetch_desc(&knmap);
+        tma_prefetch_desc(&vnmap);
+      }
     }
     int kv_iter = 0;         // K/V tiles begun, over all units of this CTA
     int q_iter = 0;          // Q tiles begun
@@ -267,6 +273,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                       ((size_t)w.tile.seq * p.kv.num_kv_heads + w.h) * p.kv.max_blocks;
         const int hcoord = p.kv.layout == 0 ? w.h : 0;
         const int box_rows = P < kKeys ? P : kKeys;
+        // first key position served from k_new / v_new (-1: none)
+        const int fuse_edge =
+            kFuse && p.fuse_rows > 0 ? (w.past + p.fuse_rows - 1) / p.fuse_rows * p.fuse_rows
+                                     : -1;
         const uint32_t box_bytes = (uint32_t)box_rows * 128u * Geo::kHalves;
         for (int j = 0; !stop && j < w.n_tiles; ++j) {
           const int it = kv_iter++;
@@ -281,6 +291,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             first_blk = (j * kKeys) >> log2P;
             nbox = ((min(j * kKeys + kKeys, w.kv_hi) - 1) >> log2P) - first_blk + 1;
           }
+          // A tile holding keys at or past fuse_edge (this step's new rows, read from k_new /
+          // v_new; the pool gets them from the writer warps of this launch) takes the loop
+          // below that decides per box; every other tile the plain pool loop.
+          const bool tile_new =
+              kFuse && fuse_edge >= 0 && (w.table ? true : j * kKeys + kKeys > fuse_edge);
           // K first (S needs it first), then V; each waits for its own slot to be released
           for (int kv = 0; kv < 2; ++kv) {
             const int ns = kv == 0 ? kStagesK : kStagesV;
@@ -295,6 +310,31 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint8_t* dst_base = (kv == 0 ? Ks : Vs) + slot * Geo::kTileBytes;
             const CUtensorMap* map = kv == 0 ? &kmap : &vmap;
             uint64_t* bar = kv == 0 ? &k_full[slot] : &v_full[slot];
+            if (tile_new) {
+              for (int i = 0; i < nbox; ++i) {
+                const int blk =
+                    w.table ? __ldg(w.table + j * (kKeys >> log2P) + i) : first_blk + i;
+                const int kst = (blk << log2P) + slot0;
+                uint8_t* dst = dst_base + i * box_rows * 128;
+                if (blk >= 0 && blk < p.kv.max_blocks && kst >= fuse_edge) {
+                  const CUtensorMap* nmap = kv == 0 ? &knmap : &vnmap;
+#pragma unroll
+                  for (int half = 0; half < Geo::kHalves; ++half)
+                    tma_load_3d(dst + half * Geo::kHalfBytes, nmap, half * 64, w.h,
+                                w.tile.t0 + (kst - w.past), bar);
+                } else {
+                  int page = -1;
+                  if (blk >= 0 && blk < p.kv.max_blocks)
+                    page = __ldg(bt_row + blk);
+                  else if (kv == 0)
+                    atomicOr(p.err, kErrBadIndex);
+#pragma unroll
+                  for (int half = 0; half < Geo::kHalves; ++half)
+                    tma_load_4d(dst + half * Geo::kHalfBytes, map, half * 64, hcoord, slot0,
+                                page, bar);
+                }
+              }
+            } else
             for (int i = 0; i < nbox; ++i) {
               const int blk =
                   w.table ? __ldg(w.table + j * (kKeys >> log2P) + i) : first_blk + i;
@@ -458,6 +498,70 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) umma_commit(mma_done);
     __syncwarp();
     warp_wait_bounded(mma_done, 0, never, nullptr, 0, kWaitTimeoutNs / 8);
+  } else if (kFuse && p.fuse_rows > 0) {
+    // ------------------------------------------------------------------ KV write (warps 2-3)
+    // For each unit whose first query head is its KV group's first, the query tile's new K
+    // and V rows of that KV head, from the first key the attention reads out of k_new / v_new,
+    // are copied into their cache slots (one 16-byte chunk per thread and step).  Nothing in
+    // this launch reads those slots; the older rows that share a box were written before it.
+    const int wt = (warp - 2) * 32 + lane;
+    constexpr int kChunks = D / 8;  // 16-byte chunks per row
+    for (int k = 0;; ++k) {
+      const int u = unit_index(k);
+      if (u >= num_units) break;
+      const int tile_idx = u / groups;
+      const int hq0 = (u - tile_idx * groups) * hpc;
+      if (hq0 % G != 0) continue;
+      const PrefillTile tile = p.tiles ? p.tiles[tile_idx] : inl.v[tile_idx];
+      const int h = hq0 / G;
+      const int past = tile.kv_len - tile.q_len;
+      const int edge = (past + p.fuse_rows - 1) / p.fuse_rows * p.fuse_rows;
+      const int i0 = max(tile.q_start, edge - past);  // local token indices [i0, i1)
+      const int i1 = min(tile.q_len, tile.q_start + kRows);
+      const int rows = i1 - i0;
+      if (rows <= 0) continue;
+      const int32_t* bt_row =
+          p.kv.layout == 0 ? p.kv.block_table + (size_t)tile.seq * p.kv.max_blocks
+                           : p.kv.block_table +
+                                 ((size_t)tile.seq * p.kv.num_kv_heads + h) * p.kv.max_blocks;
+      // four 16-byte loads in flight per thread before their stores
+      const int total = 2 * rows * kChunks;
+      for (int c0 = wt; c0 < total; c0 += 64 * 4) {
+        uint4 val[4];
+        uint4* dst[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int c = c0 + q * 64;
+          dst[q] = nullptr;
+          if (c >= total) continue;
+          const int kvsel = c / (rows * kChunks);
+          const int rem = c - kvsel * rows * kChunks;
+          const int i = i0 + rem / kChunks;
+          const int ch = rem % kChunks;
+          const int pos = past + i;
+          const int blk = pos >> log2P;
+          const int page = blk < p.kv.max_blocks ? __ldg(bt_row + blk) : -1;
+          if (page < 0 || page >= p.kv.num_pages) {
+            atomicOr(p.err, kErrBadIndex);
+            continue;
+          }
+          const int slot = pos & (P - 1);
+          const size_t row = p.kv.layout == 0
+                                 ? ((size_t)page * P + slot) * p.kv.num_kv_heads + h
+                                 : (size_t)page * P + slot;
+          val[q] = __ldg(reinterpret_cast<const uint4*>(
+                             (kvsel == 0 ? p.k_new : p.v_new) +
+                             ((size_t)(tile.t0 + i) * p.kv.num_kv_heads + h) * D) +
+                         ch);
+          dst[q] = reinterpret_cast<uint4*>(
+                       static_cast<uint16_t*>(kvsel == 0 ? p.k_pool_w : p.v_pool_w) + row * D) +
+                   ch;
+        }
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          if (dst[q]) __stcs(dst[q], val[q]);  // streaming: nothing here reads them again
+      }
+    }
   }
   } else if ((warp - 4) / 4 < hpc) {
     // ------------------------------------------------------------------ softmax (head x)
@@ -701,6 +805,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+template <int D, bool kFuse>
+cudaError_t launch_prefill_kernel(const CUtensorMap& qmap, const CUtensorMap& kmap,
+                                  const CUtensorMap& vmap, const CUtensorMap& knmap,
+                                  const CUtensorMap& vnmap, const PrefillLaunch& p,
+                                  const PrefillTilesInline* inl, dim3 grid, cudaStream_t stream) {
+  const void* k = reinterpret_cast<const void*>(prefill_kernel<D, kFuse>);
+  // the register rebalancing inside the kernel needs exactly the launch budget it was
+  // written for; refuse to launch otherwise (a short budget would stall setmaxnreg.inc)
+  cudaFuncAttributes fa;
+  cudaError_t e = cudaFuncGetAttributes(&fa, k);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs != kLaunchRegs) {
+    set_last_error("prefill kernel built with %d registers per thread, expected %d", fa.numRegs,
+                   kLaunchRegs);
+    return cudaErrorInvalidConfiguration;
+  }
+  e = ensure_smem_attr(k, PfGeom<D>::kAlloc);
+  if (e != cudaSuccess) return e;
+  prefill_kernel<D, kFuse><<<grid, kThreads, PfGeom<D>::kAlloc, stream>>>(qmap, kmap, vmap, knmap,
+                                                                          vnmap, p, *inl);
+  return cudaSuccess;
+}
+
 cudaError_t launch_prefill(const PrefillLaunch& p, const PrefillTilesInline* inl,
                            cudaStream_t stream) {
   if (p.num_tiles <= 0) return cudaSuccess;
@@ -711,6 +838,14 @@ cudaError_t launch_prefill(const PrefillLaunch& p, const PrefillTilesInline* inl
   if (e != cudaSuccess) return e;
   e = encode_kv_map(&vmap, p.kv.v_pool, p.kv, p.head_dim, kKeys);
   if (e != cudaSuccess) return e;
+  // this step's new rows [T, Hkv, D], in boxes as high as the pool's
+  CUtensorMap knmap = kmap, vnmap = vmap;
+  if (p.fuse_rows > 0) {
+    e = encode_q_map(&knmap, p.k_new, p.num_tokens, p.num_kv_heads, p.head_dim, p.fuse_rows);
+    if (e != cudaSuccess) return e;
+    e = encode_q_map(&vnmap, p.v_new, p.num_tokens, p.num_kv_heads, p.head_dim, p.fuse_rows);
+    if (e != cudaSuccess) return e;
+  }
   const int G = p.num_q_heads / p.num_kv_heads;
   const int hpc = (p.qtile_table == nullptr && (G & 1) == 0) ? 2 : 1;  // as in the kernel
   // persistent: one CTA per SM at most (each holds all of an SM's TMEM); otherwise one CTA
@@ -726,32 +861,16 @@ cudaError_t launch_prefill(const PrefillLaunch& p, const PrefillTilesInline* inl
     if (ctas > sms) ctas = sms;
   }
   const dim3 grid((unsigned)ctas);
-  // the register rebalancing inside the kernel needs exactly the launch budget it was
-  // written for; refuse to launch otherwise (a short budget would stall setmaxnreg.inc)
-  {
-    cudaFuncAttributes fa;
-    const void* k = p.head_dim == 128 ? reinterpret_cast<const void*>(prefill_kernel<128>)
-                                      : reinterpret_cast<const void*>(prefill_kernel<64>);
-    e = cudaFuncGetAttributes(&fa, k);
-    if (e != cudaSuccess) return e;
-    if (fa.numRegs != kLaunchRegs) {
-      set_last_error("prefill kernel built with %d registers per thread, expected %d",
-                     fa.numRegs, kLaunchRegs);
-      return cudaErrorInvalidConfiguration;
-    }
-  }
-  if (p.head_dim == 128) {
-    e = ensure_smem_attr(reinterpret_cast<const void*>(prefill_kernel<128>),
-                         PfGeom<128>::kAlloc);
-    if (e != cudaSuccess) return e;
-    prefill_kernel<128><<<grid, kThreads, PfGeom<128>::kAlloc, stream>>>(qmap, kmap, vmap, p,
-                                                                        *inl);
-  } else {
-    e = ensure_smem_attr(reinterpret_cast<const void*>(prefill_kernel<64>), PfGeom<64>::kAlloc);
-    if (e != cudaSuccess) return e;
-    prefill_kernel<64><<<grid, kThreads, PfGeom<64>::kAlloc, stream>>>(qmap, kmap, vmap, p,
-                                                                      *inl);
-  }
+  const bool fuse = p.fuse_rows > 0;
+  if (p.head_dim == 128)
+    e = fuse ? launch_prefill_kernel<128, true>(qmap, kmap, vmap, knmap, vnmap, p, inl, grid, stream)
+             : launch_prefill_kernel<128, false>(qmap, kmap, vmap, knmap, vnmap, p, inl, grid,
+                                                 stream);
+  else
+    e = fuse ? launch_prefill_kernel<64, true>(qmap, kmap, vmap, knmap, vnmap, p, inl, grid, stream)
+             : launch_prefill_kernel<64, false>(qmap, kmap, vmap, knmap, vnmap, p, inl, grid,
+                                                stream);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

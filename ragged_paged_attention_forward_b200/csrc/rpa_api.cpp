@@ -76,6 +76,11 @@ struct rpa_plan_s {
   PrefillTilesInline pf_inline;
   // pure decode plans fold the KV write into the decode kernel
   bool fuse_write = false;
+  // host plans over bf16 pools with rows for both kernels (mixed batches): each attention
+  // kernel writes its own rows' new K/V; only new rows that share a TMA box with older keys
+  // (pf_straddle) need the scatter kernel first
+  bool pf_straddle = false;
+  int decode_skip_rows = 0;  // the scatter kernel skips sequences with q_len * G <= this
   // device-planned plans: the lists are built on the device at every call, up to these caps
   bool device_mode = false;
   int max_kv_len = 0;
@@ -399,8 +404,20 @@ rpa_status rpa_plan(const rpa_shape* shape, const int32_t* cu_seqlens_q,
     std::copy(plan->pf_tiles.begin(), plan->pf_tiles.end(), plan->pf_inline.v);
   }
   plan->fuse_write = plan->pf_tiles.empty() && !plan->dec_items.empty();
+  {
+    const int box = std::min(s.page_size, kPrefillTileKeys);
+    for (int b = 0; b < B; ++b) {
+      const int q_len = cu_seqlens_q[b + 1] - cu_seqlens_q[b];
+      if (q_len > 0 && !to_decode[b] && (seq_lens_k[b] - q_len) % box != 0)
+        plan->pf_straddle = true;
+    }
+    plan->decode_skip_rows = plan->dec_items.empty() ? 0 : decode_rows_cap;
+  }
   plan->launches_write = T > 0 ? 1 : 0;
-  plan->launches_forward = (plan->fuse_write ? 0 : plan->launches_write) +
+  const bool pf_writes = !plan->pf_tiles.empty() && !plan->dec_items.empty() && !o.kv_e4m3;
+  const int write_in_forward =
+      plan->fuse_write ? 0 : (pf_writes ? (plan->pf_straddle ? 1 : 0) : plan->launches_write);
+  plan->launches_forward = write_in_forward +
                            (plan->dec_items.empty() ? 0 : 1) +
                            (plan->merge_rows.empty() ? 0 : 1) +
                            (plan->pf_tiles.empty() ? 0 : 1);
@@ -515,7 +532,7 @@ static rpa_status write_kv_impl(rpa_plan_t plan, const void* k_new, const void* 
                                 const int32_t* cu_seqlens_q, const int32_t* seq_lens_k,
                                 cudaStream_t stream, int skip_rows_upto = 0,
                                 const float* k_scale = nullptr,
-                                const float* v_scale = nullptr) {
+                                const float* v_scale = nullptr, int below_box = 0) {
   const rpa_shape& s = plan->shape;
   int* err = nullptr;
   rpa_status st = check_cuda(device_error_word(&err), "device error word");
@@ -542,6 +559,7 @@ static rpa_status write_kv_impl(rpa_plan_t plan, const void* k_new, const void* 
   w.tokens_on_device = plan->device_mode ? 1 : 0;
   w.skip_rows_upto = skip_rows_upto;
   w.group = s.num_q_heads / s.num_kv_heads;
+  w.below_box = below_box;
   w.err = err;
   return check_cuda(launch_write_kv(w, stream), "write_kv launch");
 }
@@ -701,10 +719,27 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0)
     RPA_FAIL(RPA_ERR_INVALID_ARG, "workspace must be 256-byte aligned");
 
-  if (k_new && !plan->fuse_write && !plan->device_mode) {
-    st = write_kv_impl(plan, k_new, v_new, k_pool, v_pool, block_table, cu_seqlens_q, seq_lens_k,
-                       stream, 0, kv8 ? k_scale : nullptr, kv8 ? v_scale : nullptr);
-    if (st != RPA_OK) return st;
+  // A mixed batch over bf16 pools (host plan): each attention kernel writes its own rows' new
+  // K/V (the cache write fused with attention); the scatter kernel runs first only for new
+  // rows that share a TMA box with older keys.  A batch of only long rows keeps the scatter
+  // kernel: measured, it is faster than the tensor-core kernel's own copy there.
+  const bool fuse_pf = k_new && !kv8 && !plan->device_mode && !plan->pf_tiles.empty() &&
+                       !plan->dec_items.empty();
+  const int fuse_box = std::min(s.page_size, kPrefillTileKeys);
+  if (k_new && !plan->device_mode) {
+    if (fuse_pf) {
+      if (plan->pf_straddle) {
+        st = write_kv_impl(plan, k_new, v_new, k_pool, v_pool, block_table, cu_seqlens_q,
+                           seq_lens_k, stream, plan->decode_skip_rows, nullptr, nullptr,
+                           fuse_box);
+        if (st != RPA_OK) return st;
+      }
+    } else if (!plan->fuse_write) {
+      st = write_kv_impl(plan, k_new, v_new, k_pool, v_pool, block_table, cu_seqlens_q,
+                         seq_lens_k, stream, 0, kv8 ? k_scale : nullptr,
+                         kv8 ? v_scale : nullptr);
+      if (st != RPA_OK) return st;
+    }
   }
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   if (plan->meta_bytes > 0 && !plan->inline_lists) {
@@ -924,6 +959,13 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     }
     p.err = err;
     p.kv = kv;
+    if (fuse_pf) {
+      p.k_new = static_cast<const uint16_t*>(k_new);
+      p.v_new = static_cast<const uint16_t*>(v_new);
+      p.k_pool_w = k_pool;
+      p.v_pool_w = v_pool;
+      p.fuse_rows = fuse_box;
+    }
     if (kv8) {
       // the bf16 scratch copy, through its own block table
       p.kv.k_pool = ws + plan->off_s8_k;
@@ -954,7 +996,7 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     d.part_lse = reinterpret_cast<float*>(ws + plan->off_part_lse);
     d.err = err;
     d.kv = kv;
-    const bool fused = k_new && plan->fuse_write;
+    const bool fused = k_new && (plan->fuse_write || fuse_pf);
     d.k_new = fused ? static_cast<const uint16_t*>(k_new) : nullptr;
     d.v_new = fused ? static_cast<const uint16_t*>(v_new) : nullptr;
     d.k_pool_w = fused ? k_pool : nullptr;

@@ -162,6 +162,17 @@ struct PrefillLaunch {
   int32_t persistent;
   int* err;
   PagedKV kv;
+  // KV write fused into this kernel (bf16 pools): when fuse_rows > 0, a TMA box of keys that
+  // starts at or past round_up(past, fuse_rows) -- fuse_rows is the box height, min(P, 128)
+  // -- is read from this step's k_new / v_new rows instead of the pool, and the unit of each
+  // (query tile, KV head) whose first query head is the group's first copies the tile's new
+  // rows from that boundary on into the pool.  New rows that share a box with older keys
+  // are written before the launch.  0: every key from the pool, nothing written.
+  const uint16_t* k_new;     // bf16 [T, Hkv, D]
+  const uint16_t* v_new;
+  void* k_pool_w;
+  void* v_pool_w;
+  int32_t fuse_rows;
 };
 
 struct WriteLaunch {
@@ -188,6 +199,9 @@ struct WriteLaunch {
   // the decode kernel, which writes them itself)
   int32_t skip_rows_upto;
   int32_t group;
+  // > 0: only positions below round_up(past, below_box) -- the new rows that share a TMA box
+  // with older keys, which the tensor-core kernel reads from the pool
+  int32_t below_box;
   int* err;
 };
 

@@ -72,6 +72,7 @@ __global__ void __launch_bounds__(256) write_kv_kernel(WriteLaunch p) {
     if (p.skip_rows_upto > 0 && q_len * p.group <= p.skip_rows_upto) continue;
     const int past = __ldg(p.seq_lens_k + b) - q_len;
     const int pos = past + (t - t0);
+    if (p.below_box > 0 && pos >= (past + p.below_box - 1) / p.below_box * p.below_box) continue;
     const int blk = pos / p.page_size;
     const int slot = pos - blk * p.page_size;
     if (pos < 0 || blk >= p.max_blocks) {  // a device-planned step past its limits

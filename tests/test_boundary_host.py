@@ -100,6 +100,23 @@ def test_plan_classifies_and_sizes():
     assert forced.num_decode_items == 0 and forced.num_prefill_tiles == 5
 
 
+def test_launch_counts_with_the_write_in_the_kernels():
+    from tests.rpa_testing import plan_for
+    # a batch of only long rows: scatter kernel + tensor-core kernel
+    pf = wl.ragged_batch([300, 64], [300, 64], 8, 2, 64, 16, seed=1, keep_logical=False)
+    assert plan_for(pf).info().launches_forward == 2
+    # a mixed batch: both attention kernels write their own rows (tensor-core kernel, decode
+    # kernel, merge), the chunk's past (64) a multiple of the TMA box height (16)
+    mx = wl.ragged_batch([300, 1000, 96], [300, 1, 32], 8, 2, 64, 16, seed=1, keep_logical=False)
+    assert plan_for(mx).info().launches_forward == 3
+    # a past of 69 leaves new rows in a box with older keys: the scatter kernel runs for them
+    st = wl.ragged_batch([300, 1000, 101], [300, 1, 32], 8, 2, 64, 16, seed=1, keep_logical=False)
+    assert plan_for(st).info().launches_forward == 4
+    # e4m3 plans keep the quantising scatter kernel
+    mx8 = wl.ragged_batch([300, 1000, 96], [300, 1, 32], 8, 2, 128, 16, seed=1, keep_logical=False)
+    assert plan_for(mx8, kv_e4m3=True).info().launches_forward == 4
+
+
 def test_zero_tokens_is_a_no_op():
     p = api.rpa_plan(**_shape(num_seqs=2, num_tokens=0, cu_seqlens_q=[0, 0, 0]))
     fake = ctypes.c_void_p(1 << 20)

@@ -49,14 +49,46 @@ def test_prefill_small_no_past():
     assert np.array_equal(orc.bits16(gk), kp) and np.array_equal(orc.bits16(gv), vp)
 
 
+@pytest.mark.parametrize("layout", [wl.SEQ_MAJOR, wl.HEAD_MAJOR])
 @pytest.mark.parametrize("page", [16, 32, 64, 128, 256])
-def test_chunked_prefill_with_past(page):
-    b = wl.ragged_batch([430, 170, 1000], [130, 40, 257], 8, 2, 128, page, seed=52 + page)
-    ref, ref_lse, _, _ = oracle_forward(b)
-    out, lse, _, _, plan = run_forward(b)
-    assert plan.info().num_prefill_tiles > 0
+def test_chunked_prefill_with_past(page, layout):
+    # pasts 300, 130 and 743, every row on the tensor-core kernel: the scatter kernel writes
+    # the new K/V first; the whole pool is compared bit for bit
+    b = wl.ragged_batch([430, 170, 1000], [130, 40, 257], 8, 2, 128, page, seed=52 + page,
+                        layout=layout)
+    ref, ref_lse, kp, vp = oracle_forward(b)
+    out, lse, gk, gv, plan = run_forward(b)
+    info = plan.info()
+    assert info.num_prefill_tiles > 0
+    assert info.launches_forward == 2      # scatter + tensor-core kernel
     assert_close(out, ref)
     assert_lse_close(lse, ref_lse)
+    assert np.array_equal(orc.bits16(gk), kp) and np.array_equal(orc.bits16(gv), vp)
+
+
+@pytest.mark.parametrize("straddle", [False, True])
+@pytest.mark.parametrize("page", [16, 64, 256])
+def test_fused_write_equals_separate_write(page, straddle):
+    # A mixed batch: both attention kernels write their rows' new K/V themselves (the
+    # tensor-core kernel reads its rows' new keys from k_new / v_new).  Against rpa_write_kv
+    # followed by an rpa_forward without new rows: same pools, same outputs bit for bit.  The
+    # chunks' pasts (256, 0, 512) are box-aligned, so no scatter kernel runs in the fused step;
+    # with a past of 33 the first new rows share a box with older keys and are scattered first.
+    kv = [400, 333 if straddle else 300, 1000, 700]
+    b = wl.ragged_batch(kv, [144, 300, 488, 1], 8, 2, 128, page, seed=59 + page)
+    plan = plan_for(b)
+    info = plan.info()
+    assert info.batch_class == api.CLASS_MIXED
+    assert info.launches_forward == (4 if straddle else 3)  # [scatter,] tensor-core, decode, merge
+    fused = run_forward(b)
+    split = run_forward(b, fused=False)
+    assert torch.equal(fused[0], split[0]) and torch.equal(fused[1], split[1])
+    # the pools hold NaN in their free slots: compare bit patterns
+    assert np.array_equal(orc.bits16(fused[2]), orc.bits16(split[2]))
+    assert np.array_equal(orc.bits16(fused[3]), orc.bits16(split[3]))
+    ref, _, kp, vp = oracle_forward(b)
+    assert_close(fused[0], ref)
+    assert np.array_equal(orc.bits16(fused[2]), kp) and np.array_equal(orc.bits16(fused[3]), vp)
 
 
 @pytest.mark.parametrize("D", [64, 128])
@@ -85,15 +117,17 @@ def test_mixed_q_len_with_past(causal):
     # the failing WebGPU case: mixed q_len with past > 0
     b = wl.ragged_batch([16, 40, 300, 77, 1000], [16, 4, 300, 1, 33], 4, 2, 128, 16, seed=55,
                         causal=causal)
-    ref, ref_lse, _, _ = oracle_forward(b)
-    out, lse, _, _, plan = run_forward(b)
+    ref, ref_lse, kp, vp = oracle_forward(b)
+    out, lse, gk, gv, plan = run_forward(b)
     info = plan.info()
     assert info.batch_class == api.CLASS_MIXED
     assert info.num_prefill_tiles > 0 and info.num_decode_items > 0
     assert_close(out, ref)
     assert_lse_close(lse, ref_lse)
+    assert np.array_equal(orc.bits16(gk), kp) and np.array_equal(orc.bits16(gv), vp)
     forced = run_forward(b, plan_opts=dict(force_class=api.CLASS_PREFILL))
     assert_close(forced[0], ref)
+    assert np.array_equal(orc.bits16(forced[2]), kp) and np.array_equal(orc.bits16(forced[3]), vp)
 
 
 @pytest.mark.parametrize("scale", [0.0, 0.02, -0.09])
@@ -254,11 +288,13 @@ def _sparse_case(kv_len, chunk, page, seed, density=None, Hq=8, Hkv=2, D=128):
 @pytest.mark.parametrize("page", [16, 64, 128])
 def test_sparse_small(page):
     b, table, count = _sparse_case(1500, 300, page, seed=60 + page)
-    ref, ref_lse, _, _ = oracle_forward(b, group_table=table.numpy(), group_count=count.numpy())
-    out, lse, _, _, plan = run_forward(b, group_table=table, group_count=count)
+    ref, ref_lse, kp, vp = oracle_forward(b, group_table=table.numpy(),
+                                          group_count=count.numpy())
+    out, lse, gk, gv, plan = run_forward(b, group_table=table, group_count=count)
     assert plan.info().num_decode_items == 0
     assert_close(out, ref)
     assert_lse_close(lse, ref_lse)
+    assert np.array_equal(orc.bits16(gk), kp) and np.array_equal(orc.bits16(gv), vp)
 
 
 def test_sparse_all_ones_equals_dense():
@@ -343,12 +379,13 @@ def test_odd_group_size_mixed_batch(Hq, Hkv, layout):
     # group), and the split-KV kernel packs G x q_len query rows of a group into its MMA's N.
     b = wl.ragged_batch([1, 300, 777, 260, 2000], [1, 2, 1, 200, 150], Hq, Hkv, 128, 16,
                         seed=97 + Hq, layout=layout)
-    ref, ref_lse, _, _ = oracle_forward(b)
-    out, lse, _, _, plan = run_forward(b)
+    ref, ref_lse, kp, vp = oracle_forward(b)
+    out, lse, gk, gv, plan = run_forward(b)
     info = plan.info()
     assert info.num_decode_items > 0 and info.num_prefill_tiles > 0
     assert_close(out, ref)
     assert_lse_close(lse, ref_lse)
+    assert np.array_equal(orc.bits16(gk), kp) and np.array_equal(orc.bits16(gv), vp)
 
 
 @pytest.mark.parametrize("Hq,Hkv", [(12, 4), (40, 8)])
