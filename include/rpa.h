@@ -106,7 +106,8 @@ typedef struct rpa_plan_info {
   int32_t launches_forward;    /* kernels rpa_forward launches when given k_new/v_new      */
   int32_t launches_write;      /* kernels rpa_write_kv launches                            */
   int32_t decode_split_keys;   /* split size used                                          */
-  int32_t reserved;
+  int32_t tensor_core_grid;    /* mixed batches: SMs given to a persistent tensor-core grid */
+                               /* launched before the decode kernel (0: one CTA per unit)  */
   size_t workspace_bytes;      /* device workspace rpa_forward needs                       */
 } rpa_plan_info;
 

@@ -47,7 +47,7 @@ class PlanInfo(ctypes.Structure):
     _fields_ = [("batch_class", ctypes.c_int32), ("num_decode_items", ctypes.c_int32),
                 ("num_prefill_tiles", ctypes.c_int32), ("num_merge_rows", ctypes.c_int32),
                 ("launches_forward", ctypes.c_int32), ("launches_write", ctypes.c_int32),
-                ("decode_split_keys", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("decode_split_keys", ctypes.c_int32), ("tensor_core_grid", ctypes.c_int32),
                 ("workspace_bytes", ctypes.c_size_t)]
 
 

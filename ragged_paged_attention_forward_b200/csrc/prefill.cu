@@ -823,9 +823,26 @@ cudaError_t launch_prefill_kernel(const CUtensorMap& qmap, const CUtensorMap& km
   }
   e = ensure_smem_attr(k, PfGeom<D>::kAlloc);
   if (e != cudaSuccess) return e;
-  prefill_kernel<D, kFuse><<<grid, kThreads, PfGeom<D>::kAlloc, stream>>>(qmap, kmap, vmap, knmap,
-                                                                          vnmap, p, *inl);
-  return cudaSuccess;
+  if (!p.launched) {
+    prefill_kernel<D, kFuse><<<grid, kThreads, PfGeom<D>::kAlloc, stream>>>(qmap, kmap, vmap,
+                                                                            knmap, vnmap, p, *inl);
+    return cudaSuccess;
+  }
+  // the event fires once every CTA has started: work that waits for it on another stream
+  // gets only the SMs these CTAs left
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = PfGeom<D>::kAlloc;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeLaunchCompletionEvent;
+  attr[0].val.launchCompletionEvent.event = p.launched;
+  attr[0].val.launchCompletionEvent.flags = 0;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, prefill_kernel<D, kFuse>, qmap, kmap, vmap, knmap, vnmap, p,
+                            *inl);
 }
 
 cudaError_t launch_prefill(const PrefillLaunch& p, const PrefillTilesInline* inl,
@@ -859,6 +876,7 @@ cudaError_t launch_prefill(const PrefillLaunch& p, const PrefillTilesInline* inl
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
     if (ctas > sms) ctas = sms;
+    if (p.max_ctas > 0 && ctas > p.max_ctas) ctas = p.max_ctas;
   }
   const dim3 grid((unsigned)ctas);
   const bool fuse = p.fuse_rows > 0;

@@ -81,6 +81,9 @@ struct rpa_plan_s {
   // (pf_straddle) need the scatter kernel first
   bool pf_straddle = false;
   int decode_skip_rows = 0;  // the scatter kernel skips sequences with q_len * G <= this
+  // mixed batches: SMs of the persistent tensor-core grid beside the decode kernel (0: one
+  // CTA per unit instead); see mixed_grid()
+  int mixed_grid = 0;
   // device-planned plans: the lists are built on the device at every call, up to these caps
   bool device_mode = false;
   int max_kv_len = 0;
@@ -93,9 +96,11 @@ struct rpa_plan_s {
   // fork/join events of a mixed batch (created on first use, on the device of that call)
   cudaEvent_t fork_ev = nullptr;
   cudaEvent_t join_ev = nullptr;
+  cudaEvent_t launched_ev = nullptr;  // the tensor-core grid of a split mixed step is resident
   ~rpa_plan_s() {
     if (fork_ev) cudaEventDestroy(fork_ev);
     if (join_ev) cudaEventDestroy(join_ev);
+    if (launched_ev) cudaEventDestroy(launched_ev);
   }
 };
 
@@ -149,6 +154,58 @@ int auto_split_keys(long total_key_heads, int sms) {
   s = std::max<long>(s, kMinSplitKeys);
   s = std::min<long>(s, kMaxSplitKeys);
   return (int)s;
+}
+
+// Mixed batches: the SMs that the tensor-core grid gets when it runs persistently beside the
+// decode kernel, or 0 to launch it with one CTA per unit instead.  Both kernels want whole
+// SMs (a tensor-core CTA holds one), so they share the GPU in space: the decode kernel is
+// launched once every tensor-core CTA is resident and takes the other SMs, and each SM a
+// persistent CTA leaves when its units are done.  Work model, in SM-microseconds (B200,
+// measured): a 128-key tile of a unit costs kTileUs, a unit kUnitUs more; the decode kernel
+// moves kDecodeGBpsPerSm per SM.  The balanced step time is both works over all SMs; the grid
+// is the smallest whose static walk over the units (rounds of the grid size, alternating
+// direction, as the kernel walks them) ends within 70% of it, so that its SMs pass to the
+// decode kernel before the decode work runs out (on the mixed workload the step measured
+// 0.463 / 0.455 / 0.444 / 0.465 ms with 64 / 72 / 80 / 88 SMs, 0.53 ms with a CTA per unit).  Batches where either part is small, or
+// that are short, keep the unit-per-CTA launch.
+int mixed_grid(const std::vector<PrefillTile>& tiles, const rpa_shape& s, int hpc,
+               double decode_bytes, int sms) {
+  if (tiles.empty() || decode_bytes <= 0 || sms < 64) return 0;
+  const double kTileUs = (s.head_dim == 128 ? 2.2 : 1.6) * (hpc == 2 ? 1.0 : 0.6);
+  const double kUnitUs = 2.0;
+  const double kDecodeGBpsPerSm = 42.0;
+  const int groups = s.num_q_heads / hpc;
+  std::vector<double> cost;
+  cost.reserve(tiles.size() * groups);
+  double wp = 0;
+  for (const PrefillTile& t : tiles) {
+    const long past = t.kv_len - t.q_len;
+    const long q_end = std::min(t.q_len, t.q_start + kPrefillTileRows);
+    const long kv_hi = s.causal ? std::min<long>(t.kv_len, past + q_end) : t.kv_len;
+    const double c = (double)((kv_hi + kPrefillTileKeys - 1) / kPrefillTileKeys) * kTileUs + kUnitUs;
+    for (int g = 0; g < groups; ++g) cost.push_back(c);
+    wp += c * groups;
+  }
+  const double wd = decode_bytes / (kDecodeGBpsPerSm * 1e3);  // bytes per us per SM
+  const double total = (wp + wd) / sms;                         // balanced step, us
+  if (total < 100.0 || wp < 0.15 * (wp + wd) || wd < 0.15 * (wp + wd) || cost.size() > 8192)
+    return 0;
+  const double target = 0.7 * total;
+  auto makespan = [&](int n) {
+    std::vector<double> fin(n, 0.0);
+    for (size_t u = 0; u < cost.size(); ++u) {
+      const int k = (int)(u / n), i = (int)(u % n);
+      fin[(k & 1) ? n - 1 - i : i] += cost[u];
+    }
+    return *std::max_element(fin.begin(), fin.end());
+  };
+  int lo = 1, hi = sms - 32;  // the decode kernel keeps at least 32 SMs
+  if (hi < lo || makespan(hi) > target) return 0;
+  while (lo < hi) {  // the makespan falls as the grid grows (close enough to search)
+    const int mid = (lo + hi) / 2;
+    if (makespan(mid) <= target) hi = mid; else lo = mid + 1;
+  }
+  return lo;
 }
 
 }  // namespace
@@ -413,6 +470,14 @@ rpa_status rpa_plan(const rpa_shape* shape, const int32_t* cu_seqlens_q,
     }
     plan->decode_skip_rows = plan->dec_items.empty() ? 0 : decode_rows_cap;
   }
+  if (!plan->pf_tiles.empty() && !plan->dec_items.empty() && !o.kv_e4m3 && !o.sparse) {
+    double dbytes = 0;
+    for (const DecodeItem& it : plan->dec_items)
+      dbytes += (double)(it.k_end - it.k_begin) * s.num_kv_heads * s.head_dim * 2 * 2;
+    const int G = s.num_q_heads / s.num_kv_heads;
+    plan->mixed_grid = mixed_grid(plan->pf_tiles, s, (G & 1) == 0 ? 2 : 1, dbytes,
+                                  device_sm_count());
+  }
   plan->launches_write = T > 0 ? 1 : 0;
   const bool pf_writes = !plan->pf_tiles.empty() && !plan->dec_items.empty() && !o.kv_e4m3;
   const int write_in_forward =
@@ -516,6 +581,7 @@ rpa_status rpa_plan_get_info(rpa_plan_t plan, rpa_plan_info* info) {
   info->launches_forward = plan->launches_forward;
   info->launches_write = plan->launches_write;
   info->decode_split_keys = plan->split_keys;
+  info->tensor_core_grid = plan->mixed_grid;
   info->workspace_bytes = plan->ws_bytes;
   if (plan->device_mode) {  // the caps the device-built lists may reach
     info->num_decode_items = plan->cap_items;
@@ -949,6 +1015,24 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     p.out = static_cast<uint16_t*>(out);
     p.lse = lse;
     p.persistent = fork ? 0 : 1;  // beside the decode kernel: one CTA per unit
+    if (fork && plan->mixed_grid > 0) {
+      // the planned split (mixed_grid): a persistent grid on part of the SMs, the decode kernel
+      // launched once it is resident.  Not under stream capture, which the launch-completion
+      // event is not meant for: there the unit-per-CTA launch stays.
+      cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+      st = check_cuda(cudaStreamIsCapturing(stream, &cap), "capture status");
+      if (st != RPA_OK) return st;
+      if (cap == cudaStreamCaptureStatusNone) {
+        if (!plan->launched_ev) {
+          st = check_cuda(cudaEventCreateWithFlags(&plan->launched_ev, cudaEventDisableTiming),
+                          "event create");
+          if (st != RPA_OK) return st;
+        }
+        p.persistent = 1;
+        p.max_ctas = plan->mixed_grid;
+        p.launched = plan->launched_ev;
+      }
+    }
     if (plan->opts.sparse == 2) {
       p.qtile_table = group_table;
       p.qtile_count = group_count;
@@ -978,6 +1062,10 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     }
     st = check_cuda(launch_prefill(p, &plan->pf_inline, pf_stream), "prefill launch");
     if (st != RPA_OK) return st;
+    if (p.launched) {
+      st = check_cuda(cudaStreamWaitEvent(stream, p.launched, 0), "launch wait");
+      if (st != RPA_OK) return st;
+    }
   }
   if (!plan->dec_items.empty()) {
     DecodeLaunch d{};

@@ -160,6 +160,10 @@ struct PrefillLaunch {
   // 1: one CTA per SM walks the units (a launch that has the GPU to itself); 0: one CTA per
   // unit, so that a decode kernel running beside it takes SMs as units finish
   int32_t persistent;
+  // persistent launches: at most this many CTAs (0: one per SM), and, when set, an event
+  // recorded once every CTA of the launch has started (host-side fields)
+  int32_t max_ctas;
+  cudaEvent_t launched;
   int* err;
   PagedKV kv;
   // KV write fused into this kernel (bf16 pools): when fuse_rows > 0, a TMA box of keys that

@@ -100,6 +100,20 @@ def test_plan_classifies_and_sizes():
     assert forced.num_decode_items == 0 and forced.num_prefill_tiles == 5
 
 
+def test_mixed_batches_plan_an_sm_split_only_when_both_parts_are_large():
+    from tests.rpa_testing import plan_for
+    # the mixed workload: the decode rows' 1.7 GB and the chunks' 192 units balance, so the
+    # tensor-core grid gets part of the SMs (the device is not visible here: 148 assumed)
+    g = plan_for(wl.mixed()).info().tensor_core_grid
+    assert 32 <= g <= 116
+    # small or lopsided batches keep one CTA per unit
+    small = wl.ragged_batch([16, 40, 300, 77, 1000], [16, 4, 300, 1, 33], 8, 2, 128, 16,
+                            seed=1, keep_logical=False)
+    assert plan_for(small).info().tensor_core_grid == 0
+    assert plan_for(wl.prefill()).info().tensor_core_grid == 0
+    assert plan_for(wl.decode(keep_logical=False)).info().tensor_core_grid == 0
+
+
 def test_launch_counts_with_the_write_in_the_kernels():
     from tests.rpa_testing import plan_for
     # a batch of only long rows: scatter kernel + tensor-core kernel

@@ -240,6 +240,37 @@ def test_mixed_output_is_stream_ordered():
     assert_close(out.cpu(), ref)
 
 
+def test_split_mixed_step_is_stream_ordered():
+    # The mixed workload plans a split: a persistent tensor-core grid on part of the SMs and
+    # the decode kernel, launched once that grid is resident, on the rest.  Work queued on the
+    # caller's stream right after the call must see every output row, and the rows must be
+    # right: every decode row's KV group and a whole unit of each chunk.
+    b = wl.mixed()
+    plan = plan_for(b)
+    info = plan.info()
+    assert 0 < info.tensor_core_grid < 148
+    d = to_device(b)
+    out = torch.full_like(d["q"], float("nan"))
+    ws = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device="cuda")
+    api.rpa_forward(plan, d["q"], d["k_new"], d["v_new"], d["k_pool"], d["v_pool"],
+                    d["block_table"], d["cu_seqlens_q"], d["seq_lens_k"], None, None, b.scale,
+                    out, None, ws)
+    snap = out.clone()  # queued on the same stream, no synchronisation in between
+    torch.cuda.synchronize()
+    assert api.rpa_device_error(clear=True) == 0
+    assert torch.equal(snap, out)
+    cu = b.cu_seqlens_q.tolist()
+    q_lens = [cu[i + 1] - cu[i] for i in range(b.num_seqs)]
+    rows = set(_unit_rows(b, [(q_lens.index(512), 2, 6), (q_lens.index(976), 5, 20)]))
+    for i in range(b.num_seqs):
+        if q_lens[i] == 1:
+            rows.update((cu[i], h) for h in range(4 * (i % 8), 4 * (i % 8) + 4))
+    rows = sorted(rows)
+    ref, _, kp, _ = oracle_forward(b, rows=rows)
+    assert_close(out.cpu(), ref, rows=rows)
+    assert np.array_equal(orc.bits16(d["k_pool"].cpu()), kp)
+
+
 def test_mixed_steps_from_two_caller_streams():
     # Two callers on two streams of one device: each mixed step forks its tensor-core kernel
     # onto a side stream that belongs to its own caller stream and joins it back, so work
