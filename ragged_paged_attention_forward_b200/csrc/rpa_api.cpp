@@ -162,18 +162,18 @@ int auto_split_keys(long total_key_heads, int sms) {
 // launched once every tensor-core CTA is resident and takes the other SMs, and each SM a
 // persistent CTA leaves when its units are done.  Work model, in SM-microseconds (B200,
 // measured): a 128-key tile of a unit costs kTileUs, a unit kUnitUs more; the decode kernel
-// moves kDecodeGBpsPerSm per SM.  The balanced step time is both works over all SMs; the grid
+// moves decode_gbps_per_sm per SM (42 GB/s of bf16 K/V, 33 GB/s of e4m3 codes: the whole-GPU
+// rates over 148 SMs).  The balanced step time is both works over all SMs; the grid
 // is the smallest whose static walk over the units (rounds of the grid size, alternating
 // direction, as the kernel walks them) ends within 70% of it, so that its SMs pass to the
 // decode kernel before the decode work runs out (on the mixed workload the step measured
 // 0.463 / 0.455 / 0.444 / 0.465 ms with 64 / 72 / 80 / 88 SMs, 0.53 ms with a CTA per unit).  Batches where either part is small, or
 // that are short, keep the unit-per-CTA launch.
 int mixed_grid(const std::vector<PrefillTile>& tiles, const rpa_shape& s, int hpc,
-               double decode_bytes, int sms) {
+               double decode_bytes, double decode_gbps_per_sm, int sms) {
   if (tiles.empty() || decode_bytes <= 0 || sms < 64) return 0;
   const double kTileUs = (s.head_dim == 128 ? 2.2 : 1.6) * (hpc == 2 ? 1.0 : 0.6);
   const double kUnitUs = 2.0;
-  const double kDecodeGBpsPerSm = 42.0;
   const int groups = s.num_q_heads / hpc;
   std::vector<double> cost;
   cost.reserve(tiles.size() * groups);
@@ -186,7 +186,7 @@ int mixed_grid(const std::vector<PrefillTile>& tiles, const rpa_shape& s, int hp
     for (int g = 0; g < groups; ++g) cost.push_back(c);
     wp += c * groups;
   }
-  const double wd = decode_bytes / (kDecodeGBpsPerSm * 1e3);  // bytes per us per SM
+  const double wd = decode_bytes / (decode_gbps_per_sm * 1e3);  // bytes per us per SM
   const double total = (wp + wd) / sms;                         // balanced step, us
   if (total < 100.0 || wp < 0.15 * (wp + wd) || wd < 0.15 * (wp + wd) || cost.size() > 8192)
     return 0;
@@ -470,13 +470,14 @@ rpa_status rpa_plan(const rpa_shape* shape, const int32_t* cu_seqlens_q,
     }
     plan->decode_skip_rows = plan->dec_items.empty() ? 0 : decode_rows_cap;
   }
-  if (!plan->pf_tiles.empty() && !plan->dec_items.empty() && !o.kv_e4m3 && !o.sparse) {
+  if (!plan->pf_tiles.empty() && !plan->dec_items.empty() && !o.sparse) {
+    const int elem = o.kv_e4m3 ? 1 : 2;  // bytes per K/V element the decode kernel reads
     double dbytes = 0;
     for (const DecodeItem& it : plan->dec_items)
-      dbytes += (double)(it.k_end - it.k_begin) * s.num_kv_heads * s.head_dim * 2 * 2;
+      dbytes += (double)(it.k_end - it.k_begin) * s.num_kv_heads * s.head_dim * 2 * elem;
     const int G = s.num_q_heads / s.num_kv_heads;
     plan->mixed_grid = mixed_grid(plan->pf_tiles, s, (G & 1) == 0 ? 2 : 1, dbytes,
-                                  device_sm_count());
+                                  o.kv_e4m3 ? 33.0 : 42.0, device_sm_count());
   }
   plan->launches_write = T > 0 ? 1 : 0;
   const bool pf_writes = !plan->pf_tiles.empty() && !plan->dec_items.empty() && !o.kv_e4m3;
