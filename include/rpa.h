@@ -87,9 +87,9 @@ typedef struct rpa_plan_options {
   int32_t decode_split_keys;   /* keys per decode split, multiple of 64; 0 = automatic     */
   int32_t sparse;              /* 1: rpa_forward will be given group tables; 2: per-(query  */
                                /* tile, query head) tables (rpa_build_qtile_tables)         */
-  int32_t kv_e4m3;             /* 1: the pools will hold e4m3 codes (rpa_forward_kv8): the   */
-                               /* workspace also holds a bf16 copy of the context of rows  */
-                               /* that go to the tensor-core kernel                        */
+  int32_t kv_e4m3;             /* 1: the pools will hold e4m3 codes (rpa_forward_kv8); the  */
+                               /* planner sizes the SM split of mixed batches for one-byte */
+                               /* elements                                                 */
   int32_t wait_test_us;        /* diagnostics, for tests of the bounded waits only: > 0    */
                                /* makes the split-KV decode kernel load no K/V and give up */
                                /* each of its waits after this many microseconds (at most  */
@@ -293,8 +293,8 @@ RPA_API rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new
  * rpa_forward_kv8 -- rpa_forward over an fp8 (e4m3) KV cache with per-KV-head scales.  Not
  * in the pages' shipped kernels: the WebGPU page's commit "FlashAttention: optional
  * seqlens_q input" lists the quantised KV cache under "Not in scope (deferred)"; this is
- * that extension for the decode path, which is bandwidth-bound, so one byte per element
- * halves its traffic.
+ * that extension: one byte per element halves the traffic of the bandwidth-bound decode path
+ * and of the tensor-core kernel's K/V tiles.
  *
  *   k_pool, v_pool    device uint8 pools of e4m3 codes (1 sign, 4 exponent bits with bias
  *                     7, 3 mantissa bits; no infinities; 0x7F / 0xFF are NaN; largest
@@ -304,24 +304,25 @@ RPA_API rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new
  *   k_new, v_new      device bf16 [T, Hkv, D], or both NULL.  Each new element x is stored as
  *                     the e4m3 code nearest to fp32(x) / scale (IEEE fp32 division; ties to
  *                     the even code; magnitudes past 448 saturate to +-448).
- *   the rest          as for rpa_forward (no group tables).
- * Supported: head_dim 128, no group tables.  Rows for the split-KV decode kernel read the
- * e4m3 pools directly: scores and P.V on f16 operands (e4m3 -> f16 is exact; q must stay
- * within f16's range, |q| < 65504), fp32 accumulation.  A host plan with rows for the
- * tensor-core kernel must be made with opts.kv_e4m3 = 1: after the write, those sequences'
- * context is copied to bf16 in the workspace (exactly: every e4m3 value is a bf16 value) and
- * the tensor-core kernel reads the copy with k_scale[h] folded into its score scale and
- * v_scale[h] into its output.  A device plan (rpa_plan_device) must be made with
- * opts.kv_e4m3 = 1 and runs decode rows only -- a row too long for the decode kernel is
- * refused with bit 16 of the device error word -- so a decode step over e4m3 pools can be
- * captured in a CUDA graph.  Anything else returns RPA_ERR_UNSUPPORTED.
+ *   group_table, group_count  as for rpa_forward (plans made with opts.sparse = 1 or 2),
+ *                     else NULL.
+ *   the rest          as for rpa_forward.
+ * Supported: head_dim 128.  Both attention kernels read the e4m3 pools in place and compute
+ * on f16 operands (e4m3 -> f16 is exact; q is converted to f16, exact within f16's range,
+ * so |q| must stay below 65504), with fp32 accumulation and P rounded to f16; k_scale[h] is
+ * folded into the score scale and v_scale[h] into the output.  Host plans with rows for the
+ * tensor-core kernel and device plans (rpa_plan_device) must be made with opts.kv_e4m3 = 1;
+ * a device plan over e4m3 pools runs every batch class, so a step can be captured in a CUDA
+ * graph.  Anything else returns RPA_ERR_UNSUPPORTED.
  */
 RPA_API rpa_status rpa_forward_kv8(rpa_plan_t plan, const void* q, const void* k_new,
                                    const void* v_new, void* k_pool, void* v_pool,
                                    const float* k_scale, const float* v_scale,
                                    const int32_t* block_table, const int32_t* cu_seqlens_q,
-                                   const int32_t* seq_lens_k, float scale, void* out, float* lse,
-                                   void* workspace, size_t workspace_bytes, void* stream);
+                                   const int32_t* seq_lens_k, const int32_t* group_table,
+                                   const int32_t* group_count, float scale, void* out,
+                                   float* lse, void* workspace, size_t workspace_bytes,
+                                   void* stream);
 
 /*
  * rpa_forward_no_alloc -- rpa_forward for callers that cannot allocate device memory.

@@ -548,9 +548,11 @@ def write_kv8(k_pool, v_pool, k_new, v_new, k_scale, v_scale, block_table, cu_se
 
 def forward_kv8(q, k_new, v_new, k_pool, v_pool, k_scale, v_scale, block_table, cu_seqlens_q,
                 seq_lens_k, *, scale: float, causal: bool, page_size: int,
-                layout: int = SEQ_MAJOR, rows=None):
+                layout: int = SEQ_MAJOR, rows=None, group_table=None, group_count=None,
+                qtile_table=None, qtile_count=None):
     """The fused step over e4m3 code pools: quantising write, then attention over the
-    dequantised keys and values.  Returns ``(out, lse, k_pool_after, v_pool_after)``."""
+    dequantised keys and values (restricted, as in ``attention``, to the blocks of the group
+    or query-tile tables when given).  Returns ``(out, lse, k_pool_after, v_pool_after)``."""
     num_kv_heads = len(np.atleast_1d(k_scale))
     if k_new is not None:
         kp, vp = write_kv8(k_pool, v_pool, k_new, v_new, k_scale, v_scale, block_table,
@@ -559,5 +561,7 @@ def forward_kv8(q, k_new, v_new, k_pool, v_pool, k_scale, v_scale, block_table, 
         kp, vp = codes8(k_pool).copy(), codes8(v_pool).copy()
     out, lse = attention(q, kp, vp, block_table, cu_seqlens_q, seq_lens_k, scale=scale,
                          causal=causal, page_size=page_size, layout=layout,
-                         num_kv_heads=num_kv_heads, rows=rows, kv_scales=(k_scale, v_scale))
+                         num_kv_heads=num_kv_heads, rows=rows, kv_scales=(k_scale, v_scale),
+                         group_table=group_table, group_count=group_count,
+                         qtile_table=qtile_table, qtile_count=qtile_count)
     return out, lse, kp, vp

@@ -95,7 +95,7 @@ def lib() -> ctypes.CDLL:
         L.rpa_forward.restype = ctypes.c_int
         L.rpa_write_kv8.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P]
         L.rpa_write_kv8.restype = ctypes.c_int
-        L.rpa_forward_kv8.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
+        L.rpa_forward_kv8.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
                                       ctypes.c_float, _P, _P, _P, ctypes.c_size_t, _P]
         L.rpa_forward_kv8.restype = ctypes.c_int
         L.rpa_forward_no_alloc.argtypes = [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P,
@@ -231,7 +231,7 @@ def rpa_plan_device(*, num_seqs: int, max_tokens: int, num_q_heads: int, num_kv_
     """A plan whose work lists are built on the device at every call (CUDA-graph friendly):
     B = num_seqs sequences, at most max_tokens new tokens and max_kv_len keys per step.  The
     q / k_new / v_new / out / lse buffers of the calls hold max_tokens rows.  kv_e4m3: for
-    rpa_forward_kv8; every row must fit the decode kernel."""
+    rpa_forward_kv8."""
     shape = Shape(num_seqs, max_tokens, num_q_heads, num_kv_heads, head_dim, page_size,
                   num_pages, max_blocks_per_seq, layout, 1 if causal else 0)
     opts = PlanOptions(0, decode_split_keys, 0, 1 if kv_e4m3 else 0)
@@ -274,15 +274,17 @@ def rpa_write_kv8(plan: Plan, k_new, v_new, k_pool, v_pool, k_scale, v_scale, bl
 
 def rpa_forward_kv8(plan: Plan, q, k_new, v_new, k_pool, v_pool, k_scale, v_scale,
                     block_table, cu_seqlens_q, seq_lens_k, scale: float, out, lse, workspace,
-                    stream=None):
+                    stream=None, group_table=None, group_count=None):
     """The fused step over e4m3 (uint8) K/V pools with fp32 per-KV-head scales
-    k_scale, v_scale [Hkv] (head_dim 128, no group tables).  Plans with rows for the
-    tensor-core kernel, and device plans, must be made with kv_e4m3=True; see include/rpa.h."""
+    k_scale, v_scale [Hkv] (head_dim 128); group_table / group_count for sparse plans.
+    Plans with rows for the tensor-core kernel, and device plans, must be made with
+    kv_e4m3=True; see include/rpa.h."""
     nbytes = workspace.numel() * workspace.element_size() if workspace is not None else 0
     _check("rpa_forward_kv8", lib().rpa_forward_kv8(
         plan.handle, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(k_pool), _ptr(v_pool),
         _ptr(k_scale), _ptr(v_scale), _ptr(block_table), _ptr(cu_seqlens_q), _ptr(seq_lens_k),
-        ctypes.c_float(scale), _ptr(out), _ptr(lse), _ptr(workspace), nbytes, _stream(stream)))
+        _ptr(group_table), _ptr(group_count), ctypes.c_float(scale), _ptr(out), _ptr(lse),
+        _ptr(workspace), nbytes, _stream(stream)))
 
 
 def no_alloc_workspace_bytes() -> int:

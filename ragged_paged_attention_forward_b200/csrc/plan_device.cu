@@ -78,10 +78,6 @@ __global__ void __launch_bounds__(kPlanThreads) plan_device_kernel(PlanDeviceLau
         atomicOr(p.err, kErrLimits);
         q_len = 0;
       }
-      if (q_len > 0 && p.no_prefill && q_len * G > p.decode_rows) {
-        atomicOr(p.err, kErrLimits);  // e4m3 device plans: decode rows only
-        q_len = 0;
-      }
       if (q_len > 0) {
         dec = q_len * G <= p.decode_rows;
         if (dec) {

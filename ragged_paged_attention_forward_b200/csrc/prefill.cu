@@ -32,6 +32,11 @@
 //               previous P.V finished), so the softmax never waits on P.V otherwise.
 // TMEM columns: S_A [0,128) S_B [128,256) O_A [256,256+D) O_B [384,384+D).  Bounded waits.
 // An odd GQA group size runs with head B switched off.
+// e4m3 pools (kKv8): the K/V boxes bring one-byte codes into the upper half of their slot;
+// warps 2-3 expand each row in place to f16 (e4m3 -> f16 is exact) and convert the unit's Q
+// from bf16 to f16 (exact in f16's range), so the MMAs run kind::f16 on f16 operands.  P is
+// then written as f16, whose range ends at 65504, so a tile is redone once its row sum passes
+// 2^15 instead of 2^64.  The score scale carries the KV head's k_scale, the output its v_scale.
 #include <cuda_bf16.h>
 #include <type_traits>
 #include <math_constants.h>
@@ -49,7 +54,8 @@ constexpr int kRows = kPrefillTileRows;  // 128
 static_assert(kRows == 128, "query-tile table rows are q_start >> 7");
 constexpr int kKeys = kPrefillTileKeys;  // 128
 constexpr uint32_t kTmemCols = 512;
-constexpr float kMaxTileSum = 0x1p64f;  // a tile whose row sum passes this is redone
+constexpr float kMaxTileSum = 0x1p64f;    // a tile whose row sum passes this is redone
+constexpr float kMaxTileSumF16 = 0x1p15f;  // the same with P as f16 (e4m3 pools)
 // Registers: the CTA launches with kLaunchRegs per thread (3 warpgroups); the producer/MMA
 // warpgroup gives most of its share to the two softmax warpgroups.
 constexpr int kLaunchRegs = 168;
@@ -67,8 +73,8 @@ struct PfGeom {
   static constexpr int kVOff = kKOff + kStagesK * kTileBytes;
   static constexpr int kBarOff = kVOff + kStagesV * kTileBytes;
   // q_full, k_full[S], v_full[S], k_empty[S], v_empty[S], s_full[2], p_ready[2], o_done[2],
-  // q_empty, mma_done
-  static constexpr int kNumBars = 1 + 2 * kStagesK + 2 * kStagesV + 6 + 2;
+  // q_empty, mma_done, q_conv, k_conv[S], v_conv[S]
+  static constexpr int kNumBars = 1 + 2 * kStagesK + 2 * kStagesV + 6 + 2 + 1 + kStagesK + kStagesV;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kBytes = kMiscOff + 64;
   // at least 120 KB so that a second CTA never shares the SM (and its 512 TMEM columns)
@@ -114,7 +120,7 @@ struct Unit {
   int n_tiles;           // 128-key tiles
 };
 
-template <int D, bool kFuse>
+template <int D, bool kFuse, bool kKv8>
 __global__ void __launch_bounds__(kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap qmap,
                    const __grid_constant__ CUtensorMap kmap,
@@ -123,6 +129,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap vnmap, PrefillLaunch p,
                    const __grid_constant__ PrefillTilesInline inl) {
   using Geo = PfGeom<D>;
+  static_assert(!(kFuse && kKv8), "the fused KV write is for bf16 pools");
+  static_assert(!kKv8 || D == 128, "e4m3 pools: head_dim 128");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -140,6 +148,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* o_done = p_ready + 2;           // [2]
   uint64_t* q_empty = o_done + 2;           // the unit's S MMAs are done with Q
   uint64_t* mma_done = q_empty + 1;
+  // e4m3 pools: the f16 operands are ready (one arrival per converting warp)
+  uint64_t* q_conv = mma_done + 1;
+  uint64_t* k_conv = q_conv + 1;           // [kStagesK]
+  uint64_t* v_conv = k_conv + kStagesK;    // [kStagesV]
   uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(smem + Geo::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Geo::kMiscOff + 8);
   volatile int* never = reinterpret_cast<volatile int*>(smem + Geo::kMiscOff + 12);  // stays 0
@@ -195,6 +207,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     return w;
   };
+  // rows of key tile j that hold real keys of the sequence (the rest of the slot is stale or
+  // a tail past the sequence end)
+  auto valid_keys = [&](const Unit& w, int j) {
+    if (w.table) {
+      const int per = kKeys >> log2P;
+      const int ne = min(per, w.n_entries - j * per);
+      const int last = __ldg(w.table + j * per + ne - 1);
+      return (ne - 1) * P + min(P, w.tile.kv_len - (last << log2P));
+    }
+    const int covered = min(w.tile.kv_len, ((w.kv_hi + P - 1) >> log2P) << log2P);
+    return min(kKeys, covered - j * kKeys);
+  };
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
@@ -213,6 +237,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&o_done[x], 1);
     }
     mbar_init(mma_done, 1);
+    mbar_init(q_conv, 2);
+    for (int s = 0; s < kStagesK; ++s) mbar_init(&k_conv[s], 2);
+    for (int s = 0; s < kStagesV; ++s) mbar_init(&v_conv[s], 2);
     *abort_flag = 0;
     *never = 0;
     fence_mbar_init();
@@ -277,7 +304,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int fuse_edge =
             kFuse && p.fuse_rows > 0 ? (w.past + p.fuse_rows - 1) / p.fuse_rows * p.fuse_rows
                                      : -1;
-        const uint32_t box_bytes = (uint32_t)box_rows * 128u * Geo::kHalves;
+        // bf16: two 128-byte halves per row; e4m3: one 128-byte run of codes per row, into
+        // the slot's upper half (expanded to f16 in place by the converting warps)
+        constexpr int kLoads = kKv8 ? 1 : Geo::kHalves;
+        constexpr int kDst0 = kKv8 ? Geo::kHalfBytes : 0;
+        const uint32_t box_bytes = (uint32_t)box_rows * 128u * kLoads;
         for (int j = 0; !stop && j < w.n_tiles; ++j) {
           const int it = kv_iter++;
           int nbox, first_blk = 0, slot0 = 0;
@@ -344,8 +375,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               else if (kv == 0)
                 atomicOr(p.err, kErrBadIndex);
 #pragma unroll
-              for (int half = 0; half < Geo::kHalves; ++half)
-                tma_load_4d(dst_base + half * Geo::kHalfBytes + i * box_rows * 128, map,
+              for (int half = 0; half < kLoads; ++half)
+                tma_load_4d(dst_base + kDst0 + half * Geo::kHalfBytes + i * box_rows * 128, map,
                             half * 64, hcoord, slot0, page, bar);
             }
             issued[kv] = it + 1;
@@ -369,8 +400,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
-    constexpr uint32_t idesc_s = idesc_bf16_f32(128, kKeys, false, false);
-    constexpr uint32_t idesc_o = idesc_bf16_f32(128, D, false, true);
+    constexpr uint32_t idesc_s = kKv8 ? idesc_f16_f32(128, kKeys, false, false)
+                                      : idesc_bf16_f32(128, kKeys, false, false);
+    constexpr uint32_t idesc_o =
+        kKv8 ? idesc_f16_f32(128, D, false, true) : idesc_bf16_f32(128, D, false, true);
+    // operands are ready: TMA done (bf16), or converted to f16 (e4m3 pools)
+    uint64_t* const q_in = kKv8 ? q_conv : q_full;
+    uint64_t* const k_in = kKv8 ? k_conv : k_full;
+    uint64_t* const v_in = kKv8 ? v_conv : v_full;
     // Descriptors are built once; an MMA's operands differ from the base only in the start
     // address field (bits 0..13, in 16-byte units, no carry for addresses below 256 KB), so
     // each MMA needs one add per operand instead of rebuilding a 64-bit descriptor.
@@ -415,8 +452,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // The unit's first S goes in as soon as its Q and first K tile are in: the softmax
       // warps are still writing out the previous unit's O (the first P.V of this unit, which
       // overwrites O, waits for their P, which they produce only after that).
-      ok = warp_wait_bounded(q_full, q_iter & 1, abort_flag, p.err, kErrPrefillWait) &&
-           warp_wait_bounded(&k_full[kv_iter % kStagesK], (kv_iter / kStagesK) & 1,
+      ok = warp_wait_bounded(q_in, q_iter & 1, abort_flag, p.err, kErrPrefillWait) &&
+           warp_wait_bounded(&k_in[kv_iter % kStagesK], (kv_iter / kStagesK) & 1,
                              abort_flag, p.err, kErrPrefillWait);
       ++q_iter;
       if (!ok) break;
@@ -430,23 +467,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int j = 0; ok && j < w.n_tiles; ++j) {
         const int it = kv_iter + j;
         const int slot = it % kStagesV;
-        if (!warp_wait_bounded(&v_full[slot], (it / kStagesV) & 1, abort_flag, p.err,
+        if (!warp_wait_bounded(&v_in[slot], (it / kStagesV) & 1, abort_flag, p.err,
                                kErrPrefillWait)) {
           ok = false;
           break;
         }
         // V rows past the last real key may hold anything (NaN tail slots, a stale tile):
-        // P = 0 there does not cancel a NaN in the product, so the rows are zeroed.
-        int nvalid;
-        if (w.table) {
-          const int per = kKeys >> log2P;
-          const int ne = min(per, w.n_entries - j * per);
-          const int last = __ldg(w.table + j * per + ne - 1);
-          nvalid = (ne - 1) * P + min(P, w.tile.kv_len - (last << log2P));
-        } else {
-          const int covered = min(w.tile.kv_len, ((w.kv_hi + P - 1) >> log2P) << log2P);
-          nvalid = min(kKeys, covered - j * kKeys);
-        }
+        // P = 0 there does not cancel a NaN in the product, so the rows are zeroed (by the
+        // converting warps for e4m3 pools).
+        const int nvalid = kKv8 ? kKeys : valid_keys(w, j);
         if (nvalid < kKeys) {
           uint8_t* vt = Vs + slot * Geo::kTileBytes;
           const int n16 = (kKeys - nvalid) * Geo::kHalves * 8;
@@ -475,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           __syncwarp();
           if (more) {
-            if (!warp_wait_bounded(&k_full[nslot], ((it + 1) / kStagesK) & 1, abort_flag,
+            if (!warp_wait_bounded(&k_in[nslot], ((it + 1) / kStagesK) & 1, abort_flag,
                                    p.err, kErrPrefillWait)) {
               ok = false;
               break;
@@ -561,6 +590,87 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int q = 0; q < 4; ++q)
           if (dst[q]) __stcs(dst[q], val[q]);  // streaming: nothing here reads them again
       }
+    }
+  } else if (kKv8) {
+    // ------------------------------------------------------------------ e4m3 -> f16 (warps 2-3)
+    // Each unit's Q tiles are converted in place (bf16 -> f16, position for position); each
+    // K and V tile's codes, which the TMA put in the upper half of the slot (row r's 128 codes
+    // in the 128-byte line of row r, 16-byte chunk c at chunk c ^ (r & 7), the 128-byte
+    // swizzle), are expanded into both halves of the slot in the layout a bf16 tile has.  A
+    // thread does whole rows: the upper half of row r is written only after all its codes were
+    // read (dims 0..63 go to the lower half first), so the expansion is in place.  V rows past
+    // the tile's last real key are written as zeros.
+    const int wt = (warp - 2) * 32 + lane;
+    // rows wt and wt + 64 of a tile (same swizzle phase), one 16-byte chunk of each per step
+    auto expand_rows = [&](uint8_t* t, bool valid0, bool valid1) {
+      uint8_t* line0 = t + wt * 128;
+      uint8_t* line1 = t + Geo::kHalfBytes + wt * 128;
+      const int sw = wt & 7;
+#pragma unroll 1
+      for (int c = 0; c < 8; ++c) {  // codes of dims 16c .. 16c + 15
+        const int ic = (c ^ sw) << 4;
+        const U4 in0 = valid0 ? *reinterpret_cast<const U4*>(line1 + ic) : U4{0u, 0u, 0u, 0u};
+        const U4 in1 =
+            valid1 ? *reinterpret_cast<const U4*>(line1 + 64 * 128 + ic) : U4{0u, 0u, 0u, 0u};
+        uint8_t* out = c < 4 ? line0 : line1;
+        const int oc = 2 * (c & 3);  // chunk of dims 16c .. 16c + 7 within its half
+        const int o0 = (oc ^ sw) << 4, o1 = ((oc + 1) ^ sw) << 4;
+        *reinterpret_cast<U4*>(out + o0) =
+            U4{e4m3x2_to_f16x2(in0.x), e4m3x2_to_f16x2(in0.x >> 16), e4m3x2_to_f16x2(in0.y),
+               e4m3x2_to_f16x2(in0.y >> 16)};
+        *reinterpret_cast<U4*>(out + o1) =
+            U4{e4m3x2_to_f16x2(in0.z), e4m3x2_to_f16x2(in0.z >> 16), e4m3x2_to_f16x2(in0.w),
+               e4m3x2_to_f16x2(in0.w >> 16)};
+        *reinterpret_cast<U4*>(out + 64 * 128 + o0) =
+            U4{e4m3x2_to_f16x2(in1.x), e4m3x2_to_f16x2(in1.x >> 16), e4m3x2_to_f16x2(in1.y),
+               e4m3x2_to_f16x2(in1.y >> 16)};
+        *reinterpret_cast<U4*>(out + 64 * 128 + o1) =
+            U4{e4m3x2_to_f16x2(in1.z), e4m3x2_to_f16x2(in1.z >> 16), e4m3x2_to_f16x2(in1.w),
+               e4m3x2_to_f16x2(in1.w >> 16)};
+      }
+    };
+    bool ok = true;
+    int kv_iter = 0;  // K/V tiles converted, over all units of this CTA
+    int q_iter = 0;   // units with key tiles
+    for (int k = 0; ok; ++k) {
+      const int u = unit_index(k);
+      if (u >= num_units) break;
+      const Unit w = unit_at(u);
+      if (w.n_tiles == 0) continue;
+      ok = warp_wait_bounded(q_full, q_iter & 1, abort_flag, p.err, kErrPrefillWait);
+      ++q_iter;
+      if (!ok) break;
+      for (int i = wt; i < hpc * Geo::kTileBytes / 16; i += 64) {
+        U4* c = reinterpret_cast<U4*>(Qs) + i;
+        U4 v = *c;
+        v.x = bf16x2_to_f16x2(v.x);
+        v.y = bf16x2_to_f16x2(v.y);
+        v.z = bf16x2_to_f16x2(v.z);
+        v.w = bf16x2_to_f16x2(v.w);
+        *c = v;
+      }
+      fence_proxy_async_smem();  // the tensor cores read these through the async proxy
+      __syncwarp();
+      if (lane == 0) mbar_arrive(q_conv);
+      for (int j = 0; ok && j < w.n_tiles; ++j) {
+        const int it = kv_iter + j;
+        const int nvalid = valid_keys(w, j);
+        for (int kv = 0; kv < 2; ++kv) {
+          const int ns = kv == 0 ? kStagesK : kStagesV;
+          const int slot = it % ns;
+          if (!warp_wait_bounded(kv == 0 ? &k_full[slot] : &v_full[slot], (it / ns) & 1,
+                                 abort_flag, p.err, kErrPrefillWait)) {
+            ok = false;
+            break;
+          }
+          uint8_t* t = (kv == 0 ? Ks : Vs) + slot * Geo::kTileBytes;
+          expand_rows(t, kv == 0 || wt < nvalid, kv == 0 || wt + 64 < nvalid);
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(kv == 0 ? &k_conv[slot] : &v_conv[slot]);
+        }
+      }
+      kv_iter += w.n_tiles;
     }
   }
   } else if ((warp - 4) / 4 < hpc) {
@@ -707,7 +817,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 p1 = (vis[(c + 1) >> 5] >> ((c + 1) & 31)) & 1u ? p1 : 0.f;
               }
               rsum2[(c >> 1) & 3] = f2_add(rsum2[(c >> 1) & 3], f2_pack(p0, p1));
-              sr[c >> 1] = pack_bf16(p0, p1);  // P as bf16 pairs, over the consumed S values
+              // P as bf16 (f16 for e4m3 pools) pairs, over the consumed S values
+              sr[c >> 1] = kKv8 ? pack_f16(p0, p1) : pack_bf16(p0, p1);
             }
           };
           if (need_mask)
@@ -721,7 +832,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             f2_unpack(rsum2[k], a, b);
             rs += a + b;
           }
-          const bool over = !(rs <= kMaxTileSum);
+          const bool over = !(rs <= (kKv8 ? kMaxTileSumF16 : kMaxTileSum));
           if (attempt > 0 || !__any_sync(0xffffffffu, over)) break;
           need_max = over;
 #pragma unroll
@@ -805,12 +916,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-template <int D, bool kFuse>
+template <int D, bool kFuse, bool kKv8>
 cudaError_t launch_prefill_kernel(const CUtensorMap& qmap, const CUtensorMap& kmap,
                                   const CUtensorMap& vmap, const CUtensorMap& knmap,
                                   const CUtensorMap& vnmap, const PrefillLaunch& p,
                                   const PrefillTilesInline* inl, dim3 grid, cudaStream_t stream) {
-  const void* k = reinterpret_cast<const void*>(prefill_kernel<D, kFuse>);
+  const void* k = reinterpret_cast<const void*>(prefill_kernel<D, kFuse, kKv8>);
   // the register rebalancing inside the kernel needs exactly the launch budget it was
   // written for; refuse to launch otherwise (a short budget would stall setmaxnreg.inc)
   cudaFuncAttributes fa;
@@ -824,8 +935,8 @@ cudaError_t launch_prefill_kernel(const CUtensorMap& qmap, const CUtensorMap& km
   e = ensure_smem_attr(k, PfGeom<D>::kAlloc);
   if (e != cudaSuccess) return e;
   if (!p.launched) {
-    prefill_kernel<D, kFuse><<<grid, kThreads, PfGeom<D>::kAlloc, stream>>>(qmap, kmap, vmap,
-                                                                            knmap, vnmap, p, *inl);
+    prefill_kernel<D, kFuse, kKv8><<<grid, kThreads, PfGeom<D>::kAlloc, stream>>>(
+        qmap, kmap, vmap, knmap, vnmap, p, *inl);
     return cudaSuccess;
   }
   // the event fires once every CTA has started: work that waits for it on another stream
@@ -841,8 +952,8 @@ cudaError_t launch_prefill_kernel(const CUtensorMap& qmap, const CUtensorMap& km
   attr[0].val.launchCompletionEvent.flags = 0;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, prefill_kernel<D, kFuse>, qmap, kmap, vmap, knmap, vnmap, p,
-                            *inl);
+  return cudaLaunchKernelEx(&cfg, prefill_kernel<D, kFuse, kKv8>, qmap, kmap, vmap, knmap, vnmap,
+                            p, *inl);
 }
 
 cudaError_t launch_prefill(const PrefillLaunch& p, const PrefillTilesInline* inl,
@@ -880,14 +991,26 @@ cudaError_t launch_prefill(const PrefillLaunch& p, const PrefillTilesInline* inl
   }
   const dim3 grid((unsigned)ctas);
   const bool fuse = p.fuse_rows > 0;
-  if (p.head_dim == 128)
-    e = fuse ? launch_prefill_kernel<128, true>(qmap, kmap, vmap, knmap, vnmap, p, inl, grid, stream)
-             : launch_prefill_kernel<128, false>(qmap, kmap, vmap, knmap, vnmap, p, inl, grid,
-                                                 stream);
-  else
-    e = fuse ? launch_prefill_kernel<64, true>(qmap, kmap, vmap, knmap, vnmap, p, inl, grid, stream)
-             : launch_prefill_kernel<64, false>(qmap, kmap, vmap, knmap, vnmap, p, inl, grid,
+  if (p.kv.kv8) {
+    // e4m3 pools: codes converted inside the kernel (head_dim 128, no fused write)
+    if (p.head_dim != 128 || fuse || !p.k_scale || !p.v_scale) {
+      set_last_error("e4m3 pools on the tensor-core kernel need head_dim 128, both scale "
+                     "vectors and no fused write");
+      return cudaErrorInvalidValue;
+    }
+    e = launch_prefill_kernel<128, false, true>(qmap, kmap, vmap, knmap, vnmap, p, inl, grid,
                                                 stream);
+  } else if (p.head_dim == 128) {
+    e = fuse ? launch_prefill_kernel<128, true, false>(qmap, kmap, vmap, knmap, vnmap, p, inl,
+                                                       grid, stream)
+             : launch_prefill_kernel<128, false, false>(qmap, kmap, vmap, knmap, vnmap, p, inl,
+                                                        grid, stream);
+  } else {
+    e = fuse ? launch_prefill_kernel<64, true, false>(qmap, kmap, vmap, knmap, vnmap, p, inl,
+                                                      grid, stream)
+             : launch_prefill_kernel<64, false, false>(qmap, kmap, vmap, knmap, vnmap, p, inl,
+                                                       grid, stream);
+  }
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

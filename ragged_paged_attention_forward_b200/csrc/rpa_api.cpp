@@ -64,10 +64,6 @@ struct rpa_plan_s {
   // workspace layout: [decode items][merge rows][prefill tiles] | [partial O][partial LSE]
   size_t off_dec = 0, off_merge = 0, off_pf = 0, meta_bytes = 0;
   size_t off_part_o = 0, off_part_lse = 0, ws_bytes = 0;
-  // e4m3 plans with tensor-core rows: bf16 copy of those sequences' context in the workspace
-  std::vector<uint8_t> meta8;       // host image: scratch block table | seqs | row offsets
-  size_t off_s8 = 0, off_s8_seqs = 0, off_s8_rows = 0, off_s8_k = 0, off_s8_v = 0;
-  int s8_list = 0, s8_rows = 0, s8_pages = 0;
   std::vector<uint8_t> meta;  // host image of the metadata region
   // every list short enough to travel as kernel parameters: no work-list copy at all
   bool inline_lists = false;
@@ -250,8 +246,6 @@ rpa_status rpa_plan(const rpa_shape* shape, const int32_t* cu_seqlens_q,
     RPA_FAIL(RPA_ERR_INVALID_ARG, "opts.kv_e4m3 %d must be 0 or 1", o.kv_e4m3);
   if (o.kv_e4m3 && s.head_dim != 128)
     RPA_FAIL(RPA_ERR_UNSUPPORTED, "e4m3 pools need head_dim 128 (got %d)", s.head_dim);
-  if (o.kv_e4m3 && o.sparse)
-    RPA_FAIL(RPA_ERR_UNSUPPORTED, "e4m3 pools: no group tables");
   if (o.force_class < RPA_CLASS_AUTO || o.force_class > RPA_CLASS_MIXED)
     RPA_FAIL(RPA_ERR_INVALID_ARG, "unknown force_class %d", o.force_class);
   if (o.decode_split_keys != 0 &&
@@ -398,45 +392,6 @@ rpa_status rpa_plan(const rpa_shape* shape, const int32_t* cu_seqlens_q,
   off = align_up(off + (size_t)slots * s.num_kv_heads * rows_per_item * s.head_dim * 4, 256);
   plan->off_part_lse = off;
   off = align_up(off + (size_t)slots * s.num_kv_heads * rows_per_item * 4, 256);
-  if (o.kv_e4m3 && !plan->pf_tiles.empty()) {
-    // scratch pages in sequence order, per sequence ceil(kv_len / P) of them (head-major:
-    // one page per KV head and block), addressed by a block table of the pool's shape
-    const int P = s.page_size;
-    const int heads_t = s.layout == RPA_LAYOUT_HEAD_MAJOR ? s.num_kv_heads : 1;
-    const size_t tbl = (size_t)B * heads_t * s.max_blocks_per_seq;
-    std::vector<int32_t> table(tbl, 0), seqs, rows(1, 0);
-    std::vector<char> is_pf(B, 0);
-    for (const PrefillTile& t : plan->pf_tiles) is_pf[t.seq] = 1;
-    int base = 0;
-    for (int b = 0; b < B; ++b) {
-      if (!is_pf[b]) continue;
-      const int nb = (seq_lens_k[b] + P - 1) / P;
-      for (int h = 0; h < heads_t; ++h)
-        for (int j = 0; j < nb; ++j)
-          table[((size_t)b * heads_t + h) * s.max_blocks_per_seq + j] =
-              heads_t == 1 ? base + j : (base + j) * heads_t + h;
-      base += nb;
-      seqs.push_back(b);
-      rows.push_back(rows.back() + seq_lens_k[b]);
-    }
-    plan->s8_list = (int)seqs.size();
-    plan->s8_rows = rows.back();
-    plan->s8_pages = base * heads_t;
-    const size_t tb = tbl * 4, sb = seqs.size() * 4, rb = rows.size() * 4;
-    plan->meta8.assign(align_up(tb, 256) + align_up(sb, 256) + rb, 0);
-    memcpy(plan->meta8.data(), table.data(), tb);
-    memcpy(plan->meta8.data() + align_up(tb, 256), seqs.data(), sb);
-    memcpy(plan->meta8.data() + align_up(tb, 256) + align_up(sb, 256), rows.data(), rb);
-    plan->off_s8 = off;
-    plan->off_s8_seqs = off + align_up(tb, 256);
-    plan->off_s8_rows = plan->off_s8_seqs + align_up(sb, 256);
-    off = align_up(off + plan->meta8.size(), 256);
-    const size_t pool = (size_t)plan->s8_pages * P * (s.num_kv_heads / heads_t) * s.head_dim * 2;
-    plan->off_s8_k = off;
-    off = align_up(off + pool, 256);
-    plan->off_s8_v = off;
-    off = align_up(off + pool, 256);
-  }
   plan->ws_bytes = std::max<size_t>(off, 256);
   plan->meta.assign(plan->meta_bytes, 0);
   if (!plan->dec_items.empty())
@@ -565,8 +520,8 @@ rpa_status rpa_plan_device(const rpa_shape* shape, int32_t max_kv_len,
   off = align_up(off + (size_t)plan->cap_items * s.num_kv_heads * rows_per_item * 4, 256);
   plan->ws_bytes = off;
   plan->launches_write = 1;
-  // planner, KV write, tensor-core, decode, merge; e4m3 plans: planner, decode, merge
-  plan->launches_forward = o.kv_e4m3 ? 3 : 5;
+  // planner, KV write, tensor-core, decode, merge
+  plan->launches_forward = 5;
   *out_plan = plan;
   if (workspace_bytes) *workspace_bytes = plan->ws_bytes;
   return RPA_OK;
@@ -819,38 +774,6 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
   st = check_cuda(device_error_word(&err), "device error word");
   if (st != RPA_OK) return st;
 
-  int* err8 = nullptr;
-  if (kv8 && !plan->pf_tiles.empty()) {
-    // e4m3 pools: the tensor-core rows read an exact bf16 copy of their sequences' context
-    // (scales folded into the kernel's score scale and output), made after the write
-    uint8_t* w8 = static_cast<uint8_t*>(workspace);
-    st = check_cuda(cudaMemcpyAsync(w8 + plan->off_s8, plan->meta8.data(), plan->meta8.size(),
-                                    cudaMemcpyHostToDevice, stream),
-                    "scratch table copy");
-    if (st != RPA_OK) return st;
-    st = check_cuda(device_error_word(&err8), "device error word");
-    if (st != RPA_OK) return st;
-    DequantLaunch q{};
-    q.k_pool = static_cast<const uint8_t*>(k_pool);
-    q.v_pool = static_cast<const uint8_t*>(v_pool);
-    q.block_table = block_table;
-    q.k_out = reinterpret_cast<uint16_t*>(w8 + plan->off_s8_k);
-    q.v_out = reinterpret_cast<uint16_t*>(w8 + plan->off_s8_v);
-    q.out_table = reinterpret_cast<const int32_t*>(w8 + plan->off_s8);
-    q.seqs = reinterpret_cast<const int32_t*>(w8 + plan->off_s8_seqs);
-    q.row_off = reinterpret_cast<const int32_t*>(w8 + plan->off_s8_rows);
-    q.num_list = plan->s8_list;
-    q.num_rows = plan->s8_rows;
-    q.num_kv_heads = s.num_kv_heads;
-    q.head_dim = s.head_dim;
-    q.page_size = s.page_size;
-    q.max_blocks = s.max_blocks_per_seq;
-    q.layout = s.layout;
-    q.num_pages = s.num_pages;
-    q.err = err8;
-    st = check_cuda(launch_dequant_kv8(q, stream), "e4m3 copy launch");
-    if (st != RPA_OK) return st;
-  }
   PagedKV kv;
   kv.k_pool = k_pool;
   kv.v_pool = v_pool;
@@ -879,7 +802,6 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     pl.causal = s.causal;
     pl.split_keys = plan->split_keys;
     pl.decode_rows = 8 * plan->decode_nt;
-    pl.no_prefill = kv8 ? 1 : 0;
     pl.cap_items = plan->cap_items;
     pl.cap_rows = plan->cap_rows;
     pl.cap_tiles = plan->cap_tiles;
@@ -892,9 +814,7 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     if (st != RPA_OK) return st;
     // both kernel families: the tensor-core kernel on the side stream, forked after the
     // planner, the decode kernel and the merge on the caller's stream; joined at the end.
-    // e4m3 device plans run decode rows only (the planner refused the others): no fork.
     cudaStream_t pf_stream = stream;
-    if (!kv8) {
     st = check_cuda(side_stream(stream, &pf_stream), "side stream");
     if (st != RPA_OK) return st;
     if (!plan->fork_ev) {
@@ -913,7 +833,8 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     // scatter kernel, on the side stream ahead of the tensor-core kernel, writes the rest
     if (k_new) {
       st = write_kv_impl(plan, k_new, v_new, k_pool, v_pool, block_table, cu_seqlens_q,
-                         seq_lens_k, pf_stream, 8 * plan->decode_nt);
+                         seq_lens_k, pf_stream, 8 * plan->decode_nt, kv8 ? k_scale : nullptr,
+                         kv8 ? v_scale : nullptr);
       if (st != RPA_OK) return st;
     }
     PrefillLaunch p{};
@@ -931,9 +852,10 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     p.lse = lse;
     p.err = err;
     p.kv = kv;
+    p.k_scale = kv8 ? k_scale : nullptr;
+    p.v_scale = kv8 ? v_scale : nullptr;
     st = check_cuda(launch_prefill(p, &plan->pf_inline, pf_stream), "prefill launch");
     if (st != RPA_OK) return st;
-    }
     DecodeLaunch d{};
     d.items = pl.items;
     d.num_items = plan->cap_items;
@@ -974,7 +896,6 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
     m.lse = lse;
     st = check_cuda(launch_merge(m, &plan->merge_inline, stream), "merge launch");
     if (st != RPA_OK) return st;
-    if (kv8) return RPA_OK;
     st = check_cuda(cudaEventRecord(plan->join_ev, pf_stream), "join record");
     if (st != RPA_OK) return st;
     return check_cuda(cudaStreamWaitEvent(stream, plan->join_ev, 0), "join wait");
@@ -1052,12 +973,7 @@ static rpa_status forward_impl(rpa_plan_t plan, const void* q, const void* k_new
       p.fuse_rows = fuse_box;
     }
     if (kv8) {
-      // the bf16 scratch copy, through its own block table
-      p.kv.k_pool = ws + plan->off_s8_k;
-      p.kv.v_pool = ws + plan->off_s8_v;
-      p.kv.block_table = reinterpret_cast<const int32_t*>(ws + plan->off_s8);
-      p.kv.num_pages = plan->s8_pages;
-      p.kv.kv8 = 0;
+      // the codes are read in place and converted inside the kernel
       p.k_scale = k_scale;
       p.v_scale = v_scale;
     }
@@ -1135,7 +1051,8 @@ rpa_status rpa_forward(rpa_plan_t plan, const void* q, const void* k_new, const 
 rpa_status rpa_forward_kv8(rpa_plan_t plan, const void* q, const void* k_new, const void* v_new,
                            void* k_pool, void* v_pool, const float* k_scale,
                            const float* v_scale, const int32_t* block_table,
-                           const int32_t* cu_seqlens_q, const int32_t* seq_lens_k, float scale,
+                           const int32_t* cu_seqlens_q, const int32_t* seq_lens_k,
+                           const int32_t* group_table, const int32_t* group_count, float scale,
                            void* out, float* lse, void* workspace, size_t workspace_bytes,
                            void* stream) {
   g_last_error.clear();
@@ -1150,13 +1067,12 @@ rpa_status rpa_forward_kv8(rpa_plan_t plan, const void* q, const void* k_new, co
     RPA_FAIL(RPA_ERR_UNSUPPORTED,
              "e4m3 pools with rows for the tensor-core kernel need a plan made with "
              "opts.kv_e4m3 = 1");
-  if (plan->opts.sparse) RPA_FAIL(RPA_ERR_UNSUPPORTED, "e4m3 pools: no group tables");
   if (!k_scale || !v_scale) RPA_FAIL(RPA_ERR_INVALID_ARG, "k_scale and v_scale are required");
   if ((reinterpret_cast<uintptr_t>(k_scale) & 3u) || (reinterpret_cast<uintptr_t>(v_scale) & 3u))
     RPA_FAIL(RPA_ERR_INVALID_ARG, "k_scale / v_scale must be 4-byte aligned");
   return forward_impl(plan, q, k_new, v_new, k_pool, v_pool, block_table, cu_seqlens_q,
-                      seq_lens_k, nullptr, nullptr, scale, out, lse, workspace, workspace_bytes,
-                      stream, true, k_scale, v_scale);
+                      seq_lens_k, group_table, group_count, scale, out, lse, workspace,
+                      workspace_bytes, stream, true, k_scale, v_scale);
 }
 
 rpa_status rpa_build_group_tables(const uint8_t* mask, int32_t num_seqs, int32_t num_q_heads,

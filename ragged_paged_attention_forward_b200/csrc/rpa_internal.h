@@ -209,31 +209,6 @@ struct WriteLaunch {
   int* err;
 };
 
-// e4m3 -> bf16 copy of the context of the sequences that the tensor-core kernel reads: row r
-// of the work list is key position pos of sequence seqs[i] (row_off[i] <= r < row_off[i+1],
-// pos = r - row_off[i]); every KV head's K and V row of that position is converted exactly
-// (every e4m3 value is a bf16 value; the scale is not applied) from the code pools, through
-// block_table, into the bf16 scratch pools, through out_table (same layout).
-struct DequantLaunch {
-  const uint8_t* k_pool;
-  const uint8_t* v_pool;
-  const int32_t* block_table;
-  uint16_t* k_out;
-  uint16_t* v_out;
-  const int32_t* out_table;
-  const int32_t* seqs;
-  const int32_t* row_off;
-  int32_t num_list;          // entries of seqs
-  int32_t num_rows;          // row_off[num_list]
-  int32_t num_kv_heads;
-  int32_t head_dim;
-  int32_t page_size;
-  int32_t max_blocks;
-  int32_t layout;
-  int32_t num_pages;
-  int* err;
-};
-
 struct RotaryLaunch {
   const uint16_t* q;      // [T, Hq, D] or packed [T, (Hq + 2 Hkv) D]
   const uint16_t* k;      // [T, Hkv, D] or null (packed)
@@ -275,7 +250,6 @@ struct PlanDeviceLaunch {
   int32_t causal;
   int32_t split_keys;
   int32_t decode_rows;           // a sequence goes to the decode kernel when q_len * G <= this
-  int32_t no_prefill;            // 1: a sequence past decode_rows raises kErrLimits, is skipped
   int32_t cap_items, cap_rows, cap_tiles;
   DecodeItem* items;
   MergeRow* rows;
@@ -293,7 +267,6 @@ cudaError_t launch_decode(const DecodeLaunch& p, const DecodeItemsInline* inl, i
 cudaError_t launch_merge(const MergeLaunch& p, const MergeRowsInline* inl, cudaStream_t stream);
 cudaError_t launch_prefill(const PrefillLaunch& p, const PrefillTilesInline* inl,
                            cudaStream_t stream);
-cudaError_t launch_dequant_kv8(const DequantLaunch& p, cudaStream_t stream);
 cudaError_t launch_qtile_tables(const uint8_t* mask, int B, int Hq, int nqb, int nkb,
                                 int qb_per_tile, int ntiles, int32_t* table, int32_t* count,
                                 cudaStream_t stream);

@@ -116,78 +116,7 @@ __global__ void __launch_bounds__(256) write_kv_kernel(WriteLaunch p) {
   }
 }
 
-// One warp per (sequence, key position) row of the list: Hkv * D codes of K and of V become
-// bf16 (e4m3 -> f16 is exact, f16 -> f32 -> bf16 too for every e4m3 value).
-__global__ void __launch_bounds__(256) dequant_kv8_kernel(DequantLaunch p) {
-  const int warps_per_block = blockDim.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int nwarps = gridDim.x * warps_per_block;
-  const int chunks = p.head_dim / 16;  // 16-code chunks per D-row
-  const int row_chunks = p.num_kv_heads * chunks;
-  for (int r = blockIdx.x * warps_per_block + (threadIdx.x >> 5); r < p.num_rows; r += nwarps) {
-    int lo = 0, hi = p.num_list;  // row_off[lo] <= r < row_off[lo + 1]
-    while (hi - lo > 1) {
-      const int mid = (lo + hi) >> 1;
-      if (__ldg(p.row_off + mid) <= r) lo = mid; else hi = mid;
-    }
-    const int b = __ldg(p.seqs + lo);
-    const int pos = r - __ldg(p.row_off + lo);
-    const int blk = pos / p.page_size;
-    const int slot = pos - blk * p.page_size;
-    if (blk >= p.max_blocks) {
-      if (lane == 0) atomicOr(p.err, kErrBadIndex);
-      continue;
-    }
-    for (int c = lane; c < row_chunks; c += 32) {
-      const int h = c / chunks;
-      const int cc = c - h * chunks;
-      const size_t trow = p.layout == 0 ? (size_t)b * p.max_blocks + blk
-                                        : ((size_t)b * p.num_kv_heads + h) * p.max_blocks + blk;
-      const int page = __ldg(p.block_table + trow);
-      const int opage = __ldg(p.out_table + trow);
-      if (page < 0 || page >= p.num_pages) {
-        atomicOr(p.err, kErrBadIndex);
-        continue;
-      }
-      const size_t irow = p.layout == 0 ? ((size_t)page * p.page_size + slot) * p.num_kv_heads + h
-                                        : (size_t)page * p.page_size + slot;
-      const size_t orow = p.layout == 0
-                              ? ((size_t)opage * p.page_size + slot) * p.num_kv_heads + h
-                              : (size_t)opage * p.page_size + slot;
-#pragma unroll
-      for (int kv = 0; kv < 2; ++kv) {
-        const uint8_t* src = (kv == 0 ? p.k_pool : p.v_pool) + irow * p.head_dim + cc * 16;
-        uint16_t* dst = (kv == 0 ? p.k_out : p.v_out) + orow * p.head_dim + cc * 16;
-        const uint4 w = __ldg(reinterpret_cast<const uint4*>(src));
-        uint32_t o[8];
-        const uint32_t in[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t lo2 = e4m3x2_to_f16x2(in[i]);        // codes 0, 1 of the word
-          const uint32_t hi2 = e4m3x2_to_f16x2(in[i] >> 16);  // codes 2, 3
-          const float2 a = __half22float2(*reinterpret_cast<const __half2*>(&lo2));
-          const float2 bb = __half22float2(*reinterpret_cast<const __half2*>(&hi2));
-          o[2 * i] = pack_bf16(a.x, a.y);
-          o[2 * i + 1] = pack_bf16(bb.x, bb.y);
-        }
-        reinterpret_cast<uint4*>(dst)[0] = make_uint4(o[0], o[1], o[2], o[3]);
-        reinterpret_cast<uint4*>(dst)[1] = make_uint4(o[4], o[5], o[6], o[7]);
-      }
-    }
-  }
-}
-
 }  // namespace
-
-cudaError_t launch_dequant_kv8(const DequantLaunch& p, cudaStream_t stream) {
-  if (p.num_rows <= 0) return cudaSuccess;
-  const int threads = 256;
-  int blocks = (p.num_rows + 7) / 8;
-  const int cap = device_sm_count() * 8;
-  if (blocks > cap) blocks = cap;
-  dequant_kv8_kernel<<<blocks, threads, 0, stream>>>(p);
-  return cudaGetLastError();
-}
 
 cudaError_t launch_write_kv(const WriteLaunch& p, cudaStream_t stream) {
   if (p.num_tokens <= 0) return cudaSuccess;

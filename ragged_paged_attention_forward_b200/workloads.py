@@ -343,12 +343,14 @@ WORKLOADS = {
 E4M3_NAN_CODE = 0x7F
 
 
-def with_kv8_pools(batch: Batch, *, seed: int, poison: bool = True):
+def with_kv8_pools(batch: Batch, *, seed: int, poison: bool = True, full_range: bool = False):
     """The batch with uint8 e4m3 code pools instead of bf16 ones, plus scales.
 
     Returns ``(batch8, k_scale [Hkv] fp32, v_scale [Hkv] fp32)``.  Context positions
-    ``0 .. past-1`` of every sequence get random finite codes; all other slots get the NaN
-    code (or 0).  ``k_new``/``v_new`` stay bf16 (they are quantised by the step itself).
+    ``0 .. past-1`` of every sequence get random finite codes -- exponent fields 3..11, or,
+    with ``full_range``, every finite code (zeros and subnormals included); all other slots
+    get the NaN code (or 0).  ``k_new``/``v_new`` stay bf16 (they are quantised by the step
+    itself).
     """
     g = torch.Generator().manual_seed(int(seed))
     fill = E4M3_NAN_CODE if poison else 0
@@ -358,9 +360,12 @@ def with_kv8_pools(batch: Batch, *, seed: int, poison: bool = True):
 
     def draw(n):
         sign = torch.randint(0, 2, (n, Hkv, D), generator=g, dtype=torch.int32)
-        expo = torch.randint(3, 12, (n, Hkv, D), generator=g, dtype=torch.int32)
+        lo, hi = (0, 16) if full_range else (3, 12)
+        expo = torch.randint(lo, hi, (n, Hkv, D), generator=g, dtype=torch.int32)
         mant = torch.randint(0, 8, (n, Hkv, D), generator=g, dtype=torch.int32)
-        return ((sign << 7) | (expo << 3) | mant).to(torch.uint8)
+        code = (sign << 7) | (expo << 3) | mant
+        code = torch.where((code & 0x7F) == 0x7F, code - 1, code)  # NaN -> largest finite
+        return code.to(torch.uint8)
 
     bt = batch.block_table.to(torch.int64)
     for b, (kv, ql) in enumerate(zip(batch.kv_lens(), batch.q_lens())):

@@ -126,7 +126,8 @@ def test_launch_counts_with_the_write_in_the_kernels():
     # a past of 69 leaves new rows in a box with older keys: the scatter kernel runs for them
     st = wl.ragged_batch([300, 1000, 101], [300, 1, 32], 8, 2, 64, 16, seed=1, keep_logical=False)
     assert plan_for(st).info().launches_forward == 4
-    # e4m3 plans keep the quantising scatter kernel
+    # e4m3 plans keep the quantising scatter kernel (the tensor-core kernel reads the codes in
+    # place: no other launch)
     mx8 = wl.ragged_batch([300, 1000, 96], [300, 1, 32], 8, 2, 128, 16, seed=1, keep_logical=False)
     assert plan_for(mx8, kv_e4m3=True).info().launches_forward == 4
 
@@ -281,10 +282,9 @@ def test_forward_kv8_rejects_before_any_device_work():
         api.rpa_forward_kv8(plan, None, None, None, None, None, None, None, None, None, None,
                             0.1, None, None, None, stream=0)
     assert ei.value.status == api.RPA_ERR_INVALID_ARG
-    # a plan with a prefill row, a head_dim-64 plan and a sparse plan are unsupported
+    # a plan with a prefill row made without kv_e4m3 and a head_dim-64 plan are unsupported
     for kw in (dict(cu_seqlens_q=[0, 1, 200], num_tokens=200, seq_lens_k=[40, 200]),
-               dict(head_dim=64),
-               dict(layout=1, sparse=True)):
+               dict(head_dim=64)):
         plan = api.rpa_plan(**_shape(**kw))
         with pytest.raises(api.RPAError) as ei:
             api.rpa_forward_kv8(plan, None, None, None, None, None, None, None, None, None,
@@ -293,29 +293,24 @@ def test_forward_kv8_rejects_before_any_device_work():
 
 
 def test_kv_e4m3_plan_option():
-    # a plan with a tensor-core row: the e4m3 option adds the bf16 copy of that sequence's
-    # context (scratch table, lists, K and V copies) to the workspace
-    kw = dict(cu_seqlens_q=[0, 1, 200], num_tokens=200, seq_lens_k=[40, 200])
-    plain = api.rpa_plan(**_shape(**kw))
-    e4 = api.rpa_plan(**_shape(**kw), kv_e4m3=True)
-    copy = 2 * 13 * 16 * 8 * 128 * 2            # ceil(200 / 16) pages of K and of V, bf16
-    assert e4.workspace_bytes >= plain.workspace_bytes + copy
-    # decode-only plans need no copy
-    d_plain = api.rpa_plan(**_shape())
-    d_e4 = api.rpa_plan(**_shape(), kv_e4m3=True)
-    assert d_e4.workspace_bytes == d_plain.workspace_bytes
-    for bad, status in ((dict(head_dim=64), api.RPA_ERR_UNSUPPORTED),
-                        (dict(layout=1, sparse=True), api.RPA_ERR_UNSUPPORTED)):
-        with pytest.raises(api.RPAError) as ei:
-            api.rpa_plan(**_shape(**bad), kv_e4m3=True)
-        assert ei.value.status == status
+    # the tensor-core kernel converts the codes itself: an e4m3 plan needs no more workspace
+    # than a bf16 one, with or without tensor-core rows, and group tables are accepted
+    for kw in (dict(cu_seqlens_q=[0, 1, 200], num_tokens=200, seq_lens_k=[40, 200]), {}):
+        plain = api.rpa_plan(**_shape(**kw))
+        e4 = api.rpa_plan(**_shape(**kw), kv_e4m3=True)
+        assert e4.workspace_bytes == plain.workspace_bytes
+        assert e4.info().launches_forward == plain.info().launches_forward
+    api.rpa_plan(**_shape(layout=1, sparse=True), kv_e4m3=True)
+    with pytest.raises(api.RPAError) as ei:
+        api.rpa_plan(**_shape(head_dim=64), kv_e4m3=True)
+    assert ei.value.status == api.RPA_ERR_UNSUPPORTED
 
 
-def test_e4m3_device_plan_runs_decode_rows_only():
-    # planner, decode (with the quantising write of its rows) and merge: no scatter, no copy,
-    # no tensor-core launch and no side stream
+def test_e4m3_device_plan_runs_both_kernel_families():
+    # planner, quantising scatter and tensor-core kernel (side stream), decode (with the
+    # quantising write of its rows) and merge, as for bf16 pools
     p = _device_plan(kv_e4m3=True)
-    assert p.info().launches_forward == 3
+    assert p.info().launches_forward == 5
     assert _device_plan().info().launches_forward == 5
     with pytest.raises(api.RPAError) as e:
         _device_plan(kv_e4m3=True, head_dim=64)

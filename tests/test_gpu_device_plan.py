@@ -8,7 +8,8 @@ import torch
 from oracle import rpa_oracle as orc
 from ragged_paged_attention_forward_b200 import api
 from ragged_paged_attention_forward_b200 import workloads as wl
-from tests.rpa_testing import assert_close, assert_lse_close, oracle_forward
+from tests.rpa_testing import (assert_close, assert_kv8_close, assert_lse_close, kv8_vmax,
+                               oracle_forward)
 
 pytestmark = pytest.mark.gpu
 
@@ -117,14 +118,16 @@ def test_step_beyond_the_limits_is_reported():
     assert api.rpa_device_error(clear=True) & 16
 
 
-def test_e4m3_device_plan_graph_replays_decode_batches():
-    # a CUDA graph of rpa_forward_kv8 with a device plan made with kv_e4m3: the decode kernel
-    # quantises its rows' new tokens and reads the codes; replayed over two batches
+def test_e4m3_device_plan_graph_replays_any_batch():
+    # a CUDA graph of rpa_forward_kv8 with a device plan made with kv_e4m3, replayed over
+    # decode, short multi-token and long-chunk batches: the decode kernel quantises its rows'
+    # new tokens and reads the codes, the scatter kernel quantises the rest and the
+    # tensor-core kernel converts its tiles of codes to f16 itself
     plan = api.rpa_plan_device(num_seqs=B, max_tokens=MAX_T, num_q_heads=HQ, num_kv_heads=HKV,
                                head_dim=D, page_size=P, num_pages=NUM_PAGES,
                                max_blocks_per_seq=MAX_BLOCKS, layout=wl.SEQ_MAJOR, causal=True,
                                max_kv_len=MAX_KV, kv_e4m3=True)
-    assert plan.info().launches_forward == 3
+    assert plan.info().launches_forward == 5
     z = lambda *s, dt=torch.bfloat16: torch.zeros(*s, dtype=dt, device="cuda")
     q, out = z(MAX_T, HQ, D), z(MAX_T, HQ, D)
     k_new, v_new = z(MAX_T, HKV, D), z(MAX_T, HKV, D)
@@ -148,8 +151,9 @@ def test_e4m3_device_plan_graph_replays_decode_batches():
         api.rpa_forward_kv8(plan, q, k_new, v_new, kp, vp, ks, vs, bt, cu, kv, 1.0 / D ** 0.5,
                             out, lse, ws)
 
-    batches = [([40, 700, 1, 3000, 129, 64], [1] * 6, 301), ([2, 90, 1500, 33, 4000, 10],
-                                                             [2, 1, 2, 1, 2, 1], 302)]
+    batches = [([40, 700, 1, 3000, 129, 64], [1] * 6, 301),
+               ([2, 90, 1500, 33, 4000, 10], [2, 1, 2, 1, 2, 1], 302),
+               ([300, 40, 1, 2100, 1, 900], [300, 1, 1, 500, 1, 64], 303)]
     first = True
     graph = None
     for kv_lens, q_lens, seed in batches:
@@ -172,15 +176,7 @@ def test_e4m3_device_plan_graph_replays_decode_batches():
             b8.block_table, b8.cu_seqlens_q, b8.seq_lens_k, scale=1.0 / D ** 0.5, causal=True,
             page_size=P, layout=wl.SEQ_MAJOR)
         assert np.array_equal(kp.cpu().numpy(), kp_ref) and np.array_equal(vp.cpu().numpy(), vp_ref)
-        got = out[:T].cpu().double().numpy()
-        bound = 2.0 ** -8 * 448.0 * float(v_scale.max()) + 2.0 ** -8 * np.abs(ref)
-        assert np.all(np.abs(got - ref) <= bound)
+        vmax = kv8_vmax(vp_ref, v_scale.numpy(), b8.block_table, wl.SEQ_MAJOR)
+        assert_kv8_close(out[:T].cpu(), ref, vmax)
         assert_lse_close(lse[:T].cpu(), ref_lse)
-    # a row too long for the decode kernel is refused (limits bit) instead of computed
-    b = _batch([300, 40, 1, 1, 1, 1], [300, 1, 1, 1, 1, 1], 303)
-    b8, k_scale, v_scale = wl.with_kv8_pools(b, seed=304)
-    load(b8, k_scale, v_scale)
-    graph.replay()
-    torch.cuda.synchronize()
-    assert api.rpa_device_error(clear=True) & 16
     del graph

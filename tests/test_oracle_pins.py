@@ -592,6 +592,46 @@ def test_kv8_attention_equals_bf16_attention_on_shared_values(layout):
     assert np.array_equal(got_o, ref_o) and np.array_equal(got_l, ref_l)
 
 
+def test_kv8_attention_with_group_tables_equals_bf16_on_shared_values():
+    # the e4m3 step restricted to a group table's blocks: the same numbers as the bf16
+    # oracle with that table on the same (exactly shared) values, and not the dense result
+    b = wl.to_head_major(wl.ragged_batch([600, 300], [100, 40], 8, 2, 128, 16, seed=85))
+    b8, _, _ = wl.with_kv8_pools(b, seed=86)
+    ks = np.array([2.0 ** -4, 2.0 ** -6], dtype=np.float32)
+    vs = np.array([2.0 ** -1, 2.0 ** 0], dtype=np.float32)
+    nqb, nkb = -(-100 // 16), b8.max_blocks
+    # a group table is the union over its heads and query blocks: a low density keeps it sparse
+    mask = wl.iid_block_mask(2, 8, nqb, nkb, seed=87, density=0.01)
+    table, count = orc.build_group_tables(mask, 2)
+    kp8, vp8 = orc.codes8(b8.k_pool), orc.codes8(b8.v_pool)
+    got_o, got_l, kpa, vpa = orc.forward_kv8(b8.q, b8.k_new, b8.v_new, kp8, vp8, ks, vs,
+                                             b8.block_table, b8.cu_seqlens_q, b8.seq_lens_k,
+                                             scale=b8.scale, causal=True, page_size=16,
+                                             layout=orc.HEAD_MAJOR, group_table=table,
+                                             group_count=count)
+    heads = np.zeros(kpa.shape[0], dtype=np.int64)
+    bt = orc.ints(b8.block_table)
+    for h in range(2):
+        heads[bt[:, h, :].reshape(-1)] = h
+
+    def to_bf16(codes, scales):
+        v = orc.e4m3_decode(codes) * scales[heads].reshape(-1, 1, 1)
+        return orc.round_bf16(np.where(np.isnan(v), 0.0, v))
+
+    ref_o, ref_l = orc.attention(b8.q, to_bf16(kpa, ks), to_bf16(vpa, vs), b8.block_table,
+                                 b8.cu_seqlens_q, b8.seq_lens_k, scale=b8.scale, causal=True,
+                                 page_size=16, layout=orc.HEAD_MAJOR, num_kv_heads=2,
+                                 group_table=table, group_count=count)
+    assert np.array_equal(got_o, ref_o, equal_nan=True) and np.array_equal(got_l, ref_l,
+                                                                           equal_nan=True)
+    dense_o, _, _, _ = orc.forward_kv8(b8.q, b8.k_new, b8.v_new, kp8, vp8, ks, vs,
+                                       b8.block_table, b8.cu_seqlens_q, b8.seq_lens_k,
+                                       scale=b8.scale, causal=True, page_size=16,
+                                       layout=orc.HEAD_MAJOR)
+    fin = np.isfinite(got_o)
+    assert fin.any() and not np.allclose(got_o[fin], dense_o[fin])
+
+
 def test_write_kv8_places_quantised_codes_in_hand_derived_slots():
     b = wl.ragged_batch([5, 19], [2, 3], 4, 2, 128, 16, seed=83)
     b8, ks, vs = wl.with_kv8_pools(b, seed=84)
