@@ -875,6 +875,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         const bool write = q_local < tile.q_len;
         uint16_t* orow = p.out + ((size_t)t * Hq + hq) * D;
         const float inv = l > 0.f ? (p.v_scale ? __ldg(p.v_scale + h) : 1.f) / l : 0.f;
+        // a thread writes its own row: each store instruction of the warp touches 32 rows, so
+        // the widest store (32 bytes, when the output is 32-byte aligned) halves the count
+        const bool wide = (reinterpret_cast<uintptr_t>(p.out) & 31) == 0;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
           uint32_t o[32];
@@ -886,14 +889,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < 32; ++i) o[i] = 0u;
           }
           if (write) {
+            uint32_t w[16];
 #pragma unroll
-            for (int i = 0; i < 32; i += 8) {
-              U4 v;
-              v.x = pack_bf16(__uint_as_float(o[i + 0]) * inv, __uint_as_float(o[i + 1]) * inv);
-              v.y = pack_bf16(__uint_as_float(o[i + 2]) * inv, __uint_as_float(o[i + 3]) * inv);
-              v.z = pack_bf16(__uint_as_float(o[i + 4]) * inv, __uint_as_float(o[i + 5]) * inv);
-              v.w = pack_bf16(__uint_as_float(o[i + 6]) * inv, __uint_as_float(o[i + 7]) * inv);
-              *reinterpret_cast<U4*>(orow + c * 32 + i) = v;
+            for (int i = 0; i < 16; ++i)
+              w[i] = pack_bf16(__uint_as_float(o[2 * i]) * inv, __uint_as_float(o[2 * i + 1]) * inv);
+            if (wide) {
+              st_global_v8(orow + c * 32, w);
+              st_global_v8(orow + c * 32 + 16, w + 8);
+            } else {
+#pragma unroll
+              for (int i = 0; i < 16; i += 4)
+                *reinterpret_cast<U4*>(orow + c * 32 + 2 * i) = U4{w[i], w[i + 1], w[i + 2], w[i + 3]};
             }
           }
         }

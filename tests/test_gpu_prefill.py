@@ -164,6 +164,33 @@ def test_prefill_large_scores_move_the_reference_max(scale):
     assert_lse_close(lse, ref_lse)
 
 
+@pytest.mark.parametrize("D", [64, 128])
+def test_prefill_output_only_16_byte_aligned(D):
+    # The epilogue writes 32 bytes per store when the output is 32-byte aligned and 16 bytes
+    # otherwise; an output 16 bytes past an aligned base takes the narrow stores and must
+    # give the same bits.
+    b = wl.ragged_batch([700, 300], [500, 300], 8, 2, D, 64, seed=59)
+    plan = plan_for(b)
+    d = to_device(b)
+    T, Hq = b.num_tokens, b.num_q_heads
+    ws = torch.empty(max(plan.workspace_bytes, 256), dtype=torch.uint8, device="cuda")
+    outs = []
+    for shift in (0, 8):  # elements: 0 and 16 bytes
+        base = torch.full((T * Hq * D + 16,), float("nan"), dtype=torch.bfloat16, device="cuda")
+        out = base[shift:shift + T * Hq * D].view(T, Hq, D)
+        assert (out.data_ptr() % 32 == 0) == (shift == 0)
+        api.rpa_forward(plan, d["q"], d["k_new"], d["v_new"], d["k_pool"], d["v_pool"],
+                        d["block_table"], d["cu_seqlens_q"], d["seq_lens_k"], None, None,
+                        b.scale, out, None, ws)
+        torch.cuda.synchronize()
+        assert api.rpa_device_error(clear=True) == 0
+        outs.append(out.cpu())
+    assert plan.info().num_prefill_tiles > 0
+    assert torch.equal(outs[0], outs[1])
+    ref, _, _, _ = oracle_forward(b)
+    assert_close(outs[1], ref)
+
+
 def test_prefill_page_permutation_gives_identical_output():
     b = wl.ragged_batch([500, 260], [300, 260], 8, 2, 128, 16, seed=58)
     o1 = run_forward(b)[0]
