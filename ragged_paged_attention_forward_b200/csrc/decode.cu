@@ -86,9 +86,15 @@ __global__ void __launch_bounds__(kDecodeThreads, 1)
 
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
-  if (p.count && (int)blockIdx.x >= __ldg(p.count)) return;  // device-planned: unused CTA
-  const DecodeItem it = p.items ? p.items[blockIdx.x] : inl.v[blockIdx.x];
-  const int h = blockIdx.y;
+  // The grid is (KV heads, items), so that the CTAs of one item's KV heads start together and
+  // read whole rows of sequence-major pages at once, or (items, KV heads) when the items pass
+  // grid y's limit.  A square grid is read as the former: both readings visit every
+  // (item, head) pair once.
+  const bool heads_fast = (int)gridDim.x == p.num_kv_heads;
+  const int item_idx = heads_fast ? (int)blockIdx.y : (int)blockIdx.x;
+  if (p.count && item_idx >= __ldg(p.count)) return;  // device-planned: unused CTA
+  const DecodeItem it = p.items ? p.items[item_idx] : inl.v[item_idx];
+  const int h = heads_fast ? (int)blockIdx.x : (int)blockIdx.y;
   const int Hq = p.num_q_heads;
   const int G = Hq / p.num_kv_heads;
   const int rows = it.q_len * G;
@@ -534,7 +540,8 @@ cudaError_t launch_decode_t(const DecodeLaunch& p, const DecodeItemsInline* inl,
   auto kern = decode_split_kernel<D, NT, KV8>;
   e = ensure_smem_attr(reinterpret_cast<const void*>(kern), Geo::kAlloc);
   if (e != cudaSuccess) return e;
-  dim3 grid(p.num_items, p.num_kv_heads);
+  const dim3 grid = p.num_items <= 65535 ? dim3(p.num_kv_heads, p.num_items)
+                                         : dim3(p.num_items, p.num_kv_heads);
   kern<<<grid, kDecodeThreads, Geo::kAlloc, stream>>>(kmap, vmap, p, *inl);
   return cudaGetLastError();
 }
